@@ -1,0 +1,209 @@
+"""ctypes front end of the CPU oracle (``ssa_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this module.  The library path never does,
+and nothing here imports the library: the two share only the seeded input generator.
+
+Every function mirrors one C routine and cites the same passages as the C source
+(the DAM review page, "What carries the argument", "Circularity Check", Referee
+Report minor comment 1).
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "ssa_oracle.c")
+LIB = os.path.join(HERE, "libssa_oracle.so")
+
+TILE = 128  # tile edge of the canonical plan
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (fp64, OpenMP, no FMA contraction)."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", "-std=c11", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+                        "-fPIC", "-shared", "-o", tmp, SRC, "-lm"], check=True)
+        os.replace(tmp, LIB)
+    return LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = C.CDLL(build())
+        _setup(_lib)
+    return _lib
+
+
+P = C.c_void_p
+
+
+def _setup(L):
+    L.ora_true_mask.argtypes = [P, C.c_int, C.c_double, C.c_double, C.c_double, P]
+    L.ora_gamma.argtypes = [P, C.c_int, P, P]
+    L.ora_select.argtypes = [P, P, C.c_int, C.c_double, P, P, P, P]
+    L.ora_capture.argtypes = [P, C.c_int, C.c_int, C.c_double, C.c_double, C.c_double, C.c_double,
+                              P, P, P, P]
+    L.ora_extend.argtypes = [C.c_int, P, P, P, P, C.c_int, P, P, P, P]
+    for name in ("ora_plan_brute", "ora_plan_interval"):
+        f = getattr(L, name)
+        f.argtypes = [C.c_int, P, P, P, P, C.c_int, C.c_longlong, P, P, P, P, P, P]
+        f.restype = C.c_longlong
+    L.ora_attn_rows.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int, P, P, P, P, P,
+                                C.c_double, C.c_int, P, P, P]
+    L.ora_attn_dense.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int, P, P, P, P, P,
+                                 C.c_double, P, P]
+    L.ora_nnz.argtypes = [C.c_int, P, P, P, P, C.c_int, P]
+    for name in ("ora_true_mask", "ora_gamma", "ora_select", "ora_capture", "ora_extend",
+                 "ora_attn_rows", "ora_attn_dense", "ora_nnz"):
+        getattr(L, name).restype = C.c_int
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _check(rc, what):
+    if rc < 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+    return rc
+
+
+# ------------------------------------------------------------------------------------
+# Stage one
+# ------------------------------------------------------------------------------------
+
+def true_mask(amap, lam=0.5, eps=1e-8, tau=0.3):
+    """Binary true mask uint8 [L, L] of one averaged map (row min-max of Box-Cox, t >= tau)."""
+    amap = _c(amap, np.float32)
+    Ln = amap.shape[0]
+    M = np.zeros((Ln, Ln), np.uint8)
+    _check(lib().ora_true_mask(_p(amap), Ln, lam, eps, tau, _p(M)), "true_mask")
+    return M
+
+
+def gamma(M):
+    """gamma_k for every diagonal r and vertical c of a binary mask."""
+    M = _c(M, np.uint8)
+    Ln = M.shape[0]
+    gd = np.zeros(Ln, np.float64)
+    gv = np.zeros(Ln, np.float64)
+    _check(lib().ora_gamma(_p(M), Ln, _p(gd), _p(gv)), "gamma")
+    return gd, gv
+
+
+def select(gd, gv, mu=0.8):
+    gd = _c(gd, np.float64)
+    gv = _c(gv, np.float64)
+    Ln = gd.shape[0]
+    do = np.zeros(Ln, np.int32)
+    vo = np.zeros(Ln, np.int32)
+    nd = np.zeros(1, np.int32)
+    nv = np.zeros(1, np.int32)
+    _check(lib().ora_select(_p(gd), _p(gv), Ln, mu, _p(do), _p(nd), _p(vo), _p(nv)), "select")
+    return do[:nd[0]].copy(), vo[:nv[0]].copy()
+
+
+def capture(maps, lam=0.5, tau=0.3, mu=0.8, eps=1e-8):
+    """Whole stage one over maps [n, L, L]; returns CSR (diag_ptr, diag_offsets, vert_ptr, vert_cols)."""
+    maps = _c(maps, np.float32)
+    n, Ln, _ = maps.shape
+    dp = np.zeros(n + 1, np.int32)
+    do = np.zeros(n * Ln + 1, np.int32)
+    vp = np.zeros(n + 1, np.int32)
+    vo = np.zeros(n * Ln + 1, np.int32)
+    _check(lib().ora_capture(_p(maps), n, Ln, lam, tau, mu, eps, _p(dp), _p(do), _p(vp), _p(vo)),
+           "capture")
+    return dp, do[:dp[-1]].copy(), vp, vo[:vp[-1]].copy()
+
+
+# ------------------------------------------------------------------------------------
+# Stage two
+# ------------------------------------------------------------------------------------
+
+def extend(diag_ptr, diag_offsets, vert_ptr, vert_cols, S):
+    dp, do, vp, vo = (_c(a, np.int32) for a in (diag_ptr, diag_offsets, vert_ptr, vert_cols))
+    H = len(dp) - 1
+    edp = np.zeros(H + 1, np.int32)
+    edo = np.zeros(max(len(do), 1), np.int32)
+    evp = np.zeros(H + 1, np.int32)
+    evo = np.zeros(max(len(vo), 1), np.int32)
+    _check(lib().ora_extend(H, _p(dp), _p(do), _p(vp), _p(vo), S, _p(edp), _p(edo), _p(evp), _p(evo)),
+           "extend")
+    return edp, edo[:edp[-1]].copy(), evp, evo[:evp[-1]].copy()
+
+
+def plan(ext, S, routine="brute"):
+    """Canonical tile plan as a dict of numpy arrays (routine: 'brute' or 'interval')."""
+    dp, do, vp, vo = (_c(a, np.int32) for a in ext)
+    H = len(dp) - 1
+    nqb = (S + TILE - 1) // TILE
+    f = getattr(lib(), "ora_plan_" + routine)
+    n = _check(f(H, _p(dp), _p(do), _p(vp), _p(vo), S, 0, None, None, None, None, None, None), "plan")
+    out = dict(tile_ptr=np.zeros(H * nqb + 1, np.int32), tile_kb=np.zeros(max(n, 1), np.int32),
+               tile_dmask=np.zeros((max(n, 1), 4), np.uint64), tile_cmask=np.zeros((max(n, 1), 2), np.uint64),
+               tile_flags=np.zeros(max(n, 1), np.uint32), stripe_cnt=np.zeros(H * nqb, np.int32))
+    n2 = _check(f(H, _p(dp), _p(do), _p(vp), _p(vo), S, n, _p(out["tile_ptr"]), _p(out["tile_kb"]),
+                  _p(out["tile_dmask"]), _p(out["tile_cmask"]), _p(out["tile_flags"]),
+                  _p(out["stripe_cnt"])), "plan")
+    assert n2 == n
+    for k in ("tile_kb", "tile_dmask", "tile_cmask", "tile_flags"):
+        out[k] = out[k][:n].copy()
+    out["n_tiles"] = n
+    out["nqb"] = nqb
+    return out
+
+
+def nnz(ext, S):
+    dp, do, vp, vo = (_c(a, np.int32) for a in ext)
+    H = len(dp) - 1
+    out = np.zeros(H, np.int64)
+    _check(lib().ora_nnz(H, _p(dp), _p(do), _p(vp), _p(vo), S, _p(out)), "nnz")
+    return out
+
+
+# ------------------------------------------------------------------------------------
+# Attention
+# ------------------------------------------------------------------------------------
+
+def attn_rows(q, k, v, ext, scale, rows, kv_map=None):
+    """List-driven fp64 attention for the given rows.  q/k/v: bf16 bits uint16 [H,S,d]."""
+    q, k, v = (_c(a, np.uint16) for a in (q, k, v))
+    Hq, S, d = q.shape
+    Hkv = k.shape[0]
+    dp, do, vp, vo = (_c(a, np.int32) for a in ext)
+    rows = _c(rows, np.int32)
+    km = None if kv_map is None else _c(kv_map, np.int32)
+    O = np.zeros((Hq, len(rows), d), np.float64)
+    LSE = np.zeros((Hq, len(rows)), np.float64)
+    _check(lib().ora_attn_rows(_p(q), _p(k), _p(v), Hq, Hkv, S, d, _p(dp), _p(do), _p(vp), _p(vo),
+                               _p(km), scale, len(rows), _p(rows), _p(O), _p(LSE)), "attn_rows")
+    return O, LSE
+
+
+def attn_dense(q, k, v, ext, scale, kv_map=None):
+    """Dense-mask fp64 attention over every row (S <= 8192)."""
+    q, k, v = (_c(a, np.uint16) for a in (q, k, v))
+    Hq, S, d = q.shape
+    Hkv = k.shape[0]
+    dp, do, vp, vo = (_c(a, np.int32) for a in ext)
+    km = None if kv_map is None else _c(kv_map, np.int32)
+    O = np.zeros((Hq, S, d), np.float64)
+    LSE = np.zeros((Hq, S), np.float64)
+    _check(lib().ora_attn_dense(_p(q), _p(k), _p(v), Hq, Hkv, S, d, _p(dp), _p(do), _p(vp), _p(vo),
+                                _p(km), scale, _p(O), _p(LSE)), "attn_dense")
+    return O, LSE

@@ -1,0 +1,154 @@
+"""Pins for the oracle's extension and canonical tile plan.
+
+Extension: the extended mask is the union of the kept patterns over the S x S causal
+square (DAM review page, "What carries the argument" and "Circularity Check" step 1),
+i.e. diagonals r < S and columns c < S.  The tile plan is this library's own data
+structure; its two oracle routines (brute force and interval arithmetic) must agree,
+and the element counts it implies must equal the retained pairs counted by brute
+force over the dense mask.
+"""
+
+import numpy as np
+import pytest
+
+from structured_sparse_attention_b200 import inputs
+
+T = 128
+
+
+def _ext(ora, diags, verts, S):
+    dp, do = inputs.to_csr(diags)
+    vp, vo = inputs.to_csr(verts)
+    return ora.extend(dp, do, vp, vo, S)
+
+
+def _dense_mask(diags, verts, h, S):
+    M = np.zeros((S, S), bool)
+    for r in diags[h]:
+        if r < S:
+            idx = np.arange(r, S)
+            M[idx, idx - r] = True
+    for c in verts[h]:
+        if c < S:
+            M[c:, c] = True
+    return M
+
+
+def _active_count_from_plan(plan, ext, h, S):
+    """Count retained pairs implied by the plan: band elements of listed tiles
+    (dmask & ~cmask & i < S) plus stripe elements (C_h[k] <= i)."""
+    nqb = plan["nqb"]
+    C = ext[3][ext[2][h]:ext[2][h + 1]]
+    total = 0
+    for qb in range(nqb):
+        a, b = plan["tile_ptr"][h * nqb + qb], plan["tile_ptr"][h * nqb + qb + 1]
+        for t in range(a, b):
+            dm = plan["tile_dmask"][t]
+            cm = plan["tile_cmask"][t]
+            for il in range(T):
+                i = T * qb + il
+                if i >= S:
+                    break
+                for jl in range(T):
+                    tb = il - jl + T - 1
+                    if (int(dm[tb >> 6]) >> (tb & 63)) & 1 and not (int(cm[jl >> 6]) >> (jl & 63)) & 1:
+                        total += 1
+        for il in range(T):
+            i = T * qb + il
+            if i >= S:
+                break
+            total += int(np.sum(C[:plan["stripe_cnt"][h * nqb + qb]] <= i))
+    return total
+
+
+def test_extend_filters_and_validates(ora):
+    diags = [np.array([0, 3, 9, 16, 20], np.int32), np.array([], np.int32)]
+    verts = [np.array([1, 10, 16], np.int32), np.array([0, 15, 16], np.int32)]
+    edp, edo, evp, evo = _ext(ora, diags, verts, 16)
+    assert edo[edp[0]:edp[1]].tolist() == [0, 3, 9]
+    assert edo[edp[1]:edp[2]].tolist() == []
+    assert evo[evp[0]:evp[1]].tolist() == [1, 10]
+    assert evo[evp[1]:evp[2]].tolist() == [0, 15]
+    with pytest.raises(RuntimeError):
+        _ext(ora, [np.array([3, 3], np.int32)], [np.array([], np.int32)], 16)
+    with pytest.raises(RuntimeError):
+        _ext(ora, [np.array([5, 2], np.int32)], [np.array([], np.int32)], 16)
+    with pytest.raises(RuntimeError):
+        _ext(ora, [np.array([-1], np.int32)], [np.array([], np.int32)], 16)
+
+
+def test_plan_main_diagonal_only(ora):
+    # D = {0}: each query block has exactly its own diagonal tile, holding only the
+    # local diagonal t = 127; never FULL; no stripes.
+    for S in (256, 300):
+        ext = _ext(ora, [np.array([0], np.int32)], [np.array([], np.int32)], S)
+        p = ora.plan(ext, S)
+        nqb = (S + T - 1) // T
+        assert p["n_tiles"] == nqb
+        assert p["tile_kb"].tolist() == list(range(nqb))
+        for t in range(nqb):
+            assert p["tile_dmask"][t].tolist() == [0, 1 << 63, 0, 0]
+            assert p["tile_cmask"][t].tolist() == [0, 0]
+            assert p["tile_flags"][t] == 0
+        assert not p["stripe_cnt"].any()
+
+
+def test_plan_full_causal(ora):
+    S = 512
+    ext = _ext(ora, [np.arange(S, dtype=np.int32)], [np.array([], np.int32)], S)
+    p = ora.plan(ext, S)
+    assert p["n_tiles"] == 4 * 5 // 2
+    for qb in range(4):
+        a, b = p["tile_ptr"][qb], p["tile_ptr"][qb + 1]
+        assert p["tile_kb"][a:b].tolist() == list(range(qb + 1))
+        for t in range(a, b):
+            kb = p["tile_kb"][t]
+            assert p["tile_flags"][t] == (1 if kb < qb else 0)
+            if kb == qb:
+                # only r >= 0, i.e. t >= 127
+                assert p["tile_dmask"][t].tolist() == [0, 0xFFFFFFFFFFFFFFFF << 63 & 0xFFFFFFFFFFFFFFFF,
+                                                       0xFFFFFFFFFFFFFFFF, 0x7FFFFFFFFFFFFFFF]
+
+
+def test_plan_column_owned_by_stripes(ora):
+    # D = {128}, C = {0..127}: every band element of tile (qb=1, kb=0) sits in a column
+    # of C, so the tile is not listed; the stripe phase owns those pairs.
+    S = 256
+    ext = _ext(ora, [np.array([128], np.int32)], [np.arange(128, dtype=np.int32)], S)
+    p = ora.plan(ext, S)
+    assert p["n_tiles"] == 0
+    assert p["stripe_cnt"].tolist() == [128, 128]
+    # one excluded column stops a tile from being FULL but keeps it listed
+    ext = _ext(ora, [np.arange(S, dtype=np.int32)], [np.array([5], np.int32)], S)
+    p = ora.plan(ext, S)
+    t = p["tile_ptr"][1]
+    assert p["tile_kb"][t] == 0 and p["tile_flags"][t] == 0
+    assert p["tile_cmask"][t].tolist() == [1 << 5, 0]
+
+
+def test_plan_ragged_tail_is_not_full(ora):
+    S = 200  # second block has 72 rows
+    ext = _ext(ora, [np.arange(S, dtype=np.int32)], [np.array([], np.int32)], S)
+    p = ora.plan(ext, S)
+    a, b = p["tile_ptr"][1], p["tile_ptr"][2]
+    assert p["tile_kb"][a:b].tolist() == [0, 1]
+    assert p["tile_flags"][a:b].tolist() == [0, 0]
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_plan_routines_agree_and_count_pairs(ora, seed):
+    g = np.random.default_rng(seed)
+    S = int(g.integers(1, 700))
+    H = 3
+    diags, verts = inputs.random_patterns(1000 + seed, H, S, max_diag=min(S, 200), max_vert=min(S, 40))
+    ext = _ext(ora, diags, verts, S)
+    pb = ora.plan(ext, S, "brute")
+    pi = ora.plan(ext, S, "interval")
+    for k in ("tile_ptr", "tile_kb", "tile_dmask", "tile_cmask", "tile_flags", "stripe_cnt"):
+        np.testing.assert_array_equal(pb[k], pi[k], err_msg=k)
+    nnz = ora.nnz(ext, S)
+    for h in range(H):
+        dense = int(_dense_mask(diags, verts, h, S).sum())
+        assert nnz[h] == dense
+        if S <= 400:
+            assert _active_count_from_plan(pb, ext, h, S) == dense
