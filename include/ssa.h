@@ -1,0 +1,230 @@
+/*
+ * ssa.h -- C ABI of libssa: DAM structured sparse attention on one B200 (sm_100a).
+ *
+ * The method is the Dynamic Attention Mask of the DAM review page ("DAM: Dynamic
+ * Attention Mask for Long-Context Large Language Model Inference Acceleration",
+ * pith review of arXiv 2506.11104):
+ *   stage one  ("What carries the argument"): averaged L x L attention maps ->
+ *              Box-Cox (lambda) -> threshold tau -> binary true mask M -> score every
+ *              diagonal (j = i - r) and vertical (j = c, i >= c) candidate by
+ *              gamma_k = sum(M P_k) / sum(P_k) -> keep gamma_k >= mu;
+ *   stage two  ("What carries the argument"; "Circularity Check", steps 1 and 2;
+ *              Referee Report summary): the kept patterns, pasted over S x S, form
+ *              the extended mask applied to QK^T / sqrt(d_k) before the softmax.
+ *
+ * Conventions shared by every call
+ *   - Every call returns an int status (SSA_OK or a negative SSA_ERR_* code) and
+ *     records a message retrievable with ssa_last_error() (thread-local).
+ *   - The caller owns all memory.  Every pointer argument named as "device" must
+ *     point to CUDA device memory of the current device; "host" pointers to host
+ *     memory.  The library allocates and frees nothing and never synchronises the
+ *     stream, except where a call says so.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     All work of a call is enqueued on it, in order.
+ *   - `dev_status` (device, one int32, may be NULL) receives faults detected on the
+ *     GPU: the first non-zero SSA_ERR_* code written by any kernel stays.  The caller
+ *     zeroes it and reads it after synchronising.  Kernels never trap: on a bad index
+ *     or an expired bounded wait they record the code and return.
+ *   - bf16 tensors are passed as raw 16-bit storage (uint16_t / void*).
+ */
+#ifndef SSA_H
+#define SSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SSA_API __attribute__((visibility("default")))
+#else
+#define SSA_API
+#endif
+
+#define SSA_OK 0
+#define SSA_ERR_INVALID (-1)     /* null pointer, bad size, unsorted/duplicate/negative list, bad map entry */
+#define SSA_ERR_UNSUPPORTED (-2) /* head dim not 64/128, lambda not 0.5/1, L > 1024 */
+#define SSA_ERR_CAPACITY (-3)    /* caller buffer or workspace too small */
+#define SSA_ERR_CUDA (-4)        /* a CUDA runtime/driver call failed */
+#define SSA_ERR_TIMEOUT (-5)     /* a bounded on-device wait expired */
+
+/* Tile edge of the query blocks and key tiles used by the plan and the kernels. */
+#define SSA_BLOCK 128
+
+/* ------------------------------------------------------------------------------ */
+/* Stage one: pattern capture                                                      */
+/* ------------------------------------------------------------------------------ */
+
+/* Workspace bytes sparse_pattern_capture needs for n_maps maps of size L x L. */
+SSA_API size_t sparse_pattern_capture_ws_bytes(int n_maps, int L);
+
+/*
+ * sparse_pattern_capture -- stage one of DAM ("What carries the argument"; lambda,
+ * tau, mu from "Assumptions & free parameters"; eps from Referee Report minor
+ * comment 1).
+ *
+ * For every map m and row i (causal entries j <= i only):
+ *   y_j = ((x_j + eps)^lambda - 1) / lambda                (Box-Cox)
+ *   t_j = (y_j - y_min) / (y_max - y_min)  (row min/max; t = 1 on a constant row)
+ *   M[i][j] = t_j >= tau
+ * then gamma_diag[r] = #{i >= r : M[i][i-r]} / (L - r), gamma_vert[c] =
+ * #{i >= c : M[i][c]} / (L - c), both in fp64, and r (resp. c) is kept iff
+ * gamma >= mu.  Every threshold decision is made with correctly rounded fp64
+ * arithmetic in the stated order, so the kept lists are exactly reproducible.
+ *
+ *   maps         device, float32 [n_maps][L][L] row-major, already averaged over the
+ *                calibration batches; causal entries must be finite and >= 0
+ *                (entries j > i are ignored)
+ *   n_maps       >= 1;  L in [1, 1024]
+ *   lambda       0.5 or 1.0 (else SSA_ERR_UNSUPPORTED); tau, mu in fp64; eps >= 0
+ *   diag_ptr     device int32 [n_maps + 1]   CSR row pointers of the kept diagonals
+ *   diag_offsets device int32 [n_maps * L]   kept r, ascending within each map
+ *   vert_ptr     device int32 [n_maps + 1]
+ *   vert_cols    device int32 [n_maps * L]   kept c, ascending within each map
+ *   ws           device workspace of at least sparse_pattern_capture_ws_bytes()
+ * A negative or non-finite map entry sets SSA_ERR_INVALID in dev_status; the lists
+ * are then unspecified.
+ */
+SSA_API int sparse_pattern_capture(const float *maps, int n_maps, int L, double lambda, double tau,
+                           double mu, double eps, int32_t *diag_ptr, int32_t *diag_offsets,
+                           int32_t *vert_ptr, int32_t *vert_cols, void *ws, size_t ws_bytes,
+                           int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------------ */
+/* Stage two: extension to S and the tile plan                                     */
+/* ------------------------------------------------------------------------------ */
+
+/* Sizes of a plan, filled by the sizing pass of sparse_pattern_extend. */
+typedef struct ssa_plan_sizes {
+    int32_t n_heads;
+    int32_t S;
+    int32_t nqb;       /* ceil(S / 128) */
+    int32_t n_diag;    /* total extended diagonals over all heads */
+    int32_t n_vert;    /* total extended columns over all heads */
+    int32_t max_vert;  /* max over heads of the extended column count */
+    int64_t n_tiles;   /* total listed band tiles */
+} ssa_plan_sizes;
+
+/*
+ * A compiled plan.  The struct itself is host memory; every pointer in it is a
+ * device buffer owned by the caller and sized from ssa_plan_sizes:
+ *   ext_diag_ptr [n_heads+1], ext_diag_offsets [max(n_diag,1)],
+ *   ext_vert_ptr [n_heads+1], ext_vert_cols [max(n_vert,1)],
+ *   tile_ptr [n_heads*nqb + 1], tile_kb [max(n_tiles,1)],
+ *   tile_dmask [max(n_tiles,1)][4] (uint64), tile_cmask [max(n_tiles,1)][2] (uint64),
+ *   tile_flags [max(n_tiles,1)], stripe_cnt [n_heads*nqb].
+ * Tile semantics, for head h, query block qb (rows 128qb..128qb+127), key tile kb:
+ *   dmask bit t (0..254) set  iff  r = 128(qb-kb) + t - 127 is an extended diagonal
+ *   cmask bit jl (0..127) set iff  column 128kb + jl is an extended column
+ *   a tile is listed, in ascending kb, iff some (i, j) in it has i < S, j <= i,
+ *   i - j a diagonal and j not a column; tile_flags bit 0 (FULL) iff kb < qb,
+ *   128(qb+1) <= S, all 255 dmask bits set and cmask == 0;
+ *   stripe_cnt[h*nqb+qb] = #{extended columns c <= min(S-1, 128qb+127)}.
+ * Columns are owned by the stripe phase only, so each retained pair is used once.
+ */
+typedef struct ssa_plan {
+    int32_t n_heads;
+    int32_t S;
+    int32_t nqb;
+    int32_t max_vert;
+    int64_t n_tiles; /* capacity of the tile arrays (from ssa_plan_sizes) */
+    int32_t *ext_diag_ptr;
+    int32_t *ext_diag_offsets;
+    int32_t *ext_vert_ptr;
+    int32_t *ext_vert_cols;
+    int32_t *tile_ptr;
+    int32_t *tile_kb;
+    uint64_t *tile_dmask;
+    uint64_t *tile_cmask;
+    uint32_t *tile_flags;
+    int32_t *stripe_cnt;
+} ssa_plan;
+
+/* Workspace bytes of either pass of sparse_pattern_extend. */
+SSA_API size_t sparse_pattern_extend_ws_bytes(int n_heads, int S);
+
+/*
+ * sparse_pattern_extend -- stage two of DAM ("What carries the argument": the kept
+ * patterns are pasted into an S x S mask; "Circularity Check" step 1: that mask is
+ * the union of the matched patterns).  The extended lists keep every diagonal r < S
+ * and column c < S of each head; the plan then lists, per query block, the key tiles
+ * the band touches.
+ *
+ *   n_heads, S   >= 1
+ *   diag_ptr, diag_offsets, vert_ptr, vert_cols
+ *                device CSR lists per head (e.g. the output of capture); each list
+ *                strictly ascending and >= 0, else SSA_ERR_INVALID
+ *   sizes        host, always filled when plan == NULL (sizing pass)
+ *   plan         NULL: sizing pass -- enqueues the counting kernels, copies the
+ *                totals to the host and SYNCHRONISES `stream`; returns
+ *                SSA_ERR_INVALID if a list is malformed.
+ *                non-NULL: fill pass -- writes every plan array (no synchronisation);
+ *                plan->n_tiles must be >= the sized n_tiles (else SSA_ERR_CAPACITY in
+ *                dev_status); plan->n_heads/S/nqb/max_vert must match the sizes.
+ *   ws           device workspace of at least sparse_pattern_extend_ws_bytes()
+ */
+SSA_API int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offsets,
+                          const int32_t *vert_ptr, const int32_t *vert_cols, int S,
+                          ssa_plan_sizes *sizes, const ssa_plan *plan, void *ws, size_t ws_bytes,
+                          int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------------ */
+/* Attention forward                                                               */
+/* ------------------------------------------------------------------------------ */
+
+/* Workspace bytes of sparse_attn_fwd (the gathered stripe keys and values). */
+SSA_API size_t sparse_attn_fwd_ws_bytes(int n_heads, int max_vert, int d);
+
+/*
+ * sparse_attn_fwd -- causal prefill attention restricted to the extended mask
+ * (Referee Report summary and "Circularity Check" step 2: the mask is applied to
+ * QK^T / sqrt(d_k) before the softmax; "What carries the argument": only the
+ * retained connections are computed).  For head h, KV head g = kv_map[h] (or
+ * h / (H_q/H_kv) when kv_map is NULL) and query i < S, with retained keys
+ * J_i = {i - r : r in D_h, r <= i} U {c in C_h : c <= i}:
+ *   O[h][i]   = sum_{j in J_i} softmax_j(scale * q_i . k_j) v_j
+ *   LSE[h][i] = log sum_{j in J_i} exp(scale * q_i . k_j)     (natural log)
+ * An empty J_i gives O = 0 and LSE = -inf.  bf16 inputs, fp32 accumulation, bf16 O.
+ *
+ *   Q, O         device bf16 [H_q][S][d], contiguous
+ *   K, V         device bf16 [H_kv][S][d], contiguous
+ *   H_q, H_kv    >= 1; H_q % H_kv == 0 when kv_map is NULL
+ *   S            must equal plan->S;  d in {64, 128} (else SSA_ERR_UNSUPPORTED)
+ *   plan         host struct of device arrays from sparse_pattern_extend, n_heads == H_q
+ *   kv_map       device int32 [H_q] or NULL; entries outside [0, H_kv) set
+ *                SSA_ERR_INVALID in dev_status
+ *   scale        softmax scale (1/sqrt(d) for the paper's formula)
+ *   LSE          device float32 [H_q][S]
+ *   ws           device workspace of at least sparse_attn_fwd_ws_bytes(H_q, plan->max_vert, d);
+ *                all base pointers must be 16-byte aligned
+ */
+SSA_API int sparse_attn_fwd(const void *Q, const void *K, const void *V, int H_q, int H_kv, int S, int d,
+                    const ssa_plan *plan, const int32_t *kv_map, float scale, void *O, float *LSE,
+                    void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------------ */
+/* Diagnostics                                                                     */
+/* ------------------------------------------------------------------------------ */
+
+/* Message of the last failing call on this thread ("" if none). */
+SSA_API const char *ssa_last_error(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+SSA_API int ssa_version(void);
+
+/*
+ * Time limit, in nanoseconds, of every bounded wait inside the attention kernel
+ * (default 2e9; 0 makes a wait give up at its first unsuccessful poll).  When a wait
+ * expires the kernel writes SSA_ERR_TIMEOUT to dev_status, drains its own copies and
+ * tensor-core work in flight, frees its tensor memory and returns.  Process-wide;
+ * meant for fault-handling tests.  Returns the previous value.
+ */
+SSA_API int64_t ssa_set_wait_limit_ns(int64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSA_H */

@@ -59,6 +59,8 @@ def _setup(L):
         f = getattr(L, name)
         f.argtypes = [C.c_int, P, P, P, P, C.c_int, C.c_longlong, P, P, P, P, P, P]
         f.restype = C.c_longlong
+    L.ora_plan_items.argtypes = [C.c_int, P, P, P, P, C.c_int, C.c_int, P, C.c_longlong, P, P, P, P, P, P]
+    L.ora_plan_items.restype = C.c_longlong
     L.ora_attn_rows.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int, P, P, P, P, P,
                                 C.c_double, C.c_int, P, P, P]
     L.ora_attn_dense.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int, P, P, P, P, P,
@@ -165,6 +167,26 @@ def plan(ext, S, routine="brute"):
         out[k] = out[k][:n].copy()
     out["n_tiles"] = n
     out["nqb"] = nqb
+    return out
+
+
+def plan_items(ext, S, items):
+    """Canonical tiles of selected (head, query block) pairs; items int32 [n, 2]."""
+    dp, do, vp, vo = (_c(a, np.int32) for a in ext)
+    H = len(dp) - 1
+    items = _c(items, np.int32).reshape(-1, 2)
+    ni = len(items)
+    f = lib().ora_plan_items
+    n = _check(f(H, _p(dp), _p(do), _p(vp), _p(vo), S, ni, _p(items), 0, None, None, None, None, None,
+                 None), "plan_items")
+    out = dict(item_ptr=np.zeros(ni + 1, np.int32), tile_kb=np.zeros(max(n, 1), np.int32),
+               tile_dmask=np.zeros((max(n, 1), 4), np.uint64), tile_cmask=np.zeros((max(n, 1), 2), np.uint64),
+               tile_flags=np.zeros(max(n, 1), np.uint32), stripe_cnt=np.zeros(ni, np.int32))
+    _check(f(H, _p(dp), _p(do), _p(vp), _p(vo), S, ni, _p(items), n, _p(out["item_ptr"]), _p(out["tile_kb"]),
+             _p(out["tile_dmask"]), _p(out["tile_cmask"]), _p(out["tile_flags"]), _p(out["stripe_cnt"])),
+           "plan_items")
+    for k in ("tile_kb", "tile_dmask", "tile_cmask", "tile_flags"):
+        out[k] = out[k][:n].copy()
     return out
 
 

@@ -330,10 +330,77 @@ long long ora_plan_brute(int n_heads, const int32_t *ext_diag_ptr, const int32_t
     return n;
 }
 
-/* Routine 2: interval arithmetic over the offsets.  Candidate tiles are those a
- * diagonal r in D_h crosses within the valid rows; dmask/cmask are range queries on
- * the sorted lists; "listed" checks, per set dmask bit, whether the diagonal's cells
- * in valid rows reach a column outside cmask. */
+/* First index k of the ascending array a[0..n) with a[k] >= x. */
+static int first_ge(const int32_t *a, int n, long x) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        int mid = (lo + hi) / 2;
+        if (a[mid] < x) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
+
+/* Routine 2 for one (head, query block): interval arithmetic over the offsets.
+ * Candidate tiles are those a diagonal r in D_h crosses within the valid rows;
+ * dmask / cmask are range queries on the sorted lists; "listed" checks, per set dmask
+ * bit, whether the diagonal's cells in valid rows reach a column outside cmask.
+ * Appends the block's tiles at out index n; returns the new n or a negative error. */
+static long long interval_block(const int32_t *D, int nd, const int32_t *C, int nc, int S, int qb,
+                                uint8_t *cand, long long n, long long capacity, int32_t *tile_kb,
+                                uint64_t *tile_dmask, uint64_t *tile_cmask, uint32_t *tile_flags) {
+    const int T = ORA_TILE;
+    int nqb = (S + T - 1) / T;
+    long lo_i = (long)T * qb;
+    long hi_i = lo_i + T - 1 < S - 1 ? lo_i + T - 1 : S - 1;
+    int nrows = (int)(hi_i - lo_i + 1);
+    memset(cand, 0, (size_t)nqb);
+    for (int k = 0; k < nd; ++k) {
+        long r = D[k];
+        if (r > hi_i) break;
+        long jlo = lo_i - r > 0 ? lo_i - r : 0;
+        long jhi = hi_i - r;
+        for (long kb = jlo / T; kb <= jhi / T; ++kb) cand[kb] = 1;
+    }
+    for (int kb = 0; kb <= qb; ++kb) {
+        if (!cand[kb]) continue;
+        long base = (long)T * (qb - kb) - (T - 1); /* r of dmask bit 0 */
+        uint64_t dm[4] = {0, 0, 0, 0}, cm[2] = {0, 0};
+        for (int k = first_ge(D, nd, base); k < nd && D[k] <= base + 2 * T - 2; ++k)
+            set_bit(dm, (int)(D[k] - base));
+        for (int k = first_ge(C, nc, (long)T * kb); k < nc && C[k] < (long)T * (kb + 1); ++k)
+            set_bit(cm, (int)(C[k] - (long)T * kb));
+        int listed = 0;
+        for (int t = 0; t <= 2 * T - 2 && !listed; ++t) {
+            if (!get_bit(dm, t)) continue;
+            int delta = t - (T - 1); /* il - jl */
+            int il_lo = delta > 0 ? delta : 0;
+            int il_hi = T - 1;
+            if (T - 1 + delta < il_hi) il_hi = T - 1 + delta;
+            if (nrows - 1 < il_hi) il_hi = nrows - 1;
+            for (int il = il_lo; il <= il_hi; ++il) {
+                if (!get_bit(cm, il - delta)) {
+                    listed = 1;
+                    break;
+                }
+            }
+        }
+        if (!listed) continue;
+        int full = (kb < qb) && ((long)T * (qb + 1) <= S) && popcount256(dm) == 2 * T - 1 &&
+                   cm[0] == 0 && cm[1] == 0;
+        if (tile_kb) {
+            if (n >= capacity) return ORA_ERR_CAPACITY;
+            tile_kb[n] = kb;
+            memcpy(tile_dmask + 4 * n, dm, sizeof dm);
+            memcpy(tile_cmask + 2 * n, cm, sizeof cm);
+            tile_flags[n] = full ? 1u : 0u;
+        }
+        ++n;
+    }
+    return n;
+}
+
+/* Routine 2 over every (head, query block); same outputs as routine 1. */
 long long ora_plan_interval(int n_heads, const int32_t *ext_diag_ptr,
                             const int32_t *ext_diag_offsets, const int32_t *ext_vert_ptr,
                             const int32_t *ext_vert_cols, int S, long long capacity,
@@ -345,70 +412,54 @@ long long ora_plan_interval(int n_heads, const int32_t *ext_diag_ptr,
     uint8_t *cand = (uint8_t *)malloc((size_t)nqb);
     if (!cand) return ORA_ERR_NOMEM;
     long long n = 0;
-    for (int h = 0; h < n_heads; ++h) {
+    for (int h = 0; h < n_heads && n >= 0; ++h) {
         const int32_t *D = ext_diag_offsets + ext_diag_ptr[h];
         int nd = ext_diag_ptr[h + 1] - ext_diag_ptr[h];
         const int32_t *C = ext_vert_cols + ext_vert_ptr[h];
         int nc = ext_vert_ptr[h + 1] - ext_vert_ptr[h];
-        for (int qb = 0; qb < nqb; ++qb) {
+        for (int qb = 0; qb < nqb && n >= 0; ++qb) {
             if (tile_ptr) tile_ptr[h * nqb + qb] = (int32_t)n;
-            long lo_i = (long)T * qb;
-            long hi_i = lo_i + T - 1 < S - 1 ? lo_i + T - 1 : S - 1;
-            int nrows = (int)(hi_i - lo_i + 1);
+            long hi_i = (long)T * qb + T - 1 < S - 1 ? (long)T * qb + T - 1 : S - 1;
             if (stripe_cnt) stripe_cnt[h * nqb + qb] = count_le(C, nc, (int32_t)hi_i);
-            memset(cand, 0, (size_t)nqb);
-            for (int k = 0; k < nd; ++k) {
-                long r = D[k];
-                if (r > hi_i) break;
-                long jlo = lo_i - r > 0 ? lo_i - r : 0;
-                long jhi = hi_i - r;
-                for (long kb = jlo / T; kb <= jhi / T; ++kb) cand[kb] = 1;
-            }
-            for (int kb = 0; kb <= qb; ++kb) {
-                if (!cand[kb]) continue;
-                long base = (long)T * (qb - kb);
-                uint64_t dm[4] = {0, 0, 0, 0}, cm[2] = {0, 0};
-                for (int k = 0; k < nd; ++k) {
-                    long t = D[k] - base + (T - 1);
-                    if (t >= 0 && t <= 2 * T - 2) set_bit(dm, (int)t);
-                }
-                for (int k = 0; k < nc; ++k) {
-                    long jl = C[k] - (long)T * kb;
-                    if (jl >= 0 && jl < T) set_bit(cm, (int)jl);
-                }
-                int listed = 0;
-                for (int t = 0; t <= 2 * T - 2 && !listed; ++t) {
-                    if (!get_bit(dm, t)) continue;
-                    int delta = t - (T - 1); /* il - jl */
-                    int il_lo = delta > 0 ? delta : 0;
-                    int il_hi = T - 1;
-                    if (T - 1 + delta < il_hi) il_hi = T - 1 + delta;
-                    if (nrows - 1 < il_hi) il_hi = nrows - 1;
-                    for (int il = il_lo; il <= il_hi; ++il) {
-                        if (!get_bit(cm, il - delta)) {
-                            listed = 1;
-                            break;
-                        }
-                    }
-                }
-                if (!listed) continue;
-                int full = (kb < qb) && ((long)T * (qb + 1) <= S) && popcount256(dm) == 2 * T - 1 &&
-                           cm[0] == 0 && cm[1] == 0;
-                if (tile_kb) {
-                    if (n >= capacity) {
-                        free(cand);
-                        return ORA_ERR_CAPACITY;
-                    }
-                    tile_kb[n] = kb;
-                    memcpy(tile_dmask + 4 * n, dm, sizeof dm);
-                    memcpy(tile_cmask + 2 * n, cm, sizeof cm);
-                    tile_flags[n] = full ? 1u : 0u;
-                }
-                ++n;
-            }
+            n = interval_block(D, nd, C, nc, S, qb, cand, n, capacity, tile_kb, tile_dmask,
+                               tile_cmask, tile_flags);
         }
     }
-    if (tile_ptr) tile_ptr[n_heads * nqb] = (int32_t)n;
+    if (tile_ptr && n >= 0) tile_ptr[n_heads * nqb] = (int32_t)n;
+    free(cand);
+    return n;
+}
+
+/* Routine 2 for selected blocks only (items[2a] = head, items[2a+1] = query block):
+ * item_ptr[n_items+1] indexes the concatenated tiles of the items in order. */
+long long ora_plan_items(int n_heads, const int32_t *ext_diag_ptr, const int32_t *ext_diag_offsets,
+                         const int32_t *ext_vert_ptr, const int32_t *ext_vert_cols, int S,
+                         int n_items, const int32_t *items, long long capacity, int32_t *item_ptr,
+                         int32_t *tile_kb, uint64_t *tile_dmask, uint64_t *tile_cmask,
+                         uint32_t *tile_flags, int32_t *stripe_cnt) {
+    if (n_heads < 0 || S <= 0 || n_items < 0) return ORA_ERR_INVALID;
+    const int T = ORA_TILE;
+    int nqb = (S + T - 1) / T;
+    uint8_t *cand = (uint8_t *)malloc((size_t)nqb);
+    if (!cand) return ORA_ERR_NOMEM;
+    long long n = 0;
+    for (int a = 0; a < n_items && n >= 0; ++a) {
+        int h = items[2 * a], qb = items[2 * a + 1];
+        if (h < 0 || h >= n_heads || qb < 0 || qb >= nqb) {
+            n = ORA_ERR_INVALID;
+            break;
+        }
+        const int32_t *D = ext_diag_offsets + ext_diag_ptr[h];
+        int nd = ext_diag_ptr[h + 1] - ext_diag_ptr[h];
+        const int32_t *C = ext_vert_cols + ext_vert_ptr[h];
+        int nc = ext_vert_ptr[h + 1] - ext_vert_ptr[h];
+        if (item_ptr) item_ptr[a] = (int32_t)n;
+        long hi_i = (long)T * qb + T - 1 < S - 1 ? (long)T * qb + T - 1 : S - 1;
+        if (stripe_cnt) stripe_cnt[a] = count_le(C, nc, (int32_t)hi_i);
+        n = interval_block(D, nd, C, nc, S, qb, cand, n, capacity, tile_kb, tile_dmask, tile_cmask,
+                           tile_flags);
+    }
+    if (item_ptr && n >= 0) item_ptr[n_items] = (int32_t)n;
     free(cand);
     return n;
 }

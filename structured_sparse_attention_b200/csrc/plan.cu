@@ -1,0 +1,398 @@
+// plan.cu -- stage two of DAM: extension of the kept patterns to S x S and their
+// compilation into per-query-block key-tile lists (DAM review page, "What carries
+// the argument": the kept patterns are pasted into an S x S mask; "Circularity
+// Check" step 1: the mask is the union of the matched patterns).
+//
+// In list form the extension keeps every diagonal r < S and every column c < S.  The
+// tile plan is this library's own layout of that mask for the attention kernel:
+// for each (head, query block) the ascending key tiles the band touches, each with a
+// 255-bit local-diagonal mask, a 128-bit column-exclusion mask and a FULL flag, plus
+// the number of columns the stripe phase covers (exact semantics in ssa.h).
+//
+// Kernels (one warp per (head, query block) for the tile work)
+//   validate_lists_kernel  lists sorted, unique, non-negative; kept counts r < S, c < S
+//   exclusive_scan_kernel  single-block scan (list offsets, tile offsets)
+//   extend_copy_kernel     the extended CSR lists
+//   plan_tiles_kernel      count pass / fill pass of the band tiles + stripe counts
+//   plan_totals_kernel     totals for the sizing pass
+#include "common.cuh"
+
+namespace ssa {
+namespace {
+
+constexpr int kTile = SSA_BLOCK;
+constexpr int kScanThreads = 1024;
+
+struct Totals {  // device-side result of the sizing pass
+    int32_t status;
+    int32_t n_diag;
+    int32_t n_vert;
+    int32_t max_vert;
+    int64_t n_tiles;
+};
+
+struct PlanParams {
+    int H, S, nqb;
+    const int32_t *dptr, *doff, *vptr, *vcol;  // input lists
+    int32_t *ext_counts;   // [2H]: kept diagonals, kept columns per head
+    int32_t *ext_scan;     // [2 (H+1)]: exclusive scans of the two count arrays
+    int32_t *tile_counts;  // [H*nqb]
+    int32_t *tile_ptr;     // [H*nqb + 1] (workspace in the sizing pass, plan in the fill pass)
+    Totals *totals;
+    int32_t *ws_status;
+    int32_t *dev_status;
+    // fill pass outputs
+    int64_t capacity;
+    int32_t *tile_kb;
+    uint64_t *tile_dmask;
+    uint64_t *tile_cmask;
+    uint32_t *tile_flags;
+    int32_t *stripe_cnt;
+    int32_t *ext_dptr, *ext_doff, *ext_vptr, *ext_vcol;
+};
+
+__global__ void validate_lists_kernel(PlanParams p) {
+    const int h = blockIdx.x;
+    const int32_t *D = p.doff + p.dptr[h];
+    const int32_t *C = p.vcol + p.vptr[h];
+    const int nd = p.dptr[h + 1] - p.dptr[h];
+    const int nc = p.vptr[h + 1] - p.vptr[h];
+    bool bad = nd < 0 || nc < 0;
+    for (int k = threadIdx.x; !bad && k < nd; k += blockDim.x)
+        if (D[k] < 0 || (k > 0 && D[k] <= D[k - 1])) bad = true;
+    for (int k = threadIdx.x; !bad && k < nc; k += blockDim.x)
+        if (C[k] < 0 || (k > 0 && C[k] <= C[k - 1])) bad = true;
+    if (__syncthreads_or(bad)) {
+        if (threadIdx.x == 0) {
+            report(p.ws_status, SSA_ERR_INVALID);
+            report(p.dev_status, SSA_ERR_INVALID);
+            p.ext_counts[2 * h] = 0;
+            p.ext_counts[2 * h + 1] = 0;
+        }
+        return;
+    }
+    if (threadIdx.x == 0) {
+        p.ext_counts[2 * h] = lower_bound_i32(D, nd, p.S);
+        p.ext_counts[2 * h + 1] = lower_bound_i32(C, nc, p.S);
+    }
+}
+
+// out[k] = sum_{k' < k} in[k' * stride + offset] for k in [0, n]; one block.
+__global__ void __launch_bounds__(kScanThreads)
+    exclusive_scan_kernel(const int32_t *in, int n, int stride, int offset, int32_t *out) {
+    __shared__ int32_t s_warp[kScanThreads / 32];
+    __shared__ int32_t s_carry;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) s_carry = 0;
+    __syncthreads();
+    for (int start = 0; start < n; start += kScanThreads) {
+        const int k = start + threadIdx.x;
+        const int v = k < n ? in[static_cast<size_t>(k) * stride + offset] : 0;
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) s_warp[warp] = x;
+        __syncthreads();
+        int before = 0, total = 0;
+        for (int w = 0; w < kScanThreads / 32; ++w) {
+            if (w < warp) before += s_warp[w];
+            total += s_warp[w];
+        }
+        const int carry = s_carry;
+        if (k < n) out[k] = carry + before + x - v;
+        __syncthreads();
+        if (threadIdx.x == 0) s_carry = carry + total;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) out[n] = s_carry;
+}
+
+__global__ void extend_copy_kernel(PlanParams p) {
+    const int h = blockIdx.x;
+    const int32_t *D = p.doff + p.dptr[h];
+    const int32_t *C = p.vcol + p.vptr[h];
+    const int nd = p.ext_counts[2 * h], nc = p.ext_counts[2 * h + 1];
+    const int od = p.ext_scan[h], oc = p.ext_scan[(p.H + 1) + h];
+    for (int k = threadIdx.x; k < nd; k += blockDim.x) p.ext_doff[od + k] = D[k];
+    for (int k = threadIdx.x; k < nc; k += blockDim.x) p.ext_vcol[oc + k] = C[k];
+    if (threadIdx.x == 0) {
+        p.ext_dptr[h] = od;
+        p.ext_vptr[h] = oc;
+        if (h == p.H - 1) {
+            p.ext_dptr[h + 1] = od + nd;
+            p.ext_vptr[h + 1] = oc + nc;
+        }
+    }
+}
+
+__device__ __forceinline__ void set_bit_range(uint64_t (&w)[4], int a, int b) {  // inclusive
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int lo = max(a, 64 * k), hi = min(b, 64 * k + 63);
+        if (lo <= hi) {
+            const int n = hi - lo + 1;
+            const uint64_t bits = (n == 64) ? ~0ull : (((1ull << n) - 1ull) << (lo - 64 * k));
+            w[k] |= bits;
+        }
+    }
+}
+
+// Evaluate tile (qb, kb) of one head.  Returns 0 (not listed), 1 (listed), 2 (FULL).
+__device__ int eval_tile(const int32_t *D, int nD, const int32_t *C, int nC, int S, int qb, int kb,
+                         uint64_t (&dm)[4], uint64_t (&cm)[2]) {
+    const int base = kTile * (qb - kb) - (kTile - 1);  // r of dmask bit 0
+    const int lb = lower_bound_i32(D, nD, max(base, 0));
+    const int ub = lower_bound_i32(D, nD, base + 2 * kTile - 1);
+    if (lb == ub) return 0;
+    dm[0] = dm[1] = dm[2] = dm[3] = 0;
+    const int dfirst = __ldg(D + lb), dlast = __ldg(D + ub - 1);
+    if (dlast - dfirst == ub - 1 - lb) {
+        set_bit_range(dm, dfirst - base, dlast - base);  // a contiguous run of offsets
+    } else {
+        for (int k = lb; k < ub; ++k) {
+            const int t = __ldg(D + k) - base;
+            dm[t >> 6] |= 1ull << (t & 63);
+        }
+    }
+    cm[0] = cm[1] = 0;
+    const int cl = lower_bound_i32(C, nC, kTile * kb);
+    for (int k = cl; k < nC; ++k) {
+        const int jl = __ldg(C + k) - kTile * kb;
+        if (jl >= kTile) break;
+        cm[jl >> 6] |= 1ull << (jl & 63);
+    }
+    const int nrows = min(kTile, S - kTile * qb);
+    bool listed = false;
+    if ((cm[0] | cm[1]) == 0) {
+        // with no excluded column, diagonal t has a cell in a valid row iff t <= nrows + 126
+        uint64_t lim[4] = {0, 0, 0, 0};
+        set_bit_range(lim, 0, nrows + kTile - 2);
+        listed = ((dm[0] & lim[0]) | (dm[1] & lim[1]) | (dm[2] & lim[2]) | (dm[3] & lim[3])) != 0;
+    } else {
+        for (int il = 0; il < nrows && !listed; ++il) {
+            uint64_t lo, hi;
+            row_diag_mask(dm, il, lo, hi);
+            listed = ((lo & ~cm[0]) | (hi & ~cm[1])) != 0;
+        }
+    }
+    if (!listed) return 0;
+    const bool all = dm[0] == ~0ull && dm[1] == ~0ull && dm[2] == ~0ull && dm[3] == (~0ull >> 1);
+    const bool full = kb < qb && kTile * (qb + 1) <= S && all && (cm[0] | cm[1]) == 0;
+    return full ? 2 : 1;
+}
+
+// One warp per (head, query block).  FILL = false: count; FILL = true: write tiles.
+template <bool FILL>
+__global__ void __launch_bounds__(128) plan_tiles_kernel(PlanParams p) {
+    const int item = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (item >= p.H * p.nqb) return;
+    const int h = item / p.nqb, qb = item % p.nqb;
+    const int32_t *D = p.doff + p.dptr[h];
+    const int32_t *C = p.vcol + p.vptr[h];
+    const int nD = p.ext_counts[2 * h], nC = p.ext_counts[2 * h + 1];
+    const int lo_i = kTile * qb, hi_i = min(kTile * qb + kTile - 1, p.S - 1);
+    if (FILL && lane == 0) p.stripe_cnt[item] = lower_bound_i32(C, nC, hi_i + 1);
+    // key tiles reachable by some diagonal r <= hi_i
+    const int nvalid = lower_bound_i32(D, nD, hi_i + 1);
+    int count = 0;
+    if (nvalid > 0) {
+        const int rmin = __ldg(D), rmax = __ldg(D + nvalid - 1);
+        const int kb_lo = max(0, lo_i - rmax) / kTile;
+        const int kb_hi = (hi_i - rmin) / kTile;
+        int64_t pos = FILL ? p.tile_ptr[item] : 0;
+        for (int kb0 = kb_lo; kb0 <= kb_hi; kb0 += 32) {
+            const int kb = kb0 + lane;
+            uint64_t dm[4], cm[2];
+            int r = 0;
+            if (kb <= kb_hi) r = eval_tile(D, nD, C, nC, p.S, qb, kb, dm, cm);
+            const uint32_t ball = __ballot_sync(0xffffffffu, r != 0);
+            if (FILL && r) {
+                const int64_t t = pos + __popc(ball & ((1u << lane) - 1u));
+                if (t < p.capacity) {
+                    p.tile_kb[t] = kb;
+                    uint64_t *dst = p.tile_dmask + 4 * t;
+                    dst[0] = dm[0];
+                    dst[1] = dm[1];
+                    dst[2] = dm[2];
+                    dst[3] = dm[3];
+                    p.tile_cmask[2 * t] = cm[0];
+                    p.tile_cmask[2 * t + 1] = cm[1];
+                    p.tile_flags[t] = (r == 2) ? 1u : 0u;
+                } else {
+                    report(p.dev_status, SSA_ERR_CAPACITY);
+                }
+            }
+            pos += __popc(ball);
+            count += __popc(ball);
+        }
+    }
+    if (!FILL && lane == 0) p.tile_counts[item] = count;
+}
+
+__global__ void plan_totals_kernel(PlanParams p) {
+    __shared__ int32_t s[3][32];
+    int nd = 0, nv = 0, mv = 0;
+    for (int h = threadIdx.x; h < p.H; h += blockDim.x) {
+        nd += p.ext_counts[2 * h];
+        nv += p.ext_counts[2 * h + 1];
+        mv = max(mv, p.ext_counts[2 * h + 1]);
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        nd += __shfl_xor_sync(0xffffffffu, nd, o);
+        nv += __shfl_xor_sync(0xffffffffu, nv, o);
+        mv = max(mv, __shfl_xor_sync(0xffffffffu, mv, o));
+    }
+    if (lane == 0) {
+        s[0][warp] = nd;
+        s[1][warp] = nv;
+        s[2][warp] = mv;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        nd = nv = mv = 0;
+        for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
+            nd += s[0][w];
+            nv += s[1][w];
+            mv = max(mv, s[2][w]);
+        }
+        p.totals->status = *p.ws_status;
+        p.totals->n_diag = nd;
+        p.totals->n_vert = nv;
+        p.totals->max_vert = mv;
+        p.totals->n_tiles = p.tile_ptr[p.H * p.nqb];
+    }
+}
+
+size_t align_up(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+}  // namespace ssa
+
+using namespace ssa;
+
+extern "C" size_t sparse_pattern_extend_ws_bytes(int n_heads, int S) {
+    if (n_heads <= 0 || S <= 0) return 0;
+    const size_t nqb = (static_cast<size_t>(S) + kTile - 1) / kTile;
+    const size_t items = static_cast<size_t>(n_heads) * nqb;
+    return align_up(sizeof(Totals)) + align_up(sizeof(int32_t) * 2 * n_heads) +
+           align_up(sizeof(int32_t) * 2 * (n_heads + 1)) + align_up(sizeof(int32_t) * items) +
+           align_up(sizeof(int32_t) * (items + 1)) + 256;
+}
+
+extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
+                                     const int32_t *diag_offsets, const int32_t *vert_ptr,
+                                     const int32_t *vert_cols, int S, ssa_plan_sizes *sizes,
+                                     const ssa_plan *plan, void *ws, size_t ws_bytes,
+                                     int32_t *dev_status, void *stream) {
+    SSA_CHECK_ARG(diag_ptr && diag_offsets && vert_ptr && vert_cols && ws,
+                  "sparse_pattern_extend: null pointer argument");
+    SSA_CHECK_ARG(n_heads >= 1 && S >= 1, "sparse_pattern_extend: n_heads and S must be >= 1");
+    const int nqb = (S + kTile - 1) / kTile;
+    SSA_CHECK_ARG(static_cast<int64_t>(n_heads) * nqb < (1 << 30),
+                  "sparse_pattern_extend: n_heads * ceil(S/128) too large");
+    const size_t need = sparse_pattern_extend_ws_bytes(n_heads, S);
+    if (ws_bytes < need) {
+        set_error("sparse_pattern_extend: workspace %zu bytes < required %zu", ws_bytes, need);
+        return SSA_ERR_CAPACITY;
+    }
+    SSA_CHECK_ARG(aligned16(ws), "sparse_pattern_extend: ws must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    char *w = static_cast<char *>(ws);
+    PlanParams p{};
+    p.H = n_heads;
+    p.S = S;
+    p.nqb = nqb;
+    p.dptr = diag_ptr;
+    p.doff = diag_offsets;
+    p.vptr = vert_ptr;
+    p.vcol = vert_cols;
+    p.totals = reinterpret_cast<Totals *>(w);
+    w += align_up(sizeof(Totals));
+    p.ws_status = &p.totals->status;
+    p.ext_counts = reinterpret_cast<int32_t *>(w);
+    w += align_up(sizeof(int32_t) * 2 * n_heads);
+    p.ext_scan = reinterpret_cast<int32_t *>(w);
+    w += align_up(sizeof(int32_t) * 2 * (n_heads + 1));
+    p.tile_counts = reinterpret_cast<int32_t *>(w);
+    w += align_up(sizeof(int32_t) * n_heads * nqb);
+    int32_t *ws_tile_ptr = reinterpret_cast<int32_t *>(w);
+    p.dev_status = dev_status;
+
+    const int items = n_heads * nqb;
+    const unsigned tile_grid = static_cast<unsigned>((items + 3) / 4);
+    SSA_CUDA_TRY(cudaMemsetAsync(p.totals, 0, sizeof(Totals), s));
+
+    if (plan == nullptr) {
+        SSA_CHECK_ARG(sizes, "sparse_pattern_extend: sizes must not be NULL in the sizing pass");
+        p.tile_ptr = ws_tile_ptr;
+        validate_lists_kernel<<<n_heads, 128, 0, s>>>(p);
+        SSA_LAUNCH_CHECK();
+        plan_tiles_kernel<false><<<tile_grid, 128, 0, s>>>(p);
+        SSA_LAUNCH_CHECK();
+        exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.tile_counts, items, 1, 0, p.tile_ptr);
+        SSA_LAUNCH_CHECK();
+        plan_totals_kernel<<<1, 1024, 0, s>>>(p);
+        SSA_LAUNCH_CHECK();
+        Totals host{};
+        SSA_CUDA_TRY(cudaMemcpyAsync(&host, p.totals, sizeof(Totals), cudaMemcpyDeviceToHost, s));
+        SSA_CUDA_TRY(cudaStreamSynchronize(s));
+        sizes->n_heads = n_heads;
+        sizes->S = S;
+        sizes->nqb = nqb;
+        sizes->n_diag = host.n_diag;
+        sizes->n_vert = host.n_vert;
+        sizes->max_vert = host.max_vert;
+        sizes->n_tiles = host.n_tiles;
+        if (host.status != 0) {
+            set_error("sparse_pattern_extend: a pattern list is not strictly ascending and >= 0");
+            return SSA_ERR_INVALID;
+        }
+        return SSA_OK;
+    }
+
+    SSA_CHECK_ARG(plan->n_heads == n_heads && plan->S == S && plan->nqb == nqb,
+                  "sparse_pattern_extend: plan header (n_heads=%d S=%d nqb=%d) does not match "
+                  "(%d, %d, %d)",
+                  plan->n_heads, plan->S, plan->nqb, n_heads, S, nqb);
+    SSA_CHECK_ARG(plan->ext_diag_ptr && plan->ext_diag_offsets && plan->ext_vert_ptr &&
+                      plan->ext_vert_cols && plan->tile_ptr && plan->tile_kb &&
+                      plan->tile_dmask && plan->tile_cmask && plan->tile_flags &&
+                      plan->stripe_cnt,
+                  "sparse_pattern_extend: null plan array");
+    SSA_CHECK_ARG(plan->n_tiles >= 0, "sparse_pattern_extend: negative tile capacity");
+    p.tile_ptr = plan->tile_ptr;
+    p.capacity = plan->n_tiles;
+    p.tile_kb = plan->tile_kb;
+    p.tile_dmask = plan->tile_dmask;
+    p.tile_cmask = plan->tile_cmask;
+    p.tile_flags = plan->tile_flags;
+    p.stripe_cnt = plan->stripe_cnt;
+    p.ext_dptr = plan->ext_diag_ptr;
+    p.ext_doff = plan->ext_diag_offsets;
+    p.ext_vptr = plan->ext_vert_ptr;
+    p.ext_vcol = plan->ext_vert_cols;
+
+    validate_lists_kernel<<<n_heads, 128, 0, s>>>(p);
+    SSA_LAUNCH_CHECK();
+    exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.ext_counts, n_heads, 2, 0, p.ext_scan);
+    SSA_LAUNCH_CHECK();
+    exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.ext_counts, n_heads, 2, 1,
+                                                     p.ext_scan + (n_heads + 1));
+    SSA_LAUNCH_CHECK();
+    extend_copy_kernel<<<n_heads, 128, 0, s>>>(p);
+    SSA_LAUNCH_CHECK();
+    plan_tiles_kernel<false><<<tile_grid, 128, 0, s>>>(p);
+    SSA_LAUNCH_CHECK();
+    exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.tile_counts, items, 1, 0, p.tile_ptr);
+    SSA_LAUNCH_CHECK();
+    plan_tiles_kernel<true><<<tile_grid, 128, 0, s>>>(p);
+    SSA_LAUNCH_CHECK();
+    return SSA_OK;
+}

@@ -22,10 +22,15 @@ Conventions
   diagonal offsets r (key j = i - r), ``vert`` the vertical columns c (key j = c,
   for queries i >= c).  ``to_csr`` packs them as (ptr, values) pairs.
 * Every generator takes an explicit seed; sub-streams come from
-  ``numpy.random.SeedSequence(seed).spawn``.
+  ``numpy.random.SeedSequence(seed).spawn`` driving NumPy's SFC64 bit generator.
+  The split into sub-streams (one per head / map) is fixed, so the values do not
+  depend on how many threads fill them.
 """
 
 from __future__ import annotations
+
+import concurrent.futures as _cf
+import os
 
 import numpy as np
 
@@ -35,8 +40,20 @@ SEED_BASE = 20261200
 BLOCK = 128
 
 
+def _gen(ss) -> np.random.Generator:
+    return np.random.Generator(np.random.SFC64(ss))
+
+
 def _streams(seed: int, n: int) -> list[np.random.Generator]:
-    return [np.random.Generator(np.random.PCG64(s)) for s in np.random.SeedSequence(seed).spawn(n)]
+    return [_gen(s) for s in np.random.SeedSequence(seed).spawn(n)]
+
+
+def _pmap(fn, items):
+    workers = max(1, min(len(items), os.cpu_count() or 1, 32))
+    if workers == 1:
+        return [fn(x) for x in items]
+    with _cf.ThreadPoolExecutor(workers) as ex:
+        return list(ex.map(fn, items))
 
 
 # --------------------------------------------------------------------------------------
@@ -56,13 +73,22 @@ def f32_from_bf16_bits(b: np.ndarray) -> np.ndarray:
     return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
+def normal_bf16(seed: int, H: int, S: int, d: int) -> np.ndarray:
+    """[H, S, d] bf16 bits of i.i.d. N(0,1) float32 samples, one sub-stream per head."""
+    out = np.empty((H, S, d), np.uint16)
+    seqs = np.random.SeedSequence(seed).spawn(H)
+
+    def fill(h):
+        out[h] = bf16_bits_from_f32(_gen(seqs[h]).standard_normal((S, d), dtype=np.float32))
+
+    _pmap(fill, list(range(H)))
+    return out
+
+
 def qkv(seed: int, H_q: int, H_kv: int, S: int, d: int):
     """Q [H_q,S,d], K [H_kv,S,d], V [H_kv,S,d] as bf16 bits from i.i.d. N(0,1)."""
-    gq, gk, gv = _streams(seed, 3)
-    q = bf16_bits_from_f32(gq.standard_normal((H_q, S, d), dtype=np.float32))
-    k = bf16_bits_from_f32(gk.standard_normal((H_kv, S, d), dtype=np.float32))
-    v = bf16_bits_from_f32(gv.standard_normal((H_kv, S, d), dtype=np.float32))
-    return q, k, v
+    sq, sk, sv = (int(x.generate_state(1)[0]) for x in np.random.SeedSequence(seed).spawn(3))
+    return normal_bf16(sq, H_q, S, d), normal_bf16(sk, H_kv, S, d), normal_bf16(sv, H_kv, S, d)
 
 
 # --------------------------------------------------------------------------------------
@@ -190,14 +216,16 @@ def averaged_maps(seed: int, n_maps: int, L: int = 512, n_samples: int = 16, boo
     ii, jj = np.meshgrid(np.arange(L), np.arange(L), indexing="ij")
     causal = jj <= ii
     out = np.zeros((len(ids), L, L), dtype=np.float32)
-    for o, m in enumerate(ids):
+
+    def one(o):
+        m = ids[o]
         dg, cl = planted[m]
         bonus = np.zeros((L, L), dtype=np.float32)
         for r in dg:
             bonus[(ii - jj) == r] = boost
         bonus[:, cl] = boost
         bonus[~causal] = -np.inf
-        g = np.random.Generator(np.random.PCG64(sample_seeds[m]))
+        g = _gen(sample_seeds[m])
         acc = np.zeros((L, L), dtype=np.float64)
         for _ in range(n_samples):
             z = g.standard_normal((L, L), dtype=np.float32) + bonus
@@ -205,4 +233,6 @@ def averaged_maps(seed: int, n_maps: int, L: int = 512, n_samples: int = 16, boo
             e = np.exp(z)
             acc += e / e.sum(axis=1, keepdims=True)
         out[o] = (acc / n_samples).astype(np.float32)
+
+    _pmap(one, list(range(len(ids))))
     return out

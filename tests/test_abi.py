@@ -1,0 +1,88 @@
+"""The C ABI library builds, loads without a GPU and exports every symbol that
+include/ssa.h declares; host-side argument checks return their documented codes."""
+
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from structured_sparse_attention_b200 import binding, build
+    build.build()
+    return binding.load()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "ssa.h")).read()
+    return re.findall(r"SSA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+
+
+def test_exports_every_declared_symbol(lib):
+    from structured_sparse_attention_b200 import binding
+    names = _declared()
+    assert len(names) >= 9
+    assert sorted(names) == sorted(binding.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_sizes(lib):
+    assert lib.ssa_version() >= 100
+    assert lib.sparse_pattern_capture_ws_bytes(512, 512) == 512 * (4 * 512 + 2) * 4
+    assert lib.sparse_attn_fwd_ws_bytes(32, 128, 128) == 2 * 32 * 128 * 128 * 2
+    assert lib.sparse_attn_fwd_ws_bytes(32, 129, 64) == 2 * 32 * 256 * 64 * 2
+    assert lib.sparse_attn_fwd_ws_bytes(4, 0, 128) == 0
+    assert lib.sparse_pattern_extend_ws_bytes(32, 65536) > 32 * 512 * 8
+
+
+def test_host_argument_checks(lib):
+    from structured_sparse_attention_b200 import binding
+    P = C.c_void_p
+    dummy = P(256)
+    # unsupported lambda and L are rejected before any device work
+    rc = lib.sparse_pattern_capture(dummy, 1, 16, 0.7, 0.3, 0.8, 1e-8, dummy, dummy, dummy, dummy,
+                                    dummy, 1 << 20, None, None)
+    assert rc == -2 and b"lambda" in lib.ssa_last_error()
+    rc = lib.sparse_pattern_capture(dummy, 1, 2048, 0.5, 0.3, 0.8, 1e-8, dummy, dummy, dummy, dummy,
+                                    dummy, 1 << 30, None, None)
+    assert rc == -2
+    rc = lib.sparse_pattern_capture(None, 1, 16, 0.5, 0.3, 0.8, 1e-8, dummy, dummy, dummy, dummy,
+                                    dummy, 1 << 20, None, None)
+    assert rc == -1
+    rc = lib.sparse_pattern_capture(dummy, 4, 16, 0.5, 0.3, 0.8, 1e-8, dummy, dummy, dummy, dummy,
+                                    dummy, 10, None, None)
+    assert rc == -3
+    # head dimension other than 64 / 128
+    plan = binding.PlanStruct()
+    plan.S, plan.n_heads, plan.nqb = 256, 1, 2
+    rc = lib.sparse_attn_fwd(dummy, dummy, dummy, 1, 1, 256, 96, C.byref(plan), None, 0.1, dummy, dummy,
+                             None, 0, None, None)
+    assert rc == -2
+    # plan / shape mismatch
+    rc = lib.sparse_attn_fwd(dummy, dummy, dummy, 1, 1, 300, 64, C.byref(plan), None, 0.1, dummy, dummy,
+                             None, 0, None, None)
+    assert rc == -1 and b"plan" in lib.ssa_last_error()
+    # extend: bad sizes
+    sizes = binding.PlanSizes()
+    rc = lib.sparse_pattern_extend(0, dummy, dummy, dummy, dummy, 10, C.byref(sizes), None, dummy, 1 << 20,
+                                   None, None)
+    assert rc == -1
+
+
+def test_wait_limit_knob(lib):
+    old = lib.ssa_set_wait_limit_ns(12345)
+    assert lib.ssa_set_wait_limit_ns(old) == 12345
+
+
+def test_product_path_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "structured_sparse_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"(from|import)\s+oracle|libssa_oracle|ssa_oracle|\bora_\w+\(", txt), f

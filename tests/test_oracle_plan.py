@@ -152,3 +152,19 @@ def test_plan_routines_agree_and_count_pairs(ora, seed):
         assert nnz[h] == dense
         if S <= 400:
             assert _active_count_from_plan(pb, ext, h, S) == dense
+
+
+def test_plan_items_equals_full_plan(ora):
+    S = 1000
+    diags, verts = inputs.random_patterns(4242, 3, S, max_diag=300, max_vert=30)
+    ext = _ext(ora, diags, verts, S)
+    full = ora.plan(ext, S, "interval")
+    nqb = full["nqb"]
+    items = np.array([[h, qb] for h in (2, 0) for qb in (7, 0, 3)], np.int32)
+    sel = ora.plan_items(ext, S, items)
+    for a, (h, qb) in enumerate(items):
+        f0, f1 = full["tile_ptr"][h * nqb + qb], full["tile_ptr"][h * nqb + qb + 1]
+        s0, s1 = sel["item_ptr"][a], sel["item_ptr"][a + 1]
+        for k in ("tile_kb", "tile_dmask", "tile_cmask", "tile_flags"):
+            np.testing.assert_array_equal(full[k][f0:f1], sel[k][s0:s1])
+        assert full["stripe_cnt"][h * nqb + qb] == sel["stripe_cnt"][a]
