@@ -1,0 +1,427 @@
+"""Benchmark of the DAM structured-sparse-attention hot path on B200.
+
+One step = one pass of the whole path over one synthetic layer:
+  sparse_pattern_capture  (one layer's 32 averaged maps at L = 512)
+  sparse_pattern_extend   (fill pass: validate, extend to S, compile the tile plan)
+  sparse_attn_fwd         (stripe gather + tcgen05 attention forward)
+The default workload is the LLaMA-3-8B-shaped layer at S = 65536 (32 Q / 8 KV heads,
+d = 128, per head 1024 contiguous diagonals at a random offset + 128 random columns).
+The sizing pass of sparse_pattern_extend (an allocation-size query) runs once at set-up.
+
+Prints ONE JSON line (rank 0).  Multi-GPU: one process per GPU (torchrun), each rank
+runs an independent replica (weak scaling), time = max over ranks.
+`--impl reference` times the CPU oracle instead (on the host cores, bounded sample).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from structured_sparse_attention_b200 import inputs  # noqa: E402
+
+METRIC = "sparse-attn prefill tokens/s & effective TFLOP/s vs roofline, per mask density"
+UNIT = "tokens/s"
+
+# Kernels launched per call (the library's own kernels).
+LAUNCHES = {"capture": 3, "extend_fill": 7, "attn": 2}
+
+WORKLOADS = {
+    # name: (H_q, H_kv, S, d, pattern builder)
+    "llama3-8b-layer-64k": (32, 8, 65536, 128, lambda: inputs.patterns_band_random(inputs.SEED_BASE + 4)),
+    "llama3.2-1b-layer-16k": (32, 8, 16384, 64, lambda: inputs.patterns_gqa_16k(inputs.SEED_BASE + 3)),
+    "long-104k-0.5pct": (24, 8, 104000, 128, lambda: inputs.patterns_density(inputs.SEED_BASE + 5, "0.5")),
+    "long-104k-2pct": (24, 8, 104000, 128, lambda: inputs.patterns_density(inputs.SEED_BASE + 5, "2")),
+    "long-104k-10pct": (24, 8, 104000, 128, lambda: inputs.patterns_density(inputs.SEED_BASE + 5, "10")),
+    "long-104k-100pct": (24, 8, 104000, 128, lambda: inputs.patterns_density(inputs.SEED_BASE + 5, "100")),
+}
+SEEDS = {"llama3-8b-layer-64k": inputs.SEED_BASE + 4, "llama3.2-1b-layer-16k": inputs.SEED_BASE + 3}
+CAPTURE_MAPS = 32  # one layer's heads
+CAPTURE_L = 512
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def nnz_per_head(diags, verts, S):
+    """Retained pairs per head of the extended mask, from the list form (integer counting)."""
+    out = []
+    for D, Cc in zip(diags, verts):
+        D = np.asarray(D, np.int64)
+        Cc = np.asarray(Cc, np.int64)
+        D = D[D < S]
+        Cc = Cc[Cc < S]
+        total = int((S - D).sum()) + int((S - Cc).sum())
+        if len(D) and len(Cc):
+            # a cell (c + r, c) lies on both a column and a diagonal: count it once
+            shared = np.searchsorted(np.sort(D), S - Cc, side="left").sum()
+            total -= int(shared)
+        out.append(total)
+    return np.array(out, np.int64)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.index = gpu_id  # nvidia-smi --id value (PCI bus id of the device in use)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        rank = int(os.environ["RANK"])
+        local = int(os.environ.get("LOCAL_RANK", rank))
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        return rank, world, local, dist
+    return 0, 1, 0, None
+
+
+def max_over_ranks(x: float, dist, device):
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------
+# CPU oracle leg
+# ------------------------------------------------------------------------------------
+
+def oracle_leg(workload, budget_s=15.0, maps=None):
+    """Time the oracle as it stands on a bounded sample of the workload.  Returns
+    (tokens/s extrapolated to the whole step, description dict)."""
+    from oracle import oracle as ora
+    Hq, Hkv, S, d, builder = WORKLOADS[workload]
+    diags, verts = builder()
+    cores = len(os.sched_getaffinity(0))
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    # capture of the layer's maps, timed in full
+    if maps is None:
+        maps = inputs.averaged_maps(inputs.SEED_BASE + 2, CAPTURE_MAPS, L=CAPTURE_L, n_samples=16)
+    t0 = time.perf_counter()
+    ora.capture(maps)
+    t_cap = time.perf_counter() - t0
+    dp, do = inputs.to_csr(diags)
+    vp, vo = inputs.to_csr(verts)
+    t0 = time.perf_counter()
+    ext = ora.extend(dp, do, vp, vo, S)
+    t_ext = time.perf_counter() - t0
+    # attention on sampled rows, growing the sample until the budget is spent
+    q, k, v = inputs.qkv(SEEDS.get(workload, inputs.SEED_BASE + 5), Hq, Hkv, S, d)
+    g = np.random.default_rng(7)
+    n_rows, t_rows, done = 8, 0.0, 0
+    while t_rows < budget_s and done < S:
+        rows = np.sort(g.choice(S, size=min(n_rows, S), replace=False)).astype(np.int32)
+        t0 = time.perf_counter()
+        ora.attn_rows(q, k, v, ext, d ** -0.5, rows)
+        t_rows += time.perf_counter() - t0
+        done += len(rows)
+        n_rows *= 2
+    t_step = t_cap + t_ext + t_rows * (S / done)
+    desc = {"kind": "oracle", "cores": int(os.environ.get("OMP_NUM_THREADS", cores)),
+            "sample": f"capture of {CAPTURE_MAPS} maps at L={CAPTURE_L} in full ({t_cap:.2f} s), "
+                      f"extension in full, attention on {done} random query rows x {Hq} heads "
+                      f"({t_rows:.1f} s), extrapolated to S={S} rows"}
+    return S / t_step, desc
+
+
+# ------------------------------------------------------------------------------------
+# GPU leg
+# ------------------------------------------------------------------------------------
+
+def run_gpu(args, rank, world, local, dist):
+    import torch
+
+    import structured_sparse_attention_b200 as ssa
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    Hq, Hkv, S, d, builder = WORKLOADS[args.workload]
+    diags, verts = builder()
+    seed = SEEDS.get(args.workload, inputs.SEED_BASE + 5)
+
+    # ---------------- inputs (host, then resident in HBM) ----------------
+    maps_h = inputs.averaged_maps(inputs.SEED_BASE + 2, CAPTURE_MAPS, L=CAPTURE_L, n_samples=16)
+    q_h, k_h, v_h = inputs.qkv(seed, Hq, Hkv, S, d)
+    dp, do = inputs.to_csr(diags)
+    vp, vo = inputs.to_csr(verts)
+
+    def pinned(a, dtype=None):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if dtype is not None:
+            t = t.view(dtype)
+        return t.pin_memory()
+
+    h_maps = pinned(maps_h)
+    h_q, h_k, h_v = (pinned(a.view(np.int16), torch.bfloat16) for a in (q_h, k_h, v_h))
+    h_lists = [pinned(a.astype(np.int32)) for a in (dp, do, vp, vo)]
+    maps = h_maps.to(dev)
+    q, k, v = h_q.to(dev), h_k.to(dev), h_v.to(dev)
+    lists = [t.to(dev) for t in h_lists]
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    cap_out = ssa.capture(maps)  # allocates outputs once
+    cap_ws = torch.empty(ssa.load().sparse_pattern_capture_ws_bytes(CAPTURE_MAPS, CAPTURE_L),
+                         dtype=torch.uint8, device=dev)
+    plan = ssa.extend(*lists, S)  # sizing pass + first fill (allocations)
+    O = torch.empty_like(q)
+    LSE = torch.empty((Hq, S), dtype=torch.float32, device=dev)
+    attn_ws = torch.empty(max(ssa.attn_ws_bytes(plan, d), 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    ev = {n: [torch.cuda.Event(enable_timing=True) for _ in range(2)] for n in ("cap", "ext", "attn")}
+
+    def step(timed_stage=None):
+        if timed_stage:
+            ev["cap"][0].record(stream)
+        ssa.capture(maps, out=cap_out, ws=cap_ws, status=status, check=False)
+        if timed_stage:
+            ev["cap"][1].record(stream)
+            ev["ext"][0].record(stream)
+        ssa.refill(plan, *lists, status=status)
+        if timed_stage:
+            ev["ext"][1].record(stream)
+            ev["attn"][0].record(stream)
+        ssa.attn_fwd(q, k, v, plan, out=O, lse=LSE, ws=attn_ws, status=status, check=False)
+        if timed_stage:
+            ev["attn"][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during warm-up")
+
+    # ---------------- device-timed region ----------------
+    stage_ms = {"cap": 0.0, "ext": 0.0, "attn": 0.0}
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0")
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)  # let the sampler take its first reading
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if dist is not None:
+        dist.barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    ms_step = max_over_ranks(ms_total / args.steps, dist, dev)
+
+    # per-stage device times, averaged over a second pass of timed steps
+    reps = max(5, min(args.steps, 50))
+    for _ in range(reps):
+        step(timed_stage=True)
+        torch.cuda.synchronize()
+        for n in stage_ms:
+            stage_ms[n] += ev[n][0].elapsed_time(ev[n][1]) / reps
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during timing")
+
+    # ---------------- end-to-end through the public API with host buffers ----------------
+    e2e = None
+    if not args.no_e2e:
+        h_O = torch.empty(O.shape, dtype=torch.bfloat16).pin_memory()
+        h_L = torch.empty(LSE.shape, dtype=torch.float32).pin_memory()
+        e_steps = max(3, min(10, args.steps))
+
+        def e2e_step():
+            maps.copy_(h_maps, non_blocking=True)
+            q.copy_(h_q, non_blocking=True)
+            k.copy_(h_k, non_blocking=True)
+            v.copy_(h_v, non_blocking=True)
+            for dst, src in zip(lists, h_lists):
+                dst.copy_(src, non_blocking=True)
+            step()
+            h_O.copy_(O, non_blocking=True)
+            h_L.copy_(LSE, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, dist, dev)
+        h2d = (h_maps.numel() * 4 + sum(t.numel() * 2 for t in (h_q, h_k, h_v)) +
+               sum(t.numel() * 4 for t in h_lists))
+        d2h = h_O.numel() * 2 + h_L.numel() * 4
+        e2e = {"value": world * S / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms}
+
+    # ---------------- metrics ----------------
+    nnz = nnz_per_head(diags, verts, S)
+    flops = 4.0 * d * float(nnz.sum())
+    causal_pairs = S * (S + 1) / 2
+    density = float(nnz.mean() / causal_pairs)
+    hbm_gbs, tf_burst, tf_sust, peak_kind = load_peaks()
+    attn_ms = max_over_ranks(stage_ms["attn"], dist, dev)
+    algo_bytes = (2 * Hq * S * d * 2) + (2 * Hkv * S * d * 2) + Hq * S * 4
+    t_tensor = flops / (tf_burst * 1e12)
+    t_hbm = algo_bytes / (hbm_gbs * 1e9)
+    bound = "tensor" if t_tensor >= t_hbm else "hbm"
+    if bound == "tensor":
+        achieved = flops / (attn_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
+                "frac": achieved / tf_burst}
+    else:
+        achieved = algo_bytes / (attn_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                "frac": achieved / hbm_gbs}
+    roof.update({"traffic": args.traffic, "kernel": "sparse_attn_fwd (stripe gather + attention kernel)",
+                 "peak_source": f"{peak_kind} ({'burst' if bound == 'tensor' else 'copy'})",
+                 "algorithmic": {"flops": flops, "bytes": algo_bytes},
+                 "roofline_ms": max(t_tensor, t_hbm) * 1e3, "frac_of_roofline_time": max(t_tensor, t_hbm) * 1e3 / attn_ms})
+
+    line = {
+        "metric": METRIC, "value": world * S / (ms_step / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "H_q": Hq, "H_kv": Hkv, "S": S, "d": d,
+                   "density_of_causal": density, "nnz_per_head_mean": float(nnz.mean()),
+                   "capture": f"{CAPTURE_MAPS} maps x L={CAPTURE_L} per step", "batch": 1,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single-gpu",
+                   "l2": "inputs larger than L2 (Q+K+V+O %.2f GB)" % ((2 * Hq + 2 * Hkv) * S * d * 2 / 1e9)},
+        "stages_ms": {"capture": stage_ms["cap"], "extend_fill": stage_ms["ext"], "attn_fwd": attn_ms},
+        "attn_tokens_per_s": S / (attn_ms / 1e3),
+        "effective_tflops": flops / (attn_ms / 1e3) / 1e12,
+        "roofline": roof,
+        "clocks": clocks,
+        "e2e": e2e,
+        "gpu_launches": args.steps * sum(LAUNCHES.values()),
+    }
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ssa", choices=["ssa", "reference"])
+    ap.add_argument("--workload", default="llama3-8b-layer-64k", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle attention work")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per attention launch from an ncu capture of the same kernel")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank, world, local, dist = dist_setup(args.gpus)
+    if args.impl == "reference":
+        if rank == 0:
+            Hq, Hkv, S, d, _ = WORKLOADS[args.workload]
+            t0 = time.perf_counter()
+            vals = []
+            desc = None
+            maps = inputs.averaged_maps(inputs.SEED_BASE + 2, CAPTURE_MAPS, L=CAPTURE_L, n_samples=16)
+            for i in range(args.warmup + args.steps):
+                budget = max(1.0, args.cpu_budget / max(1, args.steps))
+                v, desc = oracle_leg(args.workload, budget_s=budget, maps=maps)
+                if i >= args.warmup:
+                    vals.append(v)
+            value = float(np.median(vals))
+            line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                    "steps": args.steps, "warmup": args.warmup, "ms_per_step": S / value * 1e3,
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                    "data": "synthetic", "config": {"workload": args.workload, "H_q": Hq, "H_kv": Hkv, "S": S,
+                                                    "d": d},
+                    "cpu_baseline": dict(desc, value=value, unit=UNIT),
+                    "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                    "wall_s": time.perf_counter() - t0}
+            print(json.dumps(line), flush=True)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    line = run_gpu(args, rank, world, local, dist)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc = oracle_leg(args.workload, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = dict(desc, value=v, unit=UNIT)
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

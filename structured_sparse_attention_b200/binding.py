@@ -3,6 +3,9 @@
 Argument marshalling only: torch provides device memory and the current stream; every
 step of the computation runs in the library's CUDA kernels.  There is no fallback: if
 libssa.so is missing or no CUDA device is present the calls raise.
+
+A caller-provided ``status`` tensor (one int32 on the device) is used as is: the
+caller zeroes it and reads it (the functions read it themselves when ``check``).
 """
 
 from __future__ import annotations
@@ -140,8 +143,6 @@ def capture(maps: torch.Tensor, lam: float = 0.5, tau: float = 0.3, mu: float = 
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=dev)
-    else:
-        status.zero_()
     cs, s = _stream(stream)
     _check(lib.sparse_pattern_capture(_ptr(maps), n, L, lam, tau, mu, eps, _ptr(out["diag_ptr"]),
                                       _ptr(out["diag_offsets"]), _ptr(out["vert_ptr"]),
@@ -223,8 +224,6 @@ def extend(diag_ptr, diag_offsets, vert_ptr, vert_cols, S: int, *, stream=None, 
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=dev)
-    else:
-        status.zero_()
     cs, s = _stream(stream)
     sizes = PlanSizes()
     _check(lib.sparse_pattern_extend(H, _ptr(diag_ptr), _ptr(diag_offsets), _ptr(vert_ptr),
@@ -285,8 +284,6 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan, *, k
         _need_cuda(kv_map, "kv_map", torch.int32)
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=dev)
-    elif check:
-        status.zero_()
     cs, s = _stream(stream)
     _check(lib.sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, S, d, C.byref(plan.struct),
                                _ptr(kv_map), float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
