@@ -92,6 +92,36 @@ SSA_API int sparse_pattern_capture(const float *maps, int n_maps, int L, double 
                            int32_t *vert_ptr, int32_t *vert_cols, void *ws, size_t ws_bytes,
                            int32_t *dev_status, void *stream);
 
+/* Size of the fixed device scratch of sparse_pattern_capture_noalloc (8 MiB). */
+#define SSA_CAPTURE_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * sparse_pattern_capture_noalloc -- sparse_pattern_capture without a workspace
+ * argument.  The paper has no counterpart: this is a deployment variant.
+ *
+ * For callers that cannot allocate device memory: a plugin host that only hands the
+ * library its input and output buffers and has no allocator to lend, or a serving
+ * process that must not call cudaMalloc/cudaFree after start-up because those calls
+ * can synchronise the device and stall every other stream.  The call itself allocates
+ * nothing: its scratch is a fixed SSA_CAPTURE_NOALLOC_SCRATCH_BYTES device array
+ * inside the library, held by every GPU that loads the library until the process
+ * exits.  Arguments, outputs and results are those of sparse_pattern_capture; the
+ * caller still provides maps, the four output lists and dev_status.
+ *
+ *   - Sizes whose scratch (sparse_pattern_capture_ws_bytes(n_maps, L)) exceeds the
+ *     fixed size are rejected with SSA_ERR_CAPACITY before any device work
+ *     (L = 512 allows up to 1023 maps).
+ *   - The first call on each device looks up the array's device address with that
+ *     device current; make that first call before any stream capture begins.
+ *   - Every call shares the one array per device and clears what must start at zero
+ *     itself; calls that overlap on the GPU (different streams or host threads) race
+ *     on it and must be serialised by the caller.
+ */
+SSA_API int sparse_pattern_capture_noalloc(const float *maps, int n_maps, int L, double lambda,
+                                           double tau, double mu, double eps, int32_t *diag_ptr,
+                                           int32_t *diag_offsets, int32_t *vert_ptr,
+                                           int32_t *vert_cols, int32_t *dev_status, void *stream);
+
 /* ------------------------------------------------------------------------------ */
 /* Stage two: extension to S and the tile plan                                     */
 /* ------------------------------------------------------------------------------ */

@@ -24,7 +24,7 @@ ERRORS = {-1: "SSA_ERR_INVALID", -2: "SSA_ERR_UNSUPPORTED", -3: "SSA_ERR_CAPACIT
 BLOCK = 128
 
 #: Every symbol include/ssa.h declares.
-EXPORTS = ("sparse_pattern_capture_ws_bytes", "sparse_pattern_capture",
+EXPORTS = ("sparse_pattern_capture_ws_bytes", "sparse_pattern_capture", "sparse_pattern_capture_noalloc",
            "sparse_pattern_extend_ws_bytes", "sparse_pattern_extend",
            "sparse_attn_fwd_ws_bytes", "sparse_attn_fwd",
            "ssa_last_error", "ssa_version", "ssa_set_wait_limit_ns")

@@ -345,3 +345,70 @@ extern "C" int sparse_pattern_capture(const float *maps, int n_maps, int L, doub
     SSA_LAUNCH_CHECK();
     return SSA_OK;
 }
+
+// ---------------------------------------------------------------------------------
+// Allocation-free variant of sparse_pattern_capture.
+//
+// Its scratch (hit counts, staging lists and per-map counts) lives in a file-scope
+// device array instead of a caller-provided workspace.  Every GPU that loads the
+// library holds this array until the process exits.  All calls share it and it
+// keeps the last call's contents: the call clears the hit counts itself (the only
+// part that must start at zero), and calls whose work overlaps on the GPU (other
+// streams, other host threads) race on it.
+// ---------------------------------------------------------------------------------
+#include <mutex>
+
+namespace ssa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = SSA_CAPTURE_NOALLOC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) int32_t g_capture_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
+
+std::mutex g_scratch_mutex;
+void *g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_capture_scratch on the current device.  Looked up once per
+// device, with that device current; in host code the array's name is only a host-side
+// stand-in, never a device address.
+int scratch_address(void **out) {
+    int dev = -1;
+    SSA_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) {
+        set_error("sparse_pattern_capture_noalloc: device ordinal %d out of range", dev);
+        return SSA_ERR_UNSUPPORTED;
+    }
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        SSA_CUDA_TRY(cudaGetSymbolAddress(&p, g_capture_scratch));
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return SSA_OK;
+}
+
+}  // namespace
+}  // namespace ssa
+
+extern "C" int sparse_pattern_capture_noalloc(const float *maps, int n_maps, int L, double lambda,
+                                              double tau, double mu, double eps, int32_t *diag_ptr,
+                                              int32_t *diag_offsets, int32_t *vert_ptr,
+                                              int32_t *vert_cols, int32_t *dev_status,
+                                              void *stream) {
+    SSA_CHECK_ARG(n_maps >= 1 && L >= 1, "sparse_pattern_capture_noalloc: n_maps and L must be >= 1");
+    const size_t need = sparse_pattern_capture_ws_bytes(n_maps, L);
+    if (need > kNoAllocScratchBytes) {
+        set_error("sparse_pattern_capture_noalloc: %d maps of %d x %d need %zu scratch bytes, more "
+                  "than the fixed %zu; use sparse_pattern_capture with a workspace",
+                  n_maps, L, L, need, kNoAllocScratchBytes);
+        return SSA_ERR_CAPACITY;
+    }
+    void *scratch = nullptr;
+    const int rc = scratch_address(&scratch);
+    if (rc != SSA_OK) return rc;
+    return sparse_pattern_capture(maps, n_maps, L, lambda, tau, mu, eps, diag_ptr, diag_offsets,
+                                  vert_ptr, vert_cols, scratch, kNoAllocScratchBytes, dev_status,
+                                  stream);
+}
