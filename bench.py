@@ -40,12 +40,16 @@ WORKLOADS = {
     # name: (H_q, H_kv, S, d, pattern builder)
     "llama3-8b-layer-64k": (32, 8, 65536, 128, lambda: inputs.patterns_band_random(inputs.SEED_BASE + 4)),
     "llama3.2-1b-layer-16k": (32, 8, 16384, 64, lambda: inputs.patterns_gqa_16k(inputs.SEED_BASE + 3)),
+    # small case of the 8B layer (same pattern rule at S = 16384) for profiler captures
+    "llama3-8b-layer-16k": (32, 8, 16384, 128,
+                            lambda: inputs.patterns_band_random(inputs.SEED_BASE + 6, S=16384)),
     "long-104k-0.5pct": (24, 8, 104000, 128, lambda: inputs.patterns_density(inputs.SEED_BASE + 5, "0.5")),
     "long-104k-2pct": (24, 8, 104000, 128, lambda: inputs.patterns_density(inputs.SEED_BASE + 5, "2")),
     "long-104k-10pct": (24, 8, 104000, 128, lambda: inputs.patterns_density(inputs.SEED_BASE + 5, "10")),
     "long-104k-100pct": (24, 8, 104000, 128, lambda: inputs.patterns_density(inputs.SEED_BASE + 5, "100")),
 }
-SEEDS = {"llama3-8b-layer-64k": inputs.SEED_BASE + 4, "llama3.2-1b-layer-16k": inputs.SEED_BASE + 3}
+SEEDS = {"llama3-8b-layer-64k": inputs.SEED_BASE + 4, "llama3.2-1b-layer-16k": inputs.SEED_BASE + 3,
+         "llama3-8b-layer-16k": inputs.SEED_BASE + 6}
 CAPTURE_MAPS = 32  # one layer's heads
 CAPTURE_L = 512
 
