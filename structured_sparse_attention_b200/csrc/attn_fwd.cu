@@ -23,6 +23,8 @@
 //                epilogue O / l -> bf16 and LSE
 // Tensor memory (512 columns): S0 0..127, S1 128..255, P0 256..319, P1 320..383,
 // O 384..384+d-1.  P has its own buffers so a QK^T never overwrites a P still being read.
+// Barrier phases are tracked by tile index; every wait is on a barrier whose previous
+// phase is known to have completed, so a parity never aliases two phases back.
 // Every wait is bounded: on expiry the kernel records SSA_ERR_TIMEOUT, stops every role,
 // drains its own copies and MMAs, frees tensor memory and returns.
 #include <cuda.h>
@@ -36,7 +38,8 @@ namespace {
 
 constexpr int kBM = SSA_BLOCK;
 constexpr int kBN = SSA_BLOCK;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 softmax (two halves per row)
+constexpr int kSoftmaxThreads = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;
 constexpr int kBoxBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
@@ -45,29 +48,34 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if the ma
 
 template <int D>
 struct Cfg {
-    static constexpr int NS = (D == 128) ? 2 : 3;  // K/V pipeline stages
+    static constexpr int NK = (D == 128) ? 3 : 4;  // K pipeline stages
+    static constexpr int NV = (D == 128) ? 2 : 3;  // V pipeline stages
     static constexpr int BOXES = D / 64;
     static constexpr int TILE_BYTES = BOXES * kBoxBytes;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + TILE_BYTES;
-    static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
-    static constexpr int OFF_BAR = OFF_V + NS * TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + NK * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_V + NV * TILE_BYTES;
     // barriers + alignment slack; at least 120 KB so that a single CTA (and its 512
     // tensor-memory columns) occupies an SM
-    static constexpr int SMEM_RAW = OFF_BAR + 1024 + 1024;
+    static constexpr int SMEM_RAW = OFF_BAR + 4096 + 1024;
     static constexpr int SMEM_BYTES = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
 };
 
 struct Barriers {
     uint64_t q_full;
-    uint64_t k_full[3], v_full[3], k_empty[3], v_empty[3];
+    uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
     uint64_t s_full[2], p_full[2], p_free[2];
-    uint64_t o_ready;
     uint64_t epi_done;
     uint64_t mma_drain;
+    uint64_t xchg[4][2];  // per TMEM lane quarter and tile parity: row-max exchange
+    uint64_t lxchg[4];    // per quarter: final row-sum exchange
     uint32_t tmem_base;
     int abort;
+    float red_max[2][2][128];  // [tile parity][column half][row]
+    float red_l[2][128];       // [column half][row]
 };
+static_assert(sizeof(Barriers) <= 4096, "barrier block too large");
 
 struct AttnParams {
     int S, H, Hkv, nqb, npad;
@@ -174,12 +182,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (n == 0) {  // no retained key in this block: O = 0, LSE = -inf
         if (warp >= 2) {
+            const int half = (warp - 2) >> 2;
             const int i = qb * kBM + 32 * (warp & 3) + lane;
             if (i < p.S) {
-                uint4 *dst = reinterpret_cast<uint4 *>(p.O + (static_cast<size_t>(h) * p.S + i) * D);
+                uint4 *dst = reinterpret_cast<uint4 *>(p.O + (static_cast<size_t>(h) * p.S + i) * D) +
+                             half * (D / 16);
 #pragma unroll
-                for (int k = 0; k < D / 8; ++k) dst[k] = make_uint4(0, 0, 0, 0);
-                p.LSE[static_cast<size_t>(h) * p.S + i] = -INFINITY;
+                for (int k = 0; k < D / 16; ++k) dst[k] = make_uint4(0, 0, 0, 0);
+                if (half == 0) p.LSE[static_cast<size_t>(h) * p.S + i] = -INFINITY;
             }
         }
         return;
@@ -187,20 +197,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&bar->q_full, 1);
-        for (int s = 0; s < C::NS; ++s) {
+        for (int s = 0; s < C::NK; ++s) {
             mbar_init(&bar->k_full[s], 1);
-            mbar_init(&bar->v_full[s], 1);
             mbar_init(&bar->k_empty[s], 1);
+        }
+        for (int s = 0; s < C::NV; ++s) {
+            mbar_init(&bar->v_full[s], 1);
             mbar_init(&bar->v_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar->s_full[b], 1);
-            mbar_init(&bar->p_full[b], 128);
+            mbar_init(&bar->p_full[b], kSoftmaxThreads);
             mbar_init(&bar->p_free[b], 1);
         }
-        mbar_init(&bar->o_ready, 1);
-        mbar_init(&bar->epi_done, 128);
+        mbar_init(&bar->epi_done, kSoftmaxThreads);
         mbar_init(&bar->mma_drain, 1);
+        for (int q = 0; q < 4; ++q) {
+            mbar_init(&bar->xchg[q][0], 64);
+            mbar_init(&bar->xchg[q][1], 64);
+            mbar_init(&bar->lxchg[q], 64);
+        }
         bar->abort = 0;
         fence_barrier_init();
     }
@@ -215,50 +231,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t lim = p.wait_ns;
 
     if (warp == 0) {
-        // ------------------------------ TMA producer ------------------------------
-        if (lane == 0) {
-            prefetch_tmap(&tmQ);
-            prefetch_tmap(&tmK);
-            prefetch_tmap(&tmV);
-            uint8_t *sQ = smem + C::OFF_Q;
-            mbar_arrive_expect_tx(&bar->q_full, C::TILE_BYTES);
-            for (int b = 0; b < C::BOXES; ++b)
-                tma_load_3d(sQ + b * kBoxBytes, &tmQ, &bar->q_full, 64 * b, qb * kBM, h);
+        // ------------------------------ TMA producers -----------------------------
+        // lane 0 streams Q then the K tiles, lane 1 the V tiles, each with its own ring
+        if (lane < 2) {
+            const bool is_k = (lane == 0);
+            const int NSTG = is_k ? C::NK : C::NV;
+            uint64_t *full = is_k ? bar->k_full : bar->v_full;
+            uint64_t *empty = is_k ? bar->k_empty : bar->v_empty;
+            uint8_t *ring = smem + (is_k ? C::OFF_K : C::OFF_V);
+            const CUtensorMap *band_map = is_k ? &tmK : &tmV;
+            const CUtensorMap *stripe_map = is_k ? &tmKC : &tmVC;
+            prefetch_tmap(band_map);
+            if (is_k) {
+                prefetch_tmap(&tmQ);
+                uint8_t *sQ = smem + C::OFF_Q;
+                mbar_arrive_expect_tx(&bar->q_full, C::TILE_BYTES);
+                for (int b = 0; b < C::BOXES; ++b)
+                    tma_load_3d(sQ + b * kBoxBytes, &tmQ, &bar->q_full, 64 * b, qb * kBM, h);
+            }
             int issued = 0;
             bool ok = true;
-            for (int j = 0; j < n && ok; ++j) {
-                const int s = j % C::NS;
-                const uint32_t empty_par = ((j / C::NS) - 1) & 1;
-                const CUtensorMap *mk, *mv;
-                int y, z;
-                if (j < nb) {
-                    mk = &tmK;
-                    mv = &tmV;
-                    y = __ldg(p.tile_kb + tp0 + j) * kBN;
-                    z = g;
-                } else {
-                    mk = &tmKC;
-                    mv = &tmVC;
-                    y = (j - nb) * kBN;
-                    z = h;
-                }
-                if (j >= C::NS && !mbar_wait(&bar->k_empty[s], empty_par, lim, abort)) {
+            int kb_next = (nb > 0) ? __ldg(p.tile_kb + tp0) : 0;
+            for (int j = 0; j < n; ++j) {
+                const int s = j % NSTG;
+                const int kb = kb_next;
+                if (j + 1 < nb) kb_next = __ldg(p.tile_kb + tp0 + j + 1);  // overlaps the wait
+                if (j >= NSTG && !mbar_wait(&empty[s], ((j / NSTG) - 1) & 1, lim, abort)) {
                     ok = false;
                     break;
                 }
-                uint8_t *sK = smem + C::OFF_K + s * C::TILE_BYTES;
-                mbar_arrive_expect_tx(&bar->k_full[s], C::TILE_BYTES);
+                const bool band = j < nb;
+                const CUtensorMap *map = band ? band_map : stripe_map;
+                const int y = band ? kb * kBN : (j - nb) * kBN;
+                const int z = band ? g : h;
+                uint8_t *dst = ring + s * C::TILE_BYTES;
+                mbar_arrive_expect_tx(&full[s], C::TILE_BYTES);
                 for (int b = 0; b < C::BOXES; ++b)
-                    tma_load_3d(sK + b * kBoxBytes, mk, &bar->k_full[s], 64 * b, y, z);
-                if (j >= C::NS && !mbar_wait(&bar->v_empty[s], empty_par, lim, abort)) {
-                    ok = false;
-                    issued = j + 1;  // K of tile j is in flight
-                    break;
-                }
-                uint8_t *sV = smem + C::OFF_V + s * C::TILE_BYTES;
-                mbar_arrive_expect_tx(&bar->v_full[s], C::TILE_BYTES);
-                for (int b = 0; b < C::BOXES; ++b)
-                    tma_load_3d(sV + b * kBoxBytes, mv, &bar->v_full[s], 64 * b, y, z);
+                    tma_load_3d(dst + b * kBoxBytes, map, &full[s], 64 * b, y, z);
                 issued = j + 1;
             }
             if (!ok) {
@@ -266,13 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *abort = 1;
             }
             // Drain: never leave the CTA with a copy still writing shared memory.
-            mbar_wait(&bar->q_full, 0, kDrainLimitNs, nullptr);
-            for (int j = (issued > C::NS ? issued - C::NS : 0); j < issued; ++j) {
-                const int s = j % C::NS;
-                const uint32_t par = (j / C::NS) & 1;
-                mbar_wait(&bar->k_full[s], par, kDrainLimitNs, nullptr);
-                if (ok || j + 1 < issued) mbar_wait(&bar->v_full[s], par, kDrainLimitNs, nullptr);
-            }
+            if (is_k) mbar_wait(&bar->q_full, 0, kDrainLimitNs, nullptr);
+            for (int j = (issued > NSTG ? issued - NSTG : 0); j < issued; ++j)
+                mbar_wait(&full[j % NSTG], (j / NSTG) & 1, kDrainLimitNs, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------ MMA issuer --------------------------------
@@ -282,9 +287,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t sQ = smem_u32(smem + C::OFF_Q);
             bool ok = mbar_wait(&bar->q_full, 0, lim, abort);
             auto issue_pv = [&](int jj) -> bool {
-                const int b = jj & 1, s = jj % C::NS;
+                const int b = jj & 1, s = jj % C::NV;
                 if (!mbar_wait(&bar->p_full[b], (jj >> 1) & 1, lim, abort)) return false;
-                if (!mbar_wait(&bar->v_full[s], (jj / C::NS) & 1, lim, abort)) return false;
+                if (!mbar_wait(&bar->v_full[s], (jj / C::NV) & 1, lim, abort)) return false;
                 tc_fence_after();
                 const uint32_t sV = smem_u32(smem + C::OFF_V + s * C::TILE_BYTES);
 #pragma unroll
@@ -294,14 +299,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma_ts(tmem + kColO, tmem + kColP + 64 * b + 8 * kk, bd, IDESC_PV,
                             (jj > 0 || kk > 0) ? 1u : 0u);
                 }
+                // p_free[b] completes once per PV that read P[b]: PV_b, PV_{b+2}, ... It
+                // doubles as "O includes tile jj" (see the softmax waits).
                 umma_commit(&bar->p_free[b]);
                 umma_commit(&bar->v_empty[s]);
-                umma_commit(&bar->o_ready);
                 return true;
             };
             for (int j = 0; j < n && ok; ++j) {
-                const int s = j % C::NS, b = j & 1;
-                if (!mbar_wait(&bar->k_full[s], (j / C::NS) & 1, lim, abort)) {
+                const int s = j % C::NK, b = j & 1;
+                if (!mbar_wait(&bar->k_full[s], (j / C::NK) & 1, lim, abort)) {
                     ok = false;
                     break;
                 }
@@ -336,15 +342,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_dealloc(tmem, kTmemCols);
     } else {
         // ------------------------------ softmax / epilogue ------------------------
+        // Two threads per query row: warps 2-5 take key columns 0..63 of every tile,
+        // warps 6-9 columns 64..127 (and the matching halves of O).  The row max of each
+        // tile is exchanged through shared memory so both halves scale by the same
+        // reference; each half keeps its own partial row sum until the epilogue.
+        const int half = (warp - 2) >> 2;
         const int quarter = warp & 3;  // TMEM lane quarter this warp may access
         const int il = 32 * quarter + lane;
         const int i = qb * kBM + il;
         const bool row_ok = i < p.S;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
+        const uint32_t col_s = kColS + 64 * half;     // + 128 * b: this half's S columns
+        const uint32_t col_p = kColP + 32 * half;     // + 64 * b: this half's packed P columns
+        const uint32_t col_o = kColO + (D / 2) * half; // this half's O columns
         const float sl2 = p.scale_log2;
         const int32_t *Ch = p.vert_cols + p.vert_ptr[h];
         const int nC = p.vert_ptr[h + 1] - p.vert_ptr[h];
         const int n_i = row_ok ? lower_bound_i32(Ch, nC, i + 1) : 0;  // columns c <= i
+
+        // This half's 64-bit row mask of tile j (bit k = key column 64 * half + k).
+        // Band tiles: local diagonal bits of the plan minus excluded columns; stripe
+        // tiles: the first n_i - 128 * (j - nb) gathered columns.
+        uint32_t m_flags = 0;
+        uint64_t m_dm[4] = {0, 0, 0, 0}, m_cm[2] = {0, 0};
+        auto fetch_meta = [&](int j) {  // raw plan data of band tile j (loads only)
+            if (j < nb) {
+                const size_t t = static_cast<size_t>(tp0 + j);
+                m_flags = __ldg(p.tile_flags + t);
+                const uint64_t *dmp = p.tile_dmask + 4 * t;
+                m_dm[0] = __ldg(dmp);
+                m_dm[1] = __ldg(dmp + 1);
+                m_dm[2] = __ldg(dmp + 2);
+                m_dm[3] = __ldg(dmp + 3);
+                m_cm[0] = __ldg(p.tile_cmask + 2 * t + half);
+            }
+        };
+        auto make_mask = [&](int j, bool &full, uint64_t &bits) {
+            if (j < nb) {
+                full = (m_flags & 1u) != 0;
+                uint64_t lo, hi;
+                row_diag_mask(m_dm, il, lo, hi);
+                bits = (half ? hi : lo) & ~m_cm[0];
+                if (!row_ok) bits = 0;
+            } else {
+                const int lim_k = n_i - (j - nb) * kBN - 64 * half;  // active iff k < lim_k
+                full = lim_k >= 64;
+                bits = lim_k >= 64 ? ~0ull : (lim_k <= 0 ? 0ull : (1ull << lim_k) - 1ull);
+            }
+        };
+        bool cur_full = false;
+        uint64_t cur_bits = 0;
+        fetch_meta(0);
+        make_mask(0, cur_full, cur_bits);
+        fetch_meta(1);
+
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
         for (int j = 0; j < n && ok; ++j) {
@@ -355,42 +406,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            float sv[128];
+            float sv[64];
             {
-                uint32_t r[128];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + kColS + 128 * b + 32 * c, r + 32 * c);
+                uint32_t r[64];
+                tmem_ld32(tmem + lane_off + col_s + 128 * b, r);
+                tmem_ld32(tmem + lane_off + col_s + 128 * b + 32, r + 32);
                 tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 128; ++k) sv[k] = __uint_as_float(r[k]);
+                for (int k = 0; k < 64; ++k) sv[k] = __uint_as_float(r[k]);
             }
-            // element mask
-            if (j < nb) {
-                const uint32_t flags = __ldg(p.tile_flags + tp0 + j);
-                if (!(flags & 1u)) {
-                    const uint64_t *dmp = p.tile_dmask + 4 * static_cast<size_t>(tp0 + j);
-                    const uint64_t *cmp = p.tile_cmask + 2 * static_cast<size_t>(tp0 + j);
-                    const uint64_t dm[4] = {__ldg(dmp), __ldg(dmp + 1), __ldg(dmp + 2), __ldg(dmp + 3)};
-                    uint64_t lo, hi;
-                    row_diag_mask(dm, il, lo, hi);
-                    lo &= ~__ldg(cmp);
-                    hi &= ~__ldg(cmp + 1);
-                    if (!row_ok) lo = hi = 0;
+            // mask of the next tile from the metadata fetched one tile ahead
+            bool nxt_full = false;
+            uint64_t nxt_bits = 0;
+            if (j + 1 < n) make_mask(j + 1, nxt_full, nxt_bits);
+            if (j + 2 < n) fetch_meta(j + 2);
+
+            if (!__all_sync(0xffffffffu, cur_full)) {
 #pragma unroll
-                    for (int k = 0; k < 64; ++k) {
-                        if (!((lo >> k) & 1ull)) sv[k] = -INFINITY;
-                        if (!((hi >> k) & 1ull)) sv[64 + k] = -INFINITY;
-                    }
-                }
-            } else {
-                const int lim_k = n_i - (j - nb) * kBN;  // stripe column k active iff k < lim_k
-#pragma unroll
-                for (int k = 0; k < 128; ++k)
-                    if (k >= lim_k) sv[k] = -INFINITY;
+                for (int k = 0; k < 64; ++k)
+                    if (!((cur_bits >> k) & 1ull)) sv[k] = -INFINITY;
             }
-            float mt = sv[0];
+            float mx[8];
 #pragma unroll
-            for (int k = 1; k < 128; ++k) mt = fmaxf(mt, sv[k]);
+            for (int c = 0; c < 8; ++c) mx[c] = sv[c];
+#pragma unroll
+            for (int k = 8; k < 64; ++k) mx[k & 7] = fmaxf(mx[k & 7], sv[k]);
+            float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            // exchange the half-row maxima with the partner thread of the same row
+            bar->red_max[b][half][il] = mt;
+            mbar_arrive(&bar->xchg[quarter][b]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&bar->xchg[quarter][b], (j >> 1) & 1, lim, abort))) {
+                ok = false;
+                break;
+            }
+            mt = fmaxf(mt, bar->red_max[b][half ^ 1][il]);
             const float m_new = fmaxf(m_run, mt * sl2);
             // lazy rescale: keep a stale max unless the row max grew by more than 2^8
             const bool grow = (m_new != -INFINITY) &&
@@ -403,21 +453,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_run = m_new;
             }
             if (__any_sync(0xffffffffu, need_o)) {  // warp-uniform: O is read warp-collectively
-                // O must include P_{j-1} V_{j-1} before it is rescaled
-                if (!__all_sync(0xffffffffu, mbar_wait(&bar->o_ready, (j - 1) & 1, lim, abort))) {
+                // O must include P_{j-1} V_{j-1} before it is rescaled.  PV_{j-1} is the
+                // ((j-1) >> 1)-th completion of p_free[(j-1) & 1]; PV_{j-3}, the phase before
+                // it, completed before P_{j-1} was written, so the parity cannot alias.
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar->p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, lim, abort))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const float f = need_o ? factor : 1.0f;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < D / 64; ++c) {
                     uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + kColO + 32 * c, r);
+                    tmem_ld32(tmem + lane_off + col_o + 32 * c, r);
                     tmem_wait_ld();
 #pragma unroll
                     for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * f);
-                    tmem_st32(tmem + lane_off + kColO + 32 * c, r);
+                    tmem_st32(tmem + lane_off + col_o + 32 * c, r);
                 }
             }
             const float mref = (m_run == -INFINITY) ? 0.0f : m_run;
@@ -427,37 +479,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = false;
                 break;
             }
-            float lsum = 0.0f;
+            float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            uint32_t r[32];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r[32];
-#pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const float p0 = ex2_approx(fmaf(sv[64 * half + 2 * k], sl2, -mref));
-                    const float p1 = ex2_approx(fmaf(sv[64 * half + 2 * k + 1], sl2, -mref));
-                    lsum += p0 + p1;
-                    const __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
-                    r[k] = *reinterpret_cast<const uint32_t *>(&pk);
-                }
-                tmem_st32(tmem + lane_off + kColP + 64 * b + 32 * half, r);
+            for (int k = 0; k < 32; ++k) {
+                const float p0 = ex2_approx(fmaf(sv[2 * k], sl2, -mref));
+                const float p1 = ex2_approx(fmaf(sv[2 * k + 1], sl2, -mref));
+                ls[(2 * k) & 7] += p0;
+                ls[(2 * k + 1) & 7] += p1;
+                const __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
+                r[k] = *reinterpret_cast<const uint32_t *>(&pk);
             }
-            l_run += lsum;
+            tmem_st32(tmem + lane_off + col_p + 64 * b, r);
+            l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bar->p_full[b]);
+            cur_full = nxt_full;
+            cur_bits = nxt_bits;
         }
         if (ok) {
-            if (!mbar_wait(&bar->o_ready, (n - 1) & 1, lim, abort)) ok = false;
-            ok = __all_sync(0xffffffffu, ok);
+            // row sum = both halves' partial sums
+            bar->red_l[half][il] = l_run;
+            mbar_arrive(&bar->lxchg[quarter]);
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar->lxchg[quarter], 0, lim, abort));
+        }
+        if (ok) {
+            // O complete: PV_{n-1} done (the phase before it, PV_{n-3}, was awaited before
+            // P_{n-1} was written)
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar->p_free[(n - 1) & 1], ((n - 1) >> 1) & 1, lim, abort));
         }
         if (ok) {
             tc_fence_after();
-            const float inv = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
-            uint4 *dst = reinterpret_cast<uint4 *>(p.O + (static_cast<size_t>(h) * p.S + (row_ok ? i : 0)) * D);
+            const float l_tot = l_run + bar->red_l[half ^ 1][il];
+            const float inv = (l_tot > 0.0f) ? 1.0f / l_tot : 0.0f;
+            uint4 *dst = reinterpret_cast<uint4 *>(p.O + (static_cast<size_t>(h) * p.S + (row_ok ? i : 0)) * D) +
+                         half * (D / 16);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < D / 64; ++c) {
                 uint32_t r[32];
-                tmem_ld32(tmem + lane_off + kColO + 32 * c, r);
+                tmem_ld32(tmem + lane_off + col_o + 32 * c, r);
                 tmem_wait_ld();
                 if (row_ok) {
 #pragma unroll
@@ -474,9 +535,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (row_ok)
+            if (row_ok && half == 0)
                 p.LSE[static_cast<size_t>(h) * p.S + i] =
-                    (l_run > 0.0f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+                    (l_tot > 0.0f) ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
         } else {
             report(p.status, SSA_ERR_TIMEOUT);
             *abort = 1;
