@@ -204,7 +204,8 @@ SSA_API int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr, const in
 /* Attention forward                                                               */
 /* ------------------------------------------------------------------------------ */
 
-/* Workspace bytes of sparse_attn_fwd (the gathered stripe keys and values). */
+/* Workspace bytes of sparse_attn_fwd: a 256-byte work counter followed by the
+ * gathered stripe keys and values. */
 SSA_API size_t sparse_attn_fwd_ws_bytes(int n_heads, int max_vert, int d);
 
 /*

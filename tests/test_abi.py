@@ -34,9 +34,10 @@ def test_exports_every_declared_symbol(lib):
 def test_version_and_sizes(lib):
     assert lib.ssa_version() >= 100
     assert lib.sparse_pattern_capture_ws_bytes(512, 512) == 512 * (4 * 512 + 2) * 4
-    assert lib.sparse_attn_fwd_ws_bytes(32, 128, 128) == 2 * 32 * 128 * 128 * 2
-    assert lib.sparse_attn_fwd_ws_bytes(32, 129, 64) == 2 * 32 * 256 * 64 * 2
-    assert lib.sparse_attn_fwd_ws_bytes(4, 0, 128) == 0
+    # 256 bytes of scheduling counter + the gathered stripe keys and values
+    assert lib.sparse_attn_fwd_ws_bytes(32, 128, 128) == 256 + 2 * 32 * 128 * 128 * 2
+    assert lib.sparse_attn_fwd_ws_bytes(32, 129, 64) == 256 + 2 * 32 * 256 * 64 * 2
+    assert lib.sparse_attn_fwd_ws_bytes(4, 0, 128) == 256
     assert lib.sparse_pattern_extend_ws_bytes(32, 65536) > 32 * 512 * 8
 
 

@@ -58,7 +58,11 @@ def test_main_diagonal_returns_values(ora):
     S, d = 300, 128
     stats, (O, LSE, q, k, v) = _run([np.array([0], np.int32)], [np.zeros(0, np.int32)], S, 1, 1, d, 8,
                                     dense=True, ora=ora)
-    np.testing.assert_array_equal(O[0].view(torch.int16).cpu().numpy().view(np.uint16), v[0])
+    # P = 2^(s*scale - m) for the only retained key is 1 up to the rounding residual of
+    # the fused s*scale - m, so O = V within one bf16 ulp (the tolerance check above holds)
+    got = O[0].float().cpu().numpy()
+    want = inputs.f32_from_bf16_bits(v[0])
+    assert (np.abs(got - want) <= np.abs(want) * 2.0 ** -7).all()
 
 
 def test_stripes_only_and_empty_rows(ora):
@@ -66,8 +70,10 @@ def test_stripes_only_and_empty_rows(ora):
     diags = [np.zeros(0, np.int32), np.arange(400, 420, dtype=np.int32)]
     verts = [np.array([0], np.int32), np.array([650], np.int32)]
     stats, (O, LSE, q, k, v) = _run(diags, verts, S, 2, 2, d, 9, dense=True, ora=ora)
-    o = O.view(torch.int16).cpu().numpy().view(np.uint16)
-    assert (o[0] == v[0, 0]).all()  # c = 0 only: every row returns V[0]
+    # c = 0 only: every row returns V[0] (within one bf16 ulp, as above)
+    got = O[0].float().cpu().numpy()
+    want = np.broadcast_to(inputs.f32_from_bf16_bits(v[0, 0]), got.shape)
+    assert (np.abs(got - want) <= np.abs(want) * 2.0 ** -7).all()
     assert np.isneginf(LSE[1, :400].cpu().numpy()).all()
 
 
