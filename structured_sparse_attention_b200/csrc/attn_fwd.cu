@@ -11,34 +11,42 @@
 //   stripe_gather_kernel     K_C[h][k] = K[kv(h)][C_h[k]], V_C likewise, zero-padded to
 //                            a multiple of 128 rows (the vertical-pattern columns of
 //                            every head packed into dense tiles)
-//   sparse_attn_fwd_kernel   persistent: one CTA per SM takes work items (head,
-//                            128-row query block) from a global counter, heaviest
-//                            query blocks first.  Roles:
-//     warp 8 lane 0  scheduler + TMA producer of Q and K tiles (band tiles from K at
-//                    the plan's key-tile index, then stripe tiles from K_C)
-//     warp 8 lane 1  TMA producer of V tiles
-//     warp 9         allocates tensor memory; lane 0 issues tcgen05.mma:
-//                    S_t = Q K_t^T into a double-buffered TMEM S, O += P_t V_t with P
-//                    read from TMEM.  QK^T of tile t+2 is issued as soon as the softmax
-//                    has read S_t, ahead of PV of tile t.
-//     warps 0-7      softmax, two threads per query row (key columns 0-63 / 64-127 and
-//                    the matching O halves), software-pipelined one tile ahead:
-//                    tcgen05.ld S, element mask from the plan (FULL tiles skip it), row
-//                    max exchanged through shared memory at a named barrier, online
-//                    max/sum in fp32 (log2 domain, packed f32x2 arithmetic), P as bf16
-//                    into TMEM, lazy O rescale (only when the max grows by > 2^8);
-//                    epilogue O / l -> bf16 and LSE.
-// Tensor memory (512 columns): S0 0..127, S1 128..255, P0 256..319, P1 320..383,
-// O 384..384+d-1.  P has its own buffers so a QK^T never overwrites a P being read.
+//   sparse_attn_fwd_kernel   persistent: one CTA per SM takes work items from a global
+//                            counter.  An item is a PAIR of consecutive 128-row query
+//                            blocks (2p, 2p+1) of one head; the CTA walks the merged
+//                            key-tile sequence of the two blocks (band tiles in
+//                            ascending key-tile order, then stripe tiles), so a key/value
+//                            tile wanted by both blocks is staged once and feeds both.
+//     warp 8 lane 0  scheduler (work counter -> item ring), TMA producer of the two Q
+//                    tiles and of the K tiles of the merged sequence; each K stage
+//                    carries a flag word: which slot uses it, first/last tile of a
+//                    slot within the item, end of work
+//     warp 8 lane 1  TMA producer of the V tiles of the same sequence
+//     warp 9         allocates tensor memory; lane 0 issues tcgen05.mma for both slots
+//                    from a polling loop: S_s = Q_s K^T into TMEM, O_s += P_s V with P_s
+//                    read from TMEM.  P_s is written over the first half of S_s, so the
+//                    QK^T of a slot's next tile is always issued after the PV of its
+//                    current tile (tcgen05.mma operations of one thread execute in issue
+//                    order); the two slots interleave, so one slot's MMAs run while the
+//                    other slot's softmax works.
+//     warps 0-3      softmax of slot 0 (query block 2p), one thread per query row
+//     warps 4-7      softmax of slot 1 (query block 2p+1)
+//                    tcgen05.ld S (128 columns), element mask from the plan (FULL
+//                    tiles skip it), online max/sum in fp32 (log2 domain, packed f32x2
+//                    arithmetic), P as bf16 into TMEM, lazy O rescale (only when the
+//                    max grows by > 2^8); epilogue O / l -> bf16 and LSE.
+// Tensor memory (512 columns): S0 0..127, S1 128..255, O0 256.., O1 256+d...
 //
-// Barrier phases follow global counters (tiles t across items, items m, non-empty
-// items e).  Every wait is on a barrier whose previous phase is known to be complete,
-// so a parity never aliases two phases back.  Every wait is bounded: on expiry the
+// Every barrier is waited on with a counter of its own completions, and every wait
+// happens only after the previous completion of the same barrier was observed by the
+// waiter, so a parity never aliases two phases.  Every wait is bounded: on expiry the
 // kernel records SSA_ERR_TIMEOUT, stops every role, drains its own copies and MMAs,
 // frees tensor memory and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
+
+#include <climits>
 
 #include "common.cuh"
 
@@ -47,59 +55,75 @@ namespace {
 
 constexpr int kBM = SSA_BLOCK;
 constexpr int kBN = SSA_BLOCK;
-// Warps 0-7 softmax (two warpgroups), warp 8 TMA producers, warp 9 MMA issuer, warps
-// 10-11 idle.  Registers are rebalanced with setmaxnreg: the launch gives every thread
-// kLaunchRegs; the TMA/MMA warpgroup drops to kCtrlRegs and the softmax warpgroups
-// rise to kSoftmaxRegs, which together use exactly the launch allocation.
+// Warps 0-7 softmax (one warpgroup per slot), warp 8 TMA producers, warp 9 MMA issuer,
+// warps 10-11 idle.  Registers are rebalanced with setmaxnreg: the launch gives every
+// thread kLaunchRegs; the TMA/MMA warpgroup drops to kCtrlRegs and the softmax
+// warpgroups rise to kSoftmaxRegs, which together use exactly the launch allocation.
 constexpr int kThreads = 384;
-constexpr int kSoftmaxThreads = 256;
+constexpr int kSlotThreads = 128;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kWarpTma = 8, kWarpMma = 9;
 constexpr int kLaunchRegs = 168, kCtrlRegs = 56, kSoftmaxRegs = 224;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kCtrlRegs <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr int kRing = 4;  // work-item descriptors in flight
+constexpr int kMaxStages = 6;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;
 constexpr int kBoxBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr int64_t kDrainLimitNs = 1000000000LL;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if the max grows by > 256x
 constexpr size_t kCounterBytes = 256;     // work counter at the start of the workspace
+constexpr int kMaxSmem = 232448;          // 227 KB opt-in per block
+
+// Flag word of a K stage (one merged step).  Slot s: bit s = the slot uses this key
+// tile, bit 2+s = its first tile of the item, bit 4+s = its last tile of the item.
+constexpr uint32_t kStepEnd = 64;
+__host__ __device__ constexpr uint32_t f_in(int s) { return 1u << s; }
+__host__ __device__ constexpr uint32_t f_first(int s) { return 4u << s; }
+__host__ __device__ constexpr uint32_t f_last(int s) { return 16u << s; }
 
 template <int D>
 struct Cfg {
-    static constexpr int NK = (D == 128) ? 3 : 4;  // K pipeline stages
-    static constexpr int NV = (D == 128) ? 2 : 3;  // V pipeline stages
+    // K and V pipeline stages.  One slot's QK^T can run at most NK steps ahead of the
+    // other's, and a pending PV sits one step behind its QK^T, so NV >= NK + 1 keeps
+    // every V tile a slot waits for inside the V window (no circular wait).
+    static constexpr int NK = (D == 128) ? 2 : 4;
+    static constexpr int NV = (D == 128) ? 3 : 5;
     static constexpr int BOXES = D / 64;
     static constexpr int TILE_BYTES = BOXES * kBoxBytes;
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + TILE_BYTES;
+    static constexpr int OFF_Q = 0;  // Q tile of slot 0, then slot 1
+    static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
     static constexpr int OFF_V = OFF_K + NK * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + NV * TILE_BYTES;
-    // barriers + alignment slack; at least 120 KB so that a single CTA (and its 512
-    // tensor-memory columns) occupies an SM
-    static constexpr int SMEM_RAW = OFF_BAR + 4096 + 1024;
-    static constexpr int SMEM_BYTES = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
+    static constexpr int SMEM_BYTES = OFF_BAR + 1024 + 1024;  // barrier block + alignment slack
+    static constexpr uint32_t COL_O = 256;                      // O_s at COL_O + D s
+    static_assert(NK <= kMaxStages && NV <= kMaxStages, "too many stages");
+    static_assert(NV >= NK + 1, "V window must exceed the K window");
+    static_assert(SMEM_BYTES <= kMaxSmem, "shared memory budget exceeded");
 };
 
 struct ItemDesc {
-    int h, qb, g, tp0, nb, n, stripe_lo;  // n < 0 marks the end of the work
+    int h, g, end;
+    int qb[2];   // query block of each slot (-1: none)
+    int tp0[2];  // first plan tile of the block
+    int nb[2];   // band tiles
+    int ns[2];   // stripe tiles
+    int slo[2];  // stripe count of the previous block (columns < 128 qb)
 };
 
 struct Shared {
     uint64_t item_full[kRing], item_empty[kRing];
-    uint64_t q_full, q_empty;
-    uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-    uint64_t s_full[2], s_free[2], p_full[2], p_free[2];
-    uint64_t o_free;
+    uint64_t q_full[2], q_empty[2];
+    uint64_t k_full[kMaxStages], k_empty[kMaxStages];
+    uint64_t v_full[kMaxStages], v_empty[kMaxStages];
+    uint64_t s_full[2], p_full[2], o_full[2];
     uint64_t mma_drain, softmax_done;
     ItemDesc items[kRing];
+    uint32_t kflags[kMaxStages];
     uint32_t tmem_base;
     int abort;
-    float red_max[2][2][128];  // [tile parity][column half][row]
-    float red_l[2][128];       // [column half][row]
 };
-static_assert(sizeof(Shared) <= 4096, "barrier block too large");
+static_assert(sizeof(Shared) <= 1024, "barrier block too large");
 
 struct AttnParams {
     int S, H, Hkv, nqb, npad;
@@ -174,28 +198,105 @@ __global__ void __launch_bounds__(256) stripe_gather_kernel(const uint16_t *__re
 }
 
 // ---------------------------------------------------------------------------------
-// Attention forward (persistent)
+// Attention forward (persistent, two query blocks per work item)
 // ---------------------------------------------------------------------------------
 
-// Work item idx -> descriptor.  Items run from the last query block down (later
-// blocks hold more tiles under causal patterns) with the heads of one block side by
-// side, so heads of a KV group read the same key tiles close together in time.
-__device__ ItemDesc make_item(const AttnParams &p, int idx) {
+// Work item idx -> descriptor of the pair of query blocks (2 pq, 2 pq + 1) of head h.
+// Items run from the last pair down (later blocks hold more tiles under causal
+// patterns) with the heads of one pair side by side, so heads of a KV group read the
+// same key tiles close together in time.
+__device__ ItemDesc make_pair(const AttnParams &p, int idx) {
     ItemDesc d;
-    d.qb = p.nqb - 1 - idx / p.H;
+    const int npair = (p.nqb + 1) >> 1;
+    const int pq = npair - 1 - idx / p.H;
     d.h = idx % p.H;
     d.g = kv_head(p, d.h);
-    const int it = d.h * p.nqb + d.qb;
-    d.tp0 = p.tile_ptr[it];
-    d.nb = p.tile_ptr[it + 1] - d.tp0;
-    const int sc = p.stripe_cnt[it];
-    d.stripe_lo = d.qb > 0 ? p.stripe_cnt[it - 1] : 0;
-    d.n = d.nb + (sc + kBN - 1) / kBN;
-    if (d.g < 0 || d.g >= p.Hkv) {
-        report(p.status, SSA_ERR_INVALID);
-        d.n = 0;  // still writes O = 0, LSE = -inf
+    d.end = 0;
+    const bool bad = d.g < 0 || d.g >= p.Hkv;
+    if (bad) report(p.status, SSA_ERR_INVALID);  // its rows still get O = 0, LSE = -inf
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        const int qb = 2 * pq + s;
+        d.qb[s] = -1;
+        d.tp0[s] = d.nb[s] = d.ns[s] = d.slo[s] = 0;
+        if (qb >= p.nqb) continue;
+        d.qb[s] = qb;
+        const int it = d.h * p.nqb + qb;
+        d.tp0[s] = __ldg(p.tile_ptr + it);
+        d.slo[s] = qb > 0 ? __ldg(p.stripe_cnt + it - 1) : 0;
+        if (!bad) {
+            d.nb[s] = __ldg(p.tile_ptr + it + 1) - d.tp0[s];
+            d.ns[s] = (__ldg(p.stripe_cnt + it) + kBN - 1) / kBN;
+        }
     }
     return d;
+}
+
+// The merged key-tile sequence of an item: band tiles of both blocks in ascending key
+// tile (a tile listed by both is one step), then the stripe tiles (block 2p+1 holds at
+// least as many stripe columns as block 2p).  The next band entry of each block is
+// loaded one step ahead so the producers do not wait on it.
+struct Steps {
+    const int32_t *kb[2];
+    int nb[2], ns[2], i[2], a[2], an[2];
+    int js;
+    bool started[2];
+};
+
+__device__ __forceinline__ void steps_init(Steps &st, const AttnParams &p, const ItemDesc &d) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        st.kb[s] = p.tile_kb + d.tp0[s];
+        st.nb[s] = d.nb[s];
+        st.ns[s] = d.ns[s];
+        st.i[s] = 0;
+        st.a[s] = d.nb[s] > 0 ? __ldg(st.kb[s]) : INT_MAX;
+        st.an[s] = d.nb[s] > 1 ? __ldg(st.kb[s] + 1) : INT_MAX;
+        st.started[s] = false;
+    }
+    st.js = 0;
+}
+
+// Next step of the sequence: key-tile row, whether it is a band tile (else a stripe
+// tile of K_C / V_C) and the slot flags.  Returns false after the last step.
+__device__ __forceinline__ bool steps_next(Steps &st, bool &band, int &row0, uint32_t &flags) {
+    flags = 0;
+    if (st.a[0] != INT_MAX || st.a[1] != INT_MAX) {
+        const int kb = min(st.a[0], st.a[1]);
+        band = true;
+        row0 = kb * kBN;
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            if (st.a[s] != kb) continue;
+            flags |= f_in(s);
+            if (!st.started[s]) {
+                flags |= f_first(s);
+                st.started[s] = true;
+            }
+            ++st.i[s];
+            st.a[s] = st.an[s];
+            st.an[s] = (st.i[s] + 1 < st.nb[s]) ? __ldg(st.kb[s] + st.i[s] + 1) : INT_MAX;
+            if (st.i[s] == st.nb[s] && st.ns[s] == 0) flags |= f_last(s);
+        }
+        return true;
+    }
+    if (st.js < max(st.ns[0], st.ns[1])) {
+        band = false;
+        row0 = st.js * kBN;
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            if (st.js >= st.ns[s]) continue;
+            flags |= f_in(s);
+            if (!st.started[s]) {
+                flags |= f_first(s);
+                st.started[s] = true;
+            }
+            if (st.js == st.ns[s] - 1) flags |= f_last(s);
+        }
+        ++st.js;
+        return true;
+    }
+    return false;
 }
 
 template <int D>
@@ -212,32 +313,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     Shared *sh = reinterpret_cast<Shared *>(smem + C::OFF_BAR);
     volatile int *abort = &sh->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_items = p.H * p.nqb;
+    const int n_items = p.H * ((p.nqb + 1) >> 1);
 
     if (threadIdx.x == 0) {
         for (int r = 0; r < kRing; ++r) {
             mbar_init(&sh->item_full[r], 1);
-            mbar_init(&sh->item_empty[r], 2 + kSoftmaxWarps);  // V lane, MMA, softmax warps
+            mbar_init(&sh->item_empty[r], 1 + kSoftmaxWarps);  // V lane, softmax warps
         }
-        mbar_init(&sh->q_full, 1);
-        mbar_init(&sh->q_empty, 1);
-        for (int s = 0; s < C::NK; ++s) {
-            mbar_init(&sh->k_full[s], 1);
-            mbar_init(&sh->k_empty[s], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sh->q_full[s], 1);
+            mbar_init(&sh->q_empty[s], 1);
+            mbar_init(&sh->s_full[s], 1);
+            mbar_init(&sh->p_full[s], kSlotThreads);
+            mbar_init(&sh->o_full[s], 1);
         }
-        for (int s = 0; s < C::NV; ++s) {
-            mbar_init(&sh->v_full[s], 1);
-            mbar_init(&sh->v_empty[s], 1);
+        for (int st = 0; st < C::NK; ++st) {
+            mbar_init(&sh->k_full[st], 1);
+            mbar_init(&sh->k_empty[st], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&sh->s_full[b], 1);
-            mbar_init(&sh->s_free[b], kSoftmaxThreads);
-            mbar_init(&sh->p_full[b], kSoftmaxThreads);
-            mbar_init(&sh->p_free[b], 1);
+        for (int st = 0; st < C::NV; ++st) {
+            mbar_init(&sh->v_full[st], 1);
+            mbar_init(&sh->v_empty[st], 1);
         }
-        mbar_init(&sh->o_free, kSoftmaxThreads);
         mbar_init(&sh->mma_drain, 1);
-        mbar_init(&sh->softmax_done, kSoftmaxThreads);
+        mbar_init(&sh->softmax_done, 2 * kSlotThreads);
         sh->abort = 0;
         fence_barrier_init();
     }
@@ -255,12 +354,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
       if (warp == kWarpTma) {
         if (lane == 0) {
-            // --------------------- scheduler + Q/K producer ---------------------
+            // ------------------ scheduler + Q and K producer ------------------
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmKC);
             bool ok = true;
-            int m = 0, e = 0, t = 0;
+            int m = 0, tk = 0;
+            int qn[2] = {0, 0};
             while (ok) {
                 const int idx = atomicAdd(p.work_counter, 1);
                 const int slot = m % kRing;
@@ -270,40 +370,58 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ItemDesc d;
                 if (idx < n_items) {
-                    d = make_item(p, idx);
+                    d = make_pair(p, idx);
                 } else {
-                    d.n = -1;
+                    d.end = 1;
                 }
                 sh->items[slot] = d;
                 mbar_arrive(&sh->item_full[slot]);  // release: the descriptor is visible
                 ++m;
-                if (d.n < 0) break;
-                if (d.n == 0) continue;
-                // Q block of this item, once the previous item's last QK^T is done
-                if (e >= 1 && !mbar_wait(&sh->q_empty, (e - 1) & 1, lim, abort)) {
-                    ok = false;
-                    break;
+                if (d.end) break;
+                // Q tiles of the slots that have work, each once the previous item's last
+                // QK^T of that slot is done
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {
+                    if (!ok || d.nb[s] + d.ns[s] == 0) continue;
+                    if (qn[s] >= 1 && !mbar_wait(&sh->q_empty[s], (qn[s] - 1) & 1, lim, abort)) {
+                        ok = false;
+                        continue;
+                    }
+                    uint8_t *sQ = smem + C::OFF_Q + s * C::TILE_BYTES;
+                    mbar_arrive_expect_tx(&sh->q_full[s], C::TILE_BYTES);
+                    for (int b = 0; b < C::BOXES; ++b)
+                        tma_load_3d(sQ + b * kBoxBytes, &tmQ, &sh->q_full[s], 64 * b, d.qb[s] * kBM, d.h);
+                    ++qn[s];
                 }
-                uint8_t *sQ = smem + C::OFF_Q;
-                mbar_arrive_expect_tx(&sh->q_full, C::TILE_BYTES);
-                for (int b = 0; b < C::BOXES; ++b)
-                    tma_load_3d(sQ + b * kBoxBytes, &tmQ, &sh->q_full, 64 * b, d.qb * kBM, d.h);
-                ++e;
-                int kb_next = d.nb > 0 ? __ldg(p.tile_kb + d.tp0) : 0;
-                for (int j = 0; j < d.n; ++j, ++t) {
-                    const int s = t % C::NK;
-                    const int kb = kb_next;
-                    if (j + 1 < d.nb) kb_next = __ldg(p.tile_kb + d.tp0 + j + 1);
-                    if (t >= C::NK && !mbar_wait(&sh->k_empty[s], ((t / C::NK) - 1) & 1, lim, abort)) {
+                if (!ok) break;
+                Steps st;
+                steps_init(st, p, d);
+                bool band;
+                int row0;
+                uint32_t fl;
+                while (steps_next(st, band, row0, fl)) {
+                    const int si = tk % C::NK;
+                    if (tk >= C::NK && !mbar_wait(&sh->k_empty[si], ((tk / C::NK) - 1) & 1, lim, abort)) {
                         ok = false;
                         break;
                     }
-                    const bool band = j < d.nb;
-                    uint8_t *dst = smem + C::OFF_K + s * C::TILE_BYTES;
-                    mbar_arrive_expect_tx(&sh->k_full[s], C::TILE_BYTES);
+                    sh->kflags[si] = fl;
+                    uint8_t *dst = smem + C::OFF_K + si * C::TILE_BYTES;
+                    mbar_arrive_expect_tx(&sh->k_full[si], C::TILE_BYTES);
                     for (int b = 0; b < C::BOXES; ++b)
-                        tma_load_3d(dst + b * kBoxBytes, band ? &tmK : &tmKC, &sh->k_full[s], 64 * b,
-                                    band ? kb * kBN : (j - d.nb) * kBN, band ? d.g : d.h);
+                        tma_load_3d(dst + b * kBoxBytes, band ? &tmK : &tmKC, &sh->k_full[si], 64 * b, row0,
+                                    band ? d.g : d.h);
+                    ++tk;
+                }
+            }
+            if (ok) {  // end-of-work step for the MMA issuer (no data)
+                const int si = tk % C::NK;
+                if (tk >= C::NK && !mbar_wait(&sh->k_empty[si], ((tk / C::NK) - 1) & 1, lim, abort)) {
+                    ok = false;
+                } else {
+                    sh->kflags[si] = kStepEnd;
+                    mbar_arrive(&sh->k_full[si]);
+                    ++tk;
                 }
             }
             if (!ok) {
@@ -311,15 +429,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *abort = 1;
             }
             // Drain: never leave the CTA with a copy still writing shared memory.
-            if (e >= 1) mbar_wait(&sh->q_full, (e - 1) & 1, kDrainLimitNs, nullptr);
-            for (int u = (t > C::NK ? t - C::NK : 0); u < t; ++u)
+            for (int s = 0; s < 2; ++s)
+                if (qn[s] >= 1) mbar_wait(&sh->q_full[s], (qn[s] - 1) & 1, kDrainLimitNs, nullptr);
+            for (int u = (tk > C::NK ? tk - C::NK : 0); u < tk; ++u)
                 mbar_wait(&sh->k_full[u % C::NK], (u / C::NK) & 1, kDrainLimitNs, nullptr);
         } else if (lane == 1) {
             // ----------------------------- V producer ----------------------------
             prefetch_tmap(&tmV);
             prefetch_tmap(&tmVC);
             bool ok = true;
-            int m = 0, t = 0;
+            int m = 0, tv = 0;
             while (ok) {
                 const int slot = m % kRing;
                 if (!mbar_wait(&sh->item_full[slot], (m / kRing) & 1, lim, abort)) {
@@ -329,29 +448,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const ItemDesc d = sh->items[slot];
                 mbar_arrive(&sh->item_empty[slot]);
                 ++m;
-                if (d.n < 0) break;
-                int kb_next = d.nb > 0 ? __ldg(p.tile_kb + d.tp0) : 0;
-                for (int j = 0; j < d.n; ++j, ++t) {
-                    const int s = t % C::NV;
-                    const int kb = kb_next;
-                    if (j + 1 < d.nb) kb_next = __ldg(p.tile_kb + d.tp0 + j + 1);
-                    if (t >= C::NV && !mbar_wait(&sh->v_empty[s], ((t / C::NV) - 1) & 1, lim, abort)) {
+                if (d.end) break;
+                Steps st;
+                steps_init(st, p, d);
+                bool band;
+                int row0;
+                uint32_t fl;
+                while (steps_next(st, band, row0, fl)) {
+                    const int si = tv % C::NV;
+                    if (tv >= C::NV && !mbar_wait(&sh->v_empty[si], ((tv / C::NV) - 1) & 1, lim, abort)) {
                         ok = false;
                         break;
                     }
-                    const bool band = j < d.nb;
-                    uint8_t *dst = smem + C::OFF_V + s * C::TILE_BYTES;
-                    mbar_arrive_expect_tx(&sh->v_full[s], C::TILE_BYTES);
+                    uint8_t *dst = smem + C::OFF_V + si * C::TILE_BYTES;
+                    mbar_arrive_expect_tx(&sh->v_full[si], C::TILE_BYTES);
                     for (int b = 0; b < C::BOXES; ++b)
-                        tma_load_3d(dst + b * kBoxBytes, band ? &tmV : &tmVC, &sh->v_full[s], 64 * b,
-                                    band ? kb * kBN : (j - d.nb) * kBN, band ? d.g : d.h);
+                        tma_load_3d(dst + b * kBoxBytes, band ? &tmV : &tmVC, &sh->v_full[si], 64 * b, row0,
+                                    band ? d.g : d.h);
+                    ++tv;
                 }
             }
             if (!ok) {
                 report(p.status, SSA_ERR_TIMEOUT);
                 *abort = 1;
             }
-            for (int u = (t > C::NV ? t - C::NV : 0); u < t; ++u)
+            for (int u = (tv > C::NV ? tv - C::NV : 0); u < tv; ++u)
                 mbar_wait(&sh->v_full[u % C::NV], (u / C::NV) & 1, kDrainLimitNs, nullptr);
         }
       } else if (warp == kWarpMma) {
@@ -359,102 +480,89 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t IDESC_QK = idesc_bf16(kBM, kBN, false);
             constexpr uint32_t IDESC_PV = idesc_bf16(kBM, D, true);
-            const uint32_t sQ = smem_u32(smem + C::OFF_Q);
             bool ok = true;
-            // Two cursors over the global tile sequence: QK^T (item mq, tile jq, global
-            // tile tq) runs up to two tiles ahead of PV (item mp, tile jp, global tile tp).
-            // eq / ep count non-empty items started by each cursor.  Readiness is polled
-            // without blocking and a ready PV always goes first: the softmax warps (and
-            // the epilogue) wait for PVs, never for a QK^T of a later tile.
-            int mq = 0, jq = 0, tq = 0, eq = 0, nq = 0;
-            int mp = 0, jp = 0, tp = 0, ep = 0;
-            bool q_loaded = false, q_end = false;
+            // K and V stages are observed strictly in order (kobs, vobs) and released in
+            // order (krel, vrel) once neither slot needs them.  Per slot: qk_u = next
+            // step to examine, pend = a QK^T issued whose PV is not, pv_u its step.
+            int kobs = 0, vobs = 0, krel = 0, vrel = 0;
+            int qk_u[2] = {0, 0}, pv_u[2] = {0, 0}, pcnt[2] = {0, 0}, qcnt[2] = {0, 0};
+            bool pend[2] = {false, false}, fin[2] = {false, false};
+            bool pv_first[2] = {false, false}, pv_last[2] = {false, false};
             uint64_t t_progress = global_timer_ns();
             while (true) {
                 bool progress = false;
-                // QK cursor: load descriptors until a tile is available (never more than
-                // kRing - 1 items ahead of the PV cursor, whose ring slot it would need)
-                while (!q_end && !(q_loaded && jq < nq)) {
-                    if (q_loaded) {
-                        ++mq;
-                        jq = 0;
-                        q_loaded = false;
-                    }
-                    if (mq - mp >= kRing - 1) break;
-                    if (!mbar_test(&sh->item_full[mq % kRing], (mq / kRing) & 1)) break;
-                    nq = sh->items[mq % kRing].n;
-                    q_loaded = true;
-                    if (nq < 0) q_end = true;
+                if (kobs < krel + C::NK && mbar_test(&sh->k_full[kobs % C::NK], (kobs / C::NK) & 1)) {
+                    ++kobs;
                     progress = true;
                 }
-                // PV cursor: step over empty or finished items, releasing their slots
-                bool pv_end = false;
-                while (mp < mq || (q_loaded && mp == mq)) {
-                    const int np = sh->items[mp % kRing].n;
-                    if (np < 0) {
-                        pv_end = true;
-                        break;
-                    }
-                    if (jp < np) break;
-                    mbar_arrive(&sh->item_empty[mp % kRing]);
-                    ++mp;
-                    jp = 0;
+                if (vobs < vrel + C::NV && mbar_test(&sh->v_full[vobs % C::NV], (vobs / C::NV) & 1)) {
+                    ++vobs;
                     progress = true;
                 }
-                if (pv_end && tp == tq) break;  // every MMA issued
-                if (tp < tq) {
-                    // ---- PV of tile tp (item mp, tile jp) ----
-                    const int b = tp & 1, s = tp % C::NV;
-                    // the previous item's epilogue must have read O before PV overwrites it
-                    const bool o_ok = !(jp == 0 && ep >= 1) || mbar_test(&sh->o_free, (ep - 1) & 1);
-                    if (o_ok && mbar_test(&sh->p_full[b], (tp >> 1) & 1) &&
-                        mbar_test(&sh->v_full[s], (tp / C::NV) & 1)) {
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {
+                    // PV of the pending tile once its P is in TMEM and its V tile landed
+                    if (pend[s] && pv_u[s] < vobs && mbar_test(&sh->p_full[s], pcnt[s] & 1)) {
                         tc_fence_after();
-                        const uint32_t sV = smem_u32(smem + C::OFF_V + s * C::TILE_BYTES);
+                        const uint32_t sV = smem_u32(smem + C::OFF_V + (pv_u[s] % C::NV) * C::TILE_BYTES);
 #pragma unroll
                         for (int kk = 0; kk < kBN / 16; ++kk) {
                             // B = V tile, MN-major: 16 keys per step (2 x 8-row groups of 128 B)
                             const uint64_t bd = sdesc(sV + kk * 2048, kBoxBytes, 1024);
-                            umma_ts(tmem + kColO, tmem + kColP + 64 * b + 8 * kk, bd, IDESC_PV,
-                                    (jp > 0 || kk > 0) ? 1u : 0u);
+                            umma_ts(tmem + C::COL_O + D * s, tmem + 128 * s + 8 * kk, bd, IDESC_PV,
+                                    (!pv_first[s] || kk > 0) ? 1u : 0u);
                         }
-                        // p_free[b] completes once per PV that read P[b]: PV_b, PV_{b+2}, ...
-                        // It doubles as "O includes tile tp" for the softmax warps.
-                        umma_commit(&sh->p_free[b]);
-                        umma_commit(&sh->v_empty[s]);
-                        if (jp == 0) ++ep;
-                        ++jp;
-                        ++tp;
-                        t_progress = global_timer_ns();
-                        continue;
+                        if (pv_last[s]) umma_commit(&sh->o_full[s]);  // O_s of the item complete
+                        pend[s] = false;
+                        ++pcnt[s];
+                        progress = true;
                     }
-                }
-                if (!q_end && q_loaded && jq < nq && tq <= tp + 2) {
-                    // ---- QK^T of tile tq (item mq, tile jq) ----
-                    const int s = tq % C::NK, b = tq & 1;
-                    // S[b] is free once the softmax has read S_{tq-2}
-                    if ((jq != 0 || mbar_test(&sh->q_full, eq & 1)) &&
-                        mbar_test(&sh->k_full[s], (tq / C::NK) & 1) &&
-                        (tq < 2 || mbar_test(&sh->s_free[b], ((tq - 2) >> 1) & 1))) {
-                        tc_fence_after();
-                        const uint32_t sK = smem_u32(smem + C::OFF_K + s * C::TILE_BYTES);
+                    // QK^T of the slot's next tile (only after the PV that reads P_s, which
+                    // shares the S_s columns)
+                    if (!pend[s] && !fin[s] && qk_u[s] < kobs) {
+                        const uint32_t f = sh->kflags[qk_u[s] % C::NK];
+                        if (f & kStepEnd) {
+                            fin[s] = true;
+                            progress = true;
+                        } else if (!(f & f_in(s))) {
+                            ++qk_u[s];
+                            progress = true;
+                        } else if (!(f & f_first(s)) || mbar_test(&sh->q_full[s], qcnt[s] & 1)) {
+                            tc_fence_after();
+                            const uint32_t sQ = smem_u32(smem + C::OFF_Q + s * C::TILE_BYTES);
+                            const uint32_t sK = smem_u32(smem + C::OFF_K + (qk_u[s] % C::NK) * C::TILE_BYTES);
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            // A = Q, B = K tile, both K-major: 16 elements = 32 B per step
-                            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                            umma_ss(tmem + kColS + 128 * b, sdesc(sQ + off, 16, 1024),
-                                    sdesc(sK + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                // A = Q, B = K tile, both K-major: 16 elements = 32 B per step
+                                const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                                umma_ss(tmem + 128 * s, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024),
+                                        IDESC_QK, kk > 0 ? 1u : 0u);
+                            }
+                            umma_commit(&sh->s_full[s]);
+                            if (f & f_last(s)) umma_commit(&sh->q_empty[s]);  // Q_s no longer read
+                            if (f & f_first(s)) ++qcnt[s];
+                            pend[s] = true;
+                            pv_u[s] = qk_u[s];
+                            pv_first[s] = (f & f_first(s)) != 0;
+                            pv_last[s] = (f & f_last(s)) != 0;
+                            ++qk_u[s];
+                            progress = true;
                         }
-                        umma_commit(&sh->s_full[b]);
-                        umma_commit(&sh->k_empty[s]);
-                        if (jq == nq - 1) umma_commit(&sh->q_empty);  // Q of this item no longer read
-                        if (jq == 0) ++eq;
-                        ++jq;
-                        ++tq;
-                        t_progress = global_timer_ns();
-                        continue;
                     }
                 }
+                // release stages no slot needs any more (each commit completes once the
+                // MMAs issued so far, which include every reader of the stage, are done)
+                const int kf = min(qk_u[0], qk_u[1]);
+                while (krel < kf) {
+                    umma_commit(&sh->k_empty[krel % C::NK]);
+                    ++krel;
+                }
+                const int vf = min(pend[0] ? pv_u[0] : qk_u[0], pend[1] ? pv_u[1] : qk_u[1]);
+                while (vrel < vf) {
+                    umma_commit(&sh->v_empty[vrel % C::NV]);
+                    ++vrel;
+                }
+                if (fin[0] && fin[1] && !pend[0] && !pend[1]) break;
                 if (progress) {
                     t_progress = global_timer_ns();
                     continue;
@@ -483,38 +591,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         // -------------------------------- softmax / epilogue -------------------------------
-        // Two threads per query row: warps 0-3 take key columns 0..63 of every tile,
-        // warps 4-7 columns 64..127 (and the matching halves of O).  The two warps of a
-        // row quarter exchange each tile's half-row maxima through shared memory at a
-        // named barrier, so both scale by the same reference; each keeps its own partial
-        // row sum until the epilogue.  The loop is software-pipelined: while the exps of
-        // tile j run (MUFU-bound), tile j+1 is loaded, masked and reduced.
-        // A failed wait never leaves a warp early: it marks `good` false, raises the
-        // abort flag and is carried into the next named-barrier reduction, where both
-        // warps of the pair leave together.
-        const int half = warp >> 2;
-        const int quarter = warp & 3;  // TMEM lane quarter this warp may access
-        const int bar_id = 1 + quarter;
+        // Warpgroup s owns slot s: thread il of the warpgroup owns query row 128 qb + il
+        // and TMEM lane il (warp w may only touch lanes 32 (w % 4) ..).
+        const int s = warp >> 2;
+        const int quarter = warp & 3;
         const int il = 32 * quarter + lane;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
-        const uint32_t col_s = kColS + 64 * half;       // + 128 * b: this half's S columns
-        const uint32_t col_p = kColP + 32 * half;       // + 64 * b: this half's packed P columns
-        const uint32_t col_o = kColO + (D / 2) * half;  // this half's O columns
+        const uint32_t tS = tmem + lane_off + 128u * s;           // S_s; P_s in its first 64 columns
+        const uint32_t tO = tmem + lane_off + C::COL_O + D * s;   // O_s
         const float sl2 = p.scale_log2;
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
+        constexpr uint32_t kNegInf = 0xff800000u;
         bool ok = true;
-        bool good = true;  // sticky: false after any failed wait in this warp
-        auto fail = [&]() {
-            good = false;
-            *abort = 1;
-        };
-        int m = 0, e = 0, t = 0;
+        int m = 0, tcnt = 0, icnt = 0;
         while (true) {
             const int slot = m % kRing;
-            if (good && !__all_sync(0xffffffffu, mbar_wait(&sh->item_full[slot], (m / kRing) & 1, lim, abort)))
-                fail();
-            // both warps of the pair take every item (or leave) together
-            if (!bar_and(bar_id, 64, good)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&sh->item_full[slot], (m / kRing) & 1, lim, abort))) {
                 ok = false;
                 break;
             }
@@ -522,176 +614,108 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh->item_empty[slot]);
             ++m;
-            if (d.n < 0) break;
-            const int i = d.qb * kBM + il;
+            if (d.end) break;
+            const int qb = s ? d.qb[1] : d.qb[0];
+            if (qb < 0) continue;
+            const int nb = s ? d.nb[1] : d.nb[0];
+            const int ns = s ? d.ns[1] : d.ns[0];
+            const int tp0 = s ? d.tp0[1] : d.tp0[0];
+            const int slo = s ? d.slo[1] : d.slo[0];
+            const int n = nb + ns;
+            const int i = qb * kBM + il;
             const bool row_ok = i < p.S;
-            uint4 *orow = reinterpret_cast<uint4 *>(p.O + (static_cast<size_t>(d.h) * p.S + (row_ok ? i : 0)) * D) +
-                          half * (D / 16);
-            if (d.n == 0) {  // no retained key in this block: O = 0, LSE = -inf
+            uint4 *orow = reinterpret_cast<uint4 *>(p.O + (static_cast<size_t>(d.h) * p.S + (row_ok ? i : 0)) * D);
+            if (n == 0) {  // no retained key in this block: O = 0, LSE = -inf
                 if (row_ok) {
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k) orow[k] = make_uint4(0, 0, 0, 0);
-                    if (half == 0) p.LSE[static_cast<size_t>(d.h) * p.S + i] = -INFINITY;
+                    for (int k = 0; k < D / 8; ++k) orow[k] = make_uint4(0, 0, 0, 0);
+                    p.LSE[static_cast<size_t>(d.h) * p.S + i] = -INFINITY;
                 }
                 continue;
             }
             // stripe columns c <= i: between the counts of the previous and this block
             int n_i = 0;
-            if (row_ok && d.n > d.nb) {
-                const int32_t *Ch = p.vert_cols + p.vert_ptr[d.h];
-                const int hi = p.stripe_cnt[d.h * p.nqb + d.qb];
-                n_i = d.stripe_lo + lower_bound_i32(Ch + d.stripe_lo, hi - d.stripe_lo, i + 1);
+            if (row_ok && ns > 0) {
+                const int32_t *Ch = p.vert_cols + __ldg(p.vert_ptr + d.h);
+                const int hi = __ldg(p.stripe_cnt + d.h * p.nqb + qb);
+                n_i = slo + lower_bound_i32(Ch + slo, hi - slo, i + 1);
             }
-
-            // This half's 64-bit row mask of tile j (bit k = key column 64 * half + k).
-            uint32_t m_flags = 0;
-            uint64_t m_dm[4] = {0, 0, 0, 0}, m_cm = 0;
-            auto fetch_meta = [&](int j) {  // raw plan data of band tile j (loads only)
-                if (j < d.nb) {
-                    const size_t tt = static_cast<size_t>(d.tp0 + j);
-                    m_flags = __ldg(p.tile_flags + tt);
-                    const uint64_t *dmp = p.tile_dmask + 4 * tt;
-                    m_dm[0] = __ldg(dmp);
-                    m_dm[1] = __ldg(dmp + 1);
-                    m_dm[2] = __ldg(dmp + 2);
-                    m_dm[3] = __ldg(dmp + 3);
-                    m_cm = __ldg(p.tile_cmask + 2 * tt + half);
+            // plan data of band tile j: pulled into L1 one tile ahead, loaded at the tile
+            auto prefetch_l1 = [&](int j) {
+                if (j < nb) {
+                    const size_t tt = static_cast<size_t>(tp0 + j);
+                    asm volatile("prefetch.global.L1 [%0];" ::"l"(p.tile_dmask + 4 * tt));
+                    asm volatile("prefetch.global.L1 [%0];" ::"l"(p.tile_cmask + 2 * tt));
+                    asm volatile("prefetch.global.L1 [%0];" ::"l"(p.tile_flags + tt));
                 }
             };
-            auto make_mask = [&](int j, bool &full, uint64_t &bits) {
-                if (j < d.nb) {
-                    full = (m_flags & 1u) != 0;
-                    uint64_t lo, hi;
-                    row_diag_mask(m_dm, il, lo, hi);
-                    bits = (half ? hi : lo) & ~m_cm;
-                    if (!row_ok) bits = 0;
+            uint32_t mf = 0;
+            uint64_t md[4] = {0, 0, 0, 0}, mc[2] = {0, 0};
+            auto fetch = [&](int j) {
+                if (j < nb) {
+                    const size_t tt = static_cast<size_t>(tp0 + j);
+                    mf = __ldg(p.tile_flags + tt);
+                    const ulonglong2 d01 = __ldg(reinterpret_cast<const ulonglong2 *>(p.tile_dmask + 4 * tt));
+                    const ulonglong2 d23 = __ldg(reinterpret_cast<const ulonglong2 *>(p.tile_dmask + 4 * tt) + 1);
+                    const ulonglong2 c01 = __ldg(reinterpret_cast<const ulonglong2 *>(p.tile_cmask + 2 * tt));
+                    md[0] = d01.x;
+                    md[1] = d01.y;
+                    md[2] = d23.x;
+                    md[3] = d23.y;
+                    mc[0] = c01.x;
+                    mc[1] = c01.y;
+                }
+            };
+            prefetch_l1(0);
+            float m_run = -INFINITY, l_run = 0.0f;
+            for (int j = 0; j < n; ++j) {
+                // this tile's row mask (bit k = key column k), then prefetch the next tile's
+                bool full;
+                uint64_t mlo, mhi;
+                fetch(j);
+                if (j < nb) {
+                    full = (mf & 1u) != 0;
+                    row_diag_mask(md, il, mlo, mhi);
+                    mlo &= ~mc[0];
+                    mhi &= ~mc[1];
+                    if (!row_ok) mlo = mhi = 0;
                 } else {
-                    const int lim_k = n_i - (j - d.nb) * kBN - 64 * half;  // active iff k < lim_k
-                    full = lim_k >= 64;
-                    bits = lim_k >= 64 ? ~0ull : (lim_k <= 0 ? 0ull : (1ull << lim_k) - 1ull);
+                    const int lk = n_i - (j - nb) * kBN;  // key column k active iff k < lk
+                    full = lk >= kBN;
+                    mlo = lk >= 64 ? ~0ull : (lk <= 0 ? 0ull : (1ull << lk) - 1ull);
+                    mhi = lk >= 128 ? ~0ull : (lk <= 64 ? 0ull : (1ull << (lk - 64)) - 1ull);
                 }
-            };
-            // S of global tile tt -> dst; releases S[tt & 1] for the QK^T of tile tt + 2
-            auto load_s = [&](int tt, float(&dst)[64]) {
-                const int bb = tt & 1;
-                if (!good || !__all_sync(0xffffffffu, mbar_wait(&sh->s_full[bb], (tt >> 1) & 1, lim, abort))) {
-                    fail();
-                    return;
+                prefetch_l1(j + 1);
+                if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[s], tcnt & 1, lim, abort))) {
+                    ok = false;
+                    break;
                 }
                 tc_fence_after();
-                uint32_t r[64];
-                tmem_ld32(tmem + lane_off + col_s + 128 * bb, r);
-                tmem_ld32(tmem + lane_off + col_s + 128 * bb + 32, r + 32);
+                uint32_t r[128];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r + 32 * c);
                 tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(&sh->s_free[bb]);
+                if (!__all_sync(0xffffffffu, full || (mlo & mhi) == ~0ull)) {
+                    const uint32_t w[4] = {static_cast<uint32_t>(mlo), static_cast<uint32_t>(mlo >> 32),
+                                           static_cast<uint32_t>(mhi), static_cast<uint32_t>(mhi >> 32)};
 #pragma unroll
-                for (int k = 0; k < 64; ++k) dst[k] = __uint_as_float(r[k]);
-            };
-            auto apply_mask = [&](float(&v)[64], uint64_t bits) {
+                    for (int k = 0; k < 128; ++k)
+                        r[k] = (w[k >> 5] & (1u << (k & 31))) ? r[k] : kNegInf;
+                }
+                // row max of the tile (raw logits; the positive scale keeps the order)
+                float a[8];
 #pragma unroll
-                for (int k = 0; k < 64; ++k)
-                    if (!((bits >> k) & 1ull)) v[k] = -INFINITY;
-            };
-            auto half_max = [&](const float(&v)[64]) {
-                float mx[4] = {v[0], v[1], v[2], v[3]};
+                for (int q = 0; q < 8; ++q) a[q] = __uint_as_float(r[q]);
 #pragma unroll
-                for (int k = 4; k < 64; k += 8) {
-                    mx[0] = fmax3(mx[0], v[k], v[k + 1]);
-                    mx[1] = fmax3(mx[1], v[k + 2], v[k + 3]);
-                    mx[2] = fmax3(mx[2], v[k + 4], v[k + 5]);
-                    mx[3] = fmax3(mx[3], v[k + 6], v[k + 7]);
-                }
-                return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            };
-            // P = 2^(s * scale_log2 - mref) as packed bf16 pairs; returns the row-sum part
-            auto exps = [&](const float(&v)[64], float mref, uint32_t(&pk)[32]) {
-                const uint64_t nm2 = f2_pack(-mref, -mref);
-                uint64_t acc[4] = {0, 0, 0, 0};
+                for (int k = 8; k < 128; k += 16) {
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    float x0, x1;
-                    f2_unpack(f2_fma(f2_pack(v[2 * k], v[2 * k + 1]), sl2x2, nm2), x0, x1);
-                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                    acc[k & 3] = f2_add(acc[k & 3], f2_pack(p0, p1));
-                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                    pk[k] = *reinterpret_cast<const uint32_t *>(&pb);
+                    for (int q = 0; q < 8; ++q)
+                        a[q] = fmax3(a[q], __uint_as_float(r[k + 2 * q]), __uint_as_float(r[k + 2 * q + 1]));
                 }
-                float a0, a1, a2, a3, a4, a5, a6, a7;
-                f2_unpack(acc[0], a0, a1);
-                f2_unpack(acc[1], a2, a3);
-                f2_unpack(acc[2], a4, a5);
-                f2_unpack(acc[3], a6, a7);
-                return ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
-            };
-
-            // ---- prologue: first tile loaded, masked, its row max exchanged ----
-            float sA[64], sB[64];
-            bool nxt_full = false;
-            uint64_t nxt_bits = 0;
-            fetch_meta(0);
-            make_mask(0, nxt_full, nxt_bits);
-            fetch_meta(1);
-            load_s(t, sA);
-            float pm = -INFINITY;
-            if (good) {
-                if (!__all_sync(0xffffffffu, nxt_full)) apply_mask(sA, nxt_bits);
-                pm = half_max(sA);
-                sh->red_max[t & 1][half][il] = pm;
-            }
-            if (!bar_and(bar_id, 64, good)) {
-                ok = false;
-                break;
-            }
-            float m_run = fmaxf(pm, sh->red_max[t & 1][half ^ 1][il]) * sl2;  // -inf stays -inf
-            float l_run = 0.0f;
-            float mref = (m_run == -INFINITY) ? 0.0f : m_run;
-
-            // One pipeline step on tile j (global tile t): load + mask + reduce tile j+1
-            // while the exps of tile j run, hand P_j to the MMA, then agree on the
-            // reference max of tile j+1.  Returns false when the pair must leave.
-            auto step = [&](float(&cur)[64], float(&nxt)[64], int j) -> bool {
-                const bool has_next = j + 1 < d.n;
-                const int b = t & 1;
-                bool nf = true;
-                uint64_t nbits = ~0ull;
-                if (has_next) {
-                    load_s(t + 1, nxt);
-                    make_mask(j + 1, nf, nbits);
-                    if (j + 2 < d.n) fetch_meta(j + 2);
-                }
-                // P[b] may still be read by the PV of tile t-2
-                if (good && t >= 2 &&
-                    !__all_sync(0xffffffffu, mbar_wait(&sh->p_free[b], ((t - 2) >> 1) & 1, lim, abort)))
-                    fail();
-                float pmn = -INFINITY;
-                if (good) {
-                    uint32_t pk[32];
-                    float ls;
-                    if (!has_next) {
-                        ls = exps(cur, mref, pk);
-                    } else if (__all_sync(0xffffffffu, nf)) {
-                        ls = exps(cur, mref, pk);
-                        pmn = half_max(nxt);
-                    } else {
-                        apply_mask(nxt, nbits);
-                        ls = exps(cur, mref, pk);
-                        pmn = half_max(nxt);
-                    }
-                    tmem_st32(tmem + lane_off + col_p + 64 * b, pk);
-                    l_run += ls;
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(&sh->p_full[b]);
-                }
-                if (!has_next) return true;  // the epilogue reduction decides
-                const int nb2 = (t + 1) & 1;
-                if (good) sh->red_max[nb2][half][il] = pmn;
-                if (!bar_and(bar_id, 64, good)) return false;
-                const float m_new = fmaxf(m_run, fmaxf(pmn, sh->red_max[nb2][half ^ 1][il]) * sl2);
+                const float tmax = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+                const float m_new = fmaxf(m_run, tmax * sl2);  // -inf stays -inf
                 // lazy rescale: keep a stale max unless the row max grew by more than 2^8
-                const bool grow = (m_new != -INFINITY) &&
-                                  (m_run == -INFINITY || m_new > m_run + kRescaleThreshold);
+                const bool grow = (m_new != -INFINITY) && (m_run == -INFINITY || m_new > m_run + kRescaleThreshold);
                 const bool need_o = grow && (m_run != -INFINITY);
                 float factor = 1.0f;
                 if (grow) {
@@ -699,71 +723,66 @@ __global__ void __launch_bounds__(kThreads, 1)
                     l_run *= factor;
                     m_run = m_new;
                 }
-                if (__any_sync(0xffffffffu, need_o)) {  // warp-uniform: O is read warp-collectively
-                    // O must include tile t, just handed over: PV_t is the (t >> 1)-th
-                    // completion of p_free[b]; PV_{t-2} completed before P_t was written.
-                    if (!__all_sync(0xffffffffu, mbar_wait(&sh->p_free[b], (t >> 1) & 1, lim, abort))) {
-                        fail();
-                    } else {
-                        tc_fence_after();
-                        const float f = need_o ? factor : 1.0f;
+                const float mref = (m_run == -INFINITY) ? 0.0f : m_run;
+                // P = 2^(s * scale_log2 - mref), packed bf16 pairs over the first 64 S columns
+                const uint64_t nm2 = f2_pack(-mref, -mref);
+                uint64_t acc[4] = {0, 0, 0, 0};
+                uint32_t pk[64];
 #pragma unroll
-                        for (int c = 0; c < D / 64; ++c) {
-                            uint32_t r[32];
-                            tmem_ld32(tmem + lane_off + col_o + 32 * c, r);
-                            tmem_wait_ld();
+                for (int k = 0; k < 64; ++k) {
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), sl2x2, nm2),
+                              x0, x1);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    acc[k & 3] = f2_add(acc[k & 3], f2_pack(p0, p1));
+                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                    pk[k] = *reinterpret_cast<const uint32_t *>(&pb);
+                }
+                tmem_st32(tS, pk);
+                tmem_st32(tS + 32, pk + 32);
+                float a0, a1, a2, a3, a4, a5, a6, a7;
+                f2_unpack(acc[0], a0, a1);
+                f2_unpack(acc[1], a2, a3);
+                f2_unpack(acc[2], a4, a5);
+                f2_unpack(acc[3], a6, a7);
+                l_run += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+                if (__any_sync(0xffffffffu, need_o)) {
+                    // O_s holds every earlier tile: S_s of this tile was committed after the
+                    // PV of the previous tile, so that PV has completed.
+                    const float f = need_o ? factor : 1.0f;
 #pragma unroll
-                            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * f);
-                            tmem_st32(tmem + lane_off + col_o + 32 * c, r);
-                        }
-                        tmem_wait_st();
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + 32 * c, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+                        tmem_st32(tO + 32 * c, o);
                     }
                 }
-                mref = (m_run == -INFINITY) ? 0.0f : m_run;
-                return true;
-            };
-            int j = 0;
-            bool pair_ok = true;
-            while (true) {
-                pair_ok = step(sA, sB, j);
-                ++j;
-                ++t;
-                if (!pair_ok || j >= d.n) break;
-                pair_ok = step(sB, sA, j);
-                ++j;
-                ++t;
-                if (!pair_ok || j >= d.n) break;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&sh->p_full[s]);
+                ++tcnt;
             }
-            if (!pair_ok) {  // both warps of the pair left at the same reduction
+            if (!ok) break;
+            // ---- epilogue: O / l, LSE ----
+            if (!__all_sync(0xffffffffu, mbar_wait(&sh->o_full[s], icnt & 1, lim, abort))) {
                 ok = false;
                 break;
             }
-            // ---- epilogue: row sum of both halves, O / l, LSE ----
-            if (good) sh->red_l[half][il] = l_run;
-            if (!bar_and(bar_id, 64, good)) {
-                ok = false;
-                break;
-            }
-            const int t_last = t - 1;
-            // O complete: PV of the item's last tile (the phase before it, two tiles
-            // back, was awaited before the last P was written).  A failure here is
-            // settled at the next item's reduction.
-            if (!__all_sync(0xffffffffu, mbar_wait(&sh->p_free[t_last & 1], (t_last >> 1) & 1, lim, abort))) {
-                fail();
-                continue;
-            }
+            ++icnt;
             tc_fence_after();
-            uint32_t ro[D / 2];
+            uint32_t ro[D];
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c) tmem_ld32(tmem + lane_off + col_o + 32 * c, ro + 32 * c);
+            for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + 32 * c, ro + 32 * c);
             tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&sh->o_free);  // the next item's first PV may overwrite O
-            const float l_tot = l_run + sh->red_l[half ^ 1][il];
-            const float inv = (l_tot > 0.0f) ? 1.0f / l_tot : 0.0f;
+            // the next item's first PV may overwrite O_s once this slot's next P is handed
+            // over, which this thread does only after the load above has completed
+            const float inv = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
             if (row_ok) {
 #pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
+                for (int k = 0; k < D / 8; ++k) {
                     uint32_t w[4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -773,11 +792,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     orow[k] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
-                if (half == 0)
-                    p.LSE[static_cast<size_t>(d.h) * p.S + i] =
-                        (l_tot > 0.0f) ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+                p.LSE[static_cast<size_t>(d.h) * p.S + i] =
+                    (l_run > 0.0f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
             }
-            ++e;
         }
         if (!ok) {
             report(p.status, SSA_ERR_TIMEOUT);
@@ -877,7 +894,7 @@ int launch(const void *Q, const void *K, const void *V, uint16_t *KC, uint16_t *
                   fa.numRegs, kLaunchRegs);
         return SSA_ERR_UNSUPPORTED;
     }
-    const long long items = static_cast<long long>(p.H) * p.nqb;
+    const long long items = static_cast<long long>(p.H) * ((p.nqb + 1) / 2);
     const unsigned grid = static_cast<unsigned>(items < sm_count() ? items : sm_count());
     sparse_attn_fwd_kernel<D><<<grid, kThreads, C::SMEM_BYTES, s>>>(mQ, mK, mV, mKC, mVC, p);
     SSA_LAUNCH_CHECK();
@@ -919,6 +936,8 @@ extern "C" int sparse_attn_fwd(const void *Q, const void *K, const void *V, int 
                   "sparse_attn_fwd: null plan array");
     SSA_CHECK_ARG(aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(O),
                   "sparse_attn_fwd: Q, K, V and O must be 16-byte aligned");
+    SSA_CHECK_ARG(aligned16(plan->tile_dmask) && aligned16(plan->tile_cmask),
+                  "sparse_attn_fwd: plan tile_dmask and tile_cmask must be 16-byte aligned");
     SSA_CHECK_ARG(scale > 0.0f && scale < 1e30f, "sparse_attn_fwd: scale must be positive and finite");
     SSA_CHECK_ARG(static_cast<int64_t>(H_q) * ((S + kBM - 1) / kBM) < (1LL << 30),
                   "sparse_attn_fwd: too many query blocks");
