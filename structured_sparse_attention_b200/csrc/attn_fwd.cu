@@ -17,11 +17,14 @@
 //                            key-tile sequence of the two blocks (band tiles in
 //                            ascending key-tile order, then stripe tiles), so a key/value
 //                            tile wanted by both blocks is staged once and feeds both.
-//     warp 8 lane 0  scheduler (work counter -> item ring), TMA producer of the two Q
-//                    tiles and of the K tiles of the merged sequence; each K stage
+//     warp 8         lane 0: scheduler (work counter -> ring of item descriptors) and
+//                    TMA producer of the K tiles of the merged sequence; each K stage
 //                    carries a flag word: which slot uses it, first/last tile of a
 //                    slot within the item, end of work
-//     warp 8 lane 1  TMA producer of the V tiles of the same sequence
+//     warp 10        lane 0: TMA producer of the V tiles of the same sequence
+//     warp 11        lane 0: TMA producer of the two Q tiles of each item
+//                    (each blocking role has a warp of its own: single-lane loops of one
+//                    warp would serialise on each other's waits)
 //     warp 9         allocates tensor memory; lane 0 issues tcgen05.mma for both slots
 //                    from a polling loop: S_s = Q_s K^T into TMEM, O_s += P_s V with P_s
 //                    read from TMEM.  P_s is written over the first half of S_s, so the
@@ -55,15 +58,15 @@ namespace {
 
 constexpr int kBM = SSA_BLOCK;
 constexpr int kBN = SSA_BLOCK;
-// Warps 0-7 softmax (one warpgroup per slot), warp 8 TMA producers, warp 9 MMA issuer,
-// warps 10-11 idle.  Registers are rebalanced with setmaxnreg: the launch gives every
+// Warps 0-7 softmax (one warpgroup per slot), warps 8, 10, 11 TMA producers, warp 9 MMA
+// issuer.  Registers are rebalanced with setmaxnreg: the launch gives every
 // thread kLaunchRegs; the TMA/MMA warpgroup drops to kCtrlRegs and the softmax
 // warpgroups rise to kSoftmaxRegs, which together use exactly the launch allocation.
 constexpr int kThreads = 384;
 constexpr int kSlotThreads = 128;
 constexpr int kSoftmaxWarps = 8;
-constexpr int kWarpTma = 8, kWarpMma = 9;
-constexpr int kLaunchRegs = 168, kCtrlRegs = 56, kSoftmaxRegs = 224;
+constexpr int kWarpTma = 8, kWarpMma = 9, kWarpV = 10, kWarpQ = 11;
+constexpr int kLaunchRegs = 168, kCtrlRegs = 88, kSoftmaxRegs = 208;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kCtrlRegs <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr int kRing = 4;  // work-item descriptors in flight
@@ -72,6 +75,19 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kBoxBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr int64_t kDrainLimitNs = 1000000000LL;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if the max grows by > 256x
+// Exponentials on the FMA pipe: one pair in every kEmuEvery pairs of a row's 128
+// logits is computed by exp2_fma2 instead of the MUFU ex2, which alone would take as
+// long as the tile's MMAs.  Coefficients: degree-4 minimax fit of 2^f on [-1/2, 1/2]
+// (Remez exchange; printed by exp2_poly.py), relative error <= 2.7e-6 in fp32.
+constexpr int kEmuEvery = 0;  // 0: every exponential on the MUFU
+__host__ __device__ constexpr bool emulated_pair(int k) {
+    return kEmuEvery > 0 && (k % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1;
+}
+constexpr float kExp2C0 = 0.9999992847442627f;
+constexpr float kExp2C1 = 0.6931217908859253f;
+constexpr float kExp2C2 = 0.240247443318367f;
+constexpr float kExp2C3 = 0.05591785907745361f;
+constexpr float kExp2C4 = 0.009570102207362652f;
 constexpr size_t kCounterBytes = 256;     // work counter at the start of the workspace
 constexpr int kMaxSmem = 232448;          // 227 KB opt-in per block
 
@@ -153,6 +169,26 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
     return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
            (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
            (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// 2^x for a pair of floats on the FMA pipe (Cody-Waite style reduction): n = rint(x)
+// by adding 1.5 * 2^23, f = x - n in [-1/2, 1/2], 2^f by the minimax polynomial, and 2^n
+// added to the exponent field.  x is clamped to >= -126, so -inf (a masked logit) gives
+// 2^-126 instead of 0; the softmax treats a row whose max stayed -inf as empty.
+__device__ __forceinline__ void exp2_fma2(float x0, float x1, float &p0, float &p1) {
+    const uint64_t x = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+    const uint64_t t = f2_add(x, f2_pack(12582912.0f, 12582912.0f));
+    const uint64_t n = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
+    const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x);
+    uint64_t q = f2_fma(f2_pack(kExp2C4, kExp2C4), f, f2_pack(kExp2C3, kExp2C3));
+    q = f2_fma(q, f, f2_pack(kExp2C2, kExp2C2));
+    q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
+    q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
+    float q0, q1, t0, t1;
+    f2_unpack(q, q0, q1);
+    f2_unpack(t, t0, t1);
+    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
 // Instruction descriptor, kind::f16: bf16 A/B, fp32 accumulate, A K-major.
@@ -318,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int r = 0; r < kRing; ++r) {
             mbar_init(&sh->item_full[r], 1);
-            mbar_init(&sh->item_empty[r], 1 + kSoftmaxWarps);  // V lane, softmax warps
+            mbar_init(&sh->item_empty[r], 2 + kSoftmaxWarps);  // Q and V producers, softmax warps
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sh->q_full[s], 1);
@@ -354,14 +390,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
       if (warp == kWarpTma) {
         if (lane == 0) {
-            // ------------------ scheduler + Q and K producer ------------------
-            prefetch_tmap(&tmQ);
+            // ----------------- scheduler + K producer (warp 8, lane 0) -----------------
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmKC);
             bool ok = true;
             int m = 0, tk = 0;
-            int qn[2] = {0, 0};
             while (ok) {
+                // take the next work item and publish its descriptor to the other roles
                 const int idx = atomicAdd(p.work_counter, 1);
                 const int slot = m % kRing;
                 if (m >= kRing && !mbar_wait(&sh->item_empty[slot], ((m / kRing) - 1) & 1, lim, abort)) {
@@ -378,22 +413,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&sh->item_full[slot]);  // release: the descriptor is visible
                 ++m;
                 if (d.end) break;
-                // Q tiles of the slots that have work, each once the previous item's last
-                // QK^T of that slot is done
-#pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    if (!ok || d.nb[s] + d.ns[s] == 0) continue;
-                    if (qn[s] >= 1 && !mbar_wait(&sh->q_empty[s], (qn[s] - 1) & 1, lim, abort)) {
-                        ok = false;
-                        continue;
-                    }
-                    uint8_t *sQ = smem + C::OFF_Q + s * C::TILE_BYTES;
-                    mbar_arrive_expect_tx(&sh->q_full[s], C::TILE_BYTES);
-                    for (int b = 0; b < C::BOXES; ++b)
-                        tma_load_3d(sQ + b * kBoxBytes, &tmQ, &sh->q_full[s], 64 * b, d.qb[s] * kBM, d.h);
-                    ++qn[s];
-                }
-                if (!ok) break;
                 Steps st;
                 steps_init(st, p, d);
                 bool band;
@@ -429,11 +448,52 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *abort = 1;
             }
             // Drain: never leave the CTA with a copy still writing shared memory.
-            for (int s = 0; s < 2; ++s)
-                if (qn[s] >= 1) mbar_wait(&sh->q_full[s], (qn[s] - 1) & 1, kDrainLimitNs, nullptr);
             for (int u = (tk > C::NK ? tk - C::NK : 0); u < tk; ++u)
                 mbar_wait(&sh->k_full[u % C::NK], (u / C::NK) & 1, kDrainLimitNs, nullptr);
-        } else if (lane == 1) {
+        }
+      } else if (warp == kWarpQ) {
+        if (lane == 0) {
+            // ------------------------------ Q producer ------------------------------
+            // Its own warp, so a Q tile that waits for the previous item's last QK^T of its
+            // slot never holds back the K and V loads of the next item.
+            prefetch_tmap(&tmQ);
+            bool ok = true;
+            int m = 0;
+            int qn[2] = {0, 0};
+            while (ok) {
+                const int slot = m % kRing;
+                if (!mbar_wait(&sh->item_full[slot], (m / kRing) & 1, lim, abort)) {
+                    ok = false;
+                    break;
+                }
+                const ItemDesc d = sh->items[slot];
+                mbar_arrive(&sh->item_empty[slot]);
+                ++m;
+                if (d.end) break;
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {
+                    if (!ok || d.nb[s] + d.ns[s] == 0) continue;
+                    if (qn[s] >= 1 && !mbar_wait(&sh->q_empty[s], (qn[s] - 1) & 1, lim, abort)) {
+                        ok = false;
+                        continue;
+                    }
+                    uint8_t *sQ = smem + C::OFF_Q + s * C::TILE_BYTES;
+                    mbar_arrive_expect_tx(&sh->q_full[s], C::TILE_BYTES);
+                    for (int b = 0; b < C::BOXES; ++b)
+                        tma_load_3d(sQ + b * kBoxBytes, &tmQ, &sh->q_full[s], 64 * b, d.qb[s] * kBM, d.h);
+                    ++qn[s];
+                }
+            }
+            if (!ok) {
+                report(p.status, SSA_ERR_TIMEOUT);
+                *abort = 1;
+            }
+            // Drain: never leave the CTA with a copy still writing shared memory.
+            for (int s = 0; s < 2; ++s)
+                if (qn[s] >= 1) mbar_wait(&sh->q_full[s], (qn[s] - 1) & 1, kDrainLimitNs, nullptr);
+        }
+      } else if (warp == kWarpV) {
+        if (lane == 0) {
             // ----------------------------- V producer ----------------------------
             prefetch_tmap(&tmV);
             prefetch_tmap(&tmVC);
@@ -691,61 +751,80 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                uint32_t r[128];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r + 32 * c);
-                tmem_wait_ld();
-                if (!__all_sync(0xffffffffu, full || (mlo & mhi) == ~0ull)) {
-                    const uint32_t w[4] = {static_cast<uint32_t>(mlo), static_cast<uint32_t>(mlo >> 32),
-                                           static_cast<uint32_t>(mhi), static_cast<uint32_t>(mhi >> 32)};
-#pragma unroll
-                    for (int k = 0; k < 128; ++k)
-                        r[k] = (w[k >> 5] & (1u << (k & 31))) ? r[k] : kNegInf;
-                }
-                // row max of the tile (raw logits; the positive scale keeps the order)
-                float a[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) a[q] = __uint_as_float(r[q]);
-#pragma unroll
-                for (int k = 8; k < 128; k += 16) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        a[q] = fmax3(a[q], __uint_as_float(r[k + 2 * q]), __uint_as_float(r[k + 2 * q + 1]));
-                }
-                const float tmax = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-                const float m_new = fmaxf(m_run, tmax * sl2);  // -inf stays -inf
-                // lazy rescale: keep a stale max unless the row max grew by more than 2^8
-                const bool grow = (m_new != -INFINITY) && (m_run == -INFINITY || m_new > m_run + kRescaleThreshold);
-                const bool need_o = grow && (m_run != -INFINITY);
-                float factor = 1.0f;
-                if (grow) {
-                    factor = (m_run == -INFINITY) ? 0.0f : ex2_approx(m_run - m_new);
-                    l_run *= factor;
-                    m_run = m_new;
-                }
-                const float mref = (m_run == -INFINITY) ? 0.0f : m_run;
-                // P = 2^(s * scale_log2 - mref), packed bf16 pairs over the first 64 S columns
-                const uint64_t nm2 = f2_pack(-mref, -mref);
-                uint64_t acc[4] = {0, 0, 0, 0};
+                const bool do_mask = !__all_sync(0xffffffffu, full || (mlo & mhi) == ~0ull);
+                const uint32_t w[4] = {static_cast<uint32_t>(mlo), static_cast<uint32_t>(mlo >> 32),
+                                       static_cast<uint32_t>(mhi), static_cast<uint32_t>(mhi >> 32)};
                 uint32_t pk[64];
+                float psum = 0.0f;
+                auto load_s = [&](uint32_t(&r)[128]) {
 #pragma unroll
-                for (int k = 0; k < 64; ++k) {
-                    float x0, x1;
-                    f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), sl2x2, nm2),
-                              x0, x1);
-                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                    acc[k & 3] = f2_add(acc[k & 3], f2_pack(p0, p1));
-                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                    pk[k] = *reinterpret_cast<const uint32_t *>(&pb);
+                    for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r + 32 * c);
+                    tmem_wait_ld();
+                };
+                // P = 2^(s * scale_log2 - mref) over this thread's row as packed bf16 pairs for
+                // the first 64 S columns; psum is the row's sum of P
+                auto exps = [&](const uint32_t(&r)[128], float mref) {
+                    const uint64_t nm2 = f2_pack(-mref, -mref);
+                    uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+                    for (int k = 0; k < 64; ++k) {
+                        float x0, x1;
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), sl2x2,
+                                         nm2),
+                                  x0, x1);
+                        float p0, p1;
+                        if (emulated_pair(k)) {
+                            exp2_fma2(x0, x1, p0, p1);
+                        } else {
+                            p0 = ex2_approx(x0);
+                            p1 = ex2_approx(x1);
+                        }
+                        acc[k & 3] = f2_add(acc[k & 3], f2_pack(p0, p1));
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                        pk[k] = *reinterpret_cast<const uint32_t *>(&pb);
+                    }
+                    float a0, a1, a2, a3, a4, a5, a6, a7;
+                    f2_unpack(acc[0], a0, a1);
+                    f2_unpack(acc[1], a2, a3);
+                    f2_unpack(acc[2], a4, a5);
+                    f2_unpack(acc[3], a6, a7);
+                    psum = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+                };
+                // Mask the logits, take the tile's row max, then the lazy rescale rule: a new
+                // reference only when the row max grows by more than 2^8.
+                bool need_o = false;
+                float factor = 1.0f;
+                {
+                    uint32_t r[128];
+                    load_s(r);
+                    if (do_mask) {
+#pragma unroll
+                        for (int k = 0; k < 128; ++k)
+                            r[k] = (w[k >> 5] & (1u << (k & 31))) ? r[k] : kNegInf;
+                    }
+                    float a[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) a[q] = fmaxf(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+#pragma unroll
+                    for (int k = 16; k < 128; k += 16) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            a[q] = fmax3(a[q], __uint_as_float(r[k + 2 * q]), __uint_as_float(r[k + 2 * q + 1]));
+                    }
+                    const float tmax = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+                    const float m_new = fmaxf(m_run, tmax * sl2);  // -inf stays -inf
+                    const bool grow = (m_new != -INFINITY) && (m_run == -INFINITY || m_new > m_run + kRescaleThreshold);
+                    need_o = grow && (m_run != -INFINITY);
+                    if (grow) {
+                        factor = (m_run == -INFINITY) ? 0.0f : ex2_approx(m_run - m_new);
+                        l_run *= factor;
+                        m_run = m_new;
+                    }
+                    exps(r, (m_run == -INFINITY) ? 0.0f : m_run);
+                    l_run += psum;
                 }
                 tmem_st32(tS, pk);
                 tmem_st32(tS + 32, pk + 32);
-                float a0, a1, a2, a3, a4, a5, a6, a7;
-                f2_unpack(acc[0], a0, a1);
-                f2_unpack(acc[1], a2, a3);
-                f2_unpack(acc[2], a4, a5);
-                f2_unpack(acc[3], a6, a7);
-                l_run += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
                 if (__any_sync(0xffffffffu, need_o)) {
                     // O_s holds every earlier tile: S_s of this tile was committed after the
                     // PV of the previous tile, so that PV has completed.
@@ -779,7 +858,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
             // the next item's first PV may overwrite O_s once this slot's next P is handed
             // over, which this thread does only after the load above has completed
-            const float inv = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+            // a row whose max stayed -inf has no retained key: O = 0, LSE = -inf
+            const bool empty = !(m_run > -INFINITY) || !(l_run > 0.0f);
+            const float inv = empty ? 0.0f : 1.0f / l_run;
             if (row_ok) {
 #pragma unroll
                 for (int k = 0; k < D / 8; ++k) {
@@ -793,7 +874,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     orow[k] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
                 p.LSE[static_cast<size_t>(d.h) * p.S + i] =
-                    (l_run > 0.0f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+                    empty ? -INFINITY : (m_run + log2f(l_run)) * 0.69314718055994531f;
             }
         }
         if (!ok) {

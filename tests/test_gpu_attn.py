@@ -65,6 +65,49 @@ def test_main_diagonal_returns_values(ora):
     assert (np.abs(got - want) <= np.abs(want) * 2.0 ** -7).all()
 
 
+def _scaled_run(ora, diags, verts, S, d, q32, k32, v, scale):
+    """Attention on explicit (float32 -> bf16) Q/K and bf16-bit V against the dense oracle."""
+    import structured_sparse_attention_b200 as ssa
+    dev_lists, host = lists_to_device(diags, verts)
+    plan = ssa.extend(*dev_lists, S)
+    q = inputs.bf16_bits_from_f32(q32)
+    k = inputs.bf16_bits_from_f32(k32)
+    O, LSE = ssa.attn_fwd(t_bf16(q), t_bf16(k), t_bf16(v), plan, scale=scale)
+    ext = ora.extend(*host, S)
+    Oref, Lref = ora.attn_dense(q, k, v, ext, scale)
+    return compare_attn(O, LSE, Oref, Lref), (O, LSE, Oref, Lref)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_large_negative_logits(ora, d):
+    """The only retained key of every row (r = 0) scores about -32 sqrt(d), below the natural
+    log of 2^-126: its exponential underflows unless the row max is the reference, so a
+    wrong reference shows up as an empty row."""
+    S = 300
+    _, k, v = inputs.qkv(21, 1, 1, S, d)
+    k32 = inputs.f32_from_bf16_bits(k)
+    stats, (O, LSE, Oref, Lref) = _scaled_run(ora, [np.array([0], np.int32)], [np.zeros(0, np.int32)], S, d,
+                                              -32.0 * k32, k32, v, d ** -0.5)
+    assert np.isfinite(Lref).all() and (Lref < -126 * np.log(2)).all()
+    got = O[0].float().cpu().numpy()
+    want = inputs.f32_from_bf16_bits(v[0])
+    assert (np.abs(got - want) <= np.abs(want) * 2.0 ** -7).all()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_growing_logits(ora, d):
+    """Key norms grow along the sequence, so a row's max rises across its key tiles by far
+    more than the lazy-rescale threshold (2^8): exercises the rescale of O and the redo of a
+    tile whose stale reference is too small."""
+    S = 700
+    q, k, v = inputs.qkv(22, 2, 1, S, d)
+    q32 = 3.0 * inputs.f32_from_bf16_bits(q)
+    k32 = inputs.f32_from_bf16_bits(k) * (0.25 + 6.0 * np.arange(S, dtype=np.float32) / S)[None, :, None]
+    diags = [np.arange(0, 400, dtype=np.int32), np.array([0, 3, 130, 131, 260, 500], np.int32)]
+    verts = [np.array([5, 300], np.int32), np.array([0, 1, 2, 650], np.int32)]
+    _scaled_run(ora, diags, verts, S, d, q32, np.ascontiguousarray(k32), v, d ** -0.5)
+
+
 def test_stripes_only_and_empty_rows(ora):
     S, d = 700, 64
     diags = [np.zeros(0, np.int32), np.arange(400, 420, dtype=np.int32)]
