@@ -26,12 +26,12 @@
 //                    (each blocking role has a warp of its own: single-lane loops of one
 //                    warp would serialise on each other's waits)
 //     warp 9         allocates tensor memory; lane 0 issues tcgen05.mma for both slots
-//                    from a polling loop: S_s = Q_s K^T into TMEM, O_s += P_s V with P_s
-//                    read from TMEM.  P_s is written over the first half of S_s, so the
-//                    QK^T of a slot's next tile is always issued after the PV of its
-//                    current tile (tcgen05.mma operations of one thread execute in issue
-//                    order); the two slots interleave, so one slot's MMAs run while the
-//                    other slot's softmax works.
+//                    in a fixed order with blocking waits: for merged step u,
+//                    PV_0(u-1), QK_0(u), PV_1(u-1), QK_1(u).  S_s = Q_s K^T goes to TMEM,
+//                    O_s += P_s V with P_s read from TMEM.  P_s is written over the first
+//                    half of S_s, so a slot's QK^T always follows the PV of its previous
+//                    tile (tcgen05.mma operations of one thread execute in issue order);
+//                    while one slot's softmax works, the tensor core runs the other's MMAs.
 //     warps 0-3      softmax of slot 0 (query block 2p), one thread per query row
 //     warps 4-7      softmax of slot 1 (query block 2p+1)
 //                    tcgen05.ld S (128 columns), element mask from the plan (FULL
@@ -100,9 +100,7 @@ __host__ __device__ constexpr uint32_t f_last(int s) { return 16u << s; }
 
 template <int D>
 struct Cfg {
-    // K and V pipeline stages.  One slot's QK^T can run at most NK steps ahead of the
-    // other's, and a pending PV sits one step behind its QK^T, so NV >= NK + 1 keeps
-    // every V tile a slot waits for inside the V window (no circular wait).
+    // K and V pipeline stages (the issue order holds every V tile for one step at most).
     static constexpr int NK = (D == 128) ? 2 : 4;
     static constexpr int NV = (D == 128) ? 3 : 5;
     static constexpr int BOXES = D / 64;
@@ -114,7 +112,6 @@ struct Cfg {
     static constexpr int SMEM_BYTES = OFF_BAR + 1024 + 1024;  // barrier block + alignment slack
     static constexpr uint32_t COL_O = 256;                      // O_s at COL_O + D s
     static_assert(NK <= kMaxStages && NV <= kMaxStages, "too many stages");
-    static_assert(NV >= NK + 1, "V window must exceed the K window");
     static_assert(SMEM_BYTES <= kMaxSmem, "shared memory budget exceeded");
 };
 
@@ -537,100 +534,76 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else if (warp == kWarpMma) {
         // --------------------------------- MMA issuer ---------------------------------
+        // A fixed issue order with blocking waits (the warp sleeps in mbarrier.try_wait
+        // instead of taking issue slots from the softmax warps on its SM sub-partition).
+        // For merged step u:  PV_0(u-1) | wait K_u | QK_0(u) | PV_1(u-1) | QK_1(u) |
+        // release K_u and V_(u-1).  A slot's QK^T is issued after the PV of its previous
+        // tile (P shares the S columns), and while one slot's softmax works the tensor
+        // core runs the other slot's PV and QK^T.  Every PV is issued at the step after
+        // its QK^T, so no V tile is held longer than one step.
         if (lane == 0) {
             constexpr uint32_t IDESC_QK = idesc_bf16(kBM, kBN, false);
             constexpr uint32_t IDESC_PV = idesc_bf16(kBM, D, true);
+            const uint32_t sQ0 = smem_u32(smem + C::OFF_Q);
             bool ok = true;
-            // K and V stages are observed strictly in order (kobs, vobs) and released in
-            // order (krel, vrel) once neither slot needs them.  Per slot: qk_u = next
-            // step to examine, pend = a QK^T issued whose PV is not, pv_u its step.
-            int kobs = 0, vobs = 0, krel = 0, vrel = 0;
-            int qk_u[2] = {0, 0}, pv_u[2] = {0, 0}, pcnt[2] = {0, 0}, qcnt[2] = {0, 0};
-            bool pend[2] = {false, false}, fin[2] = {false, false};
-            bool pv_first[2] = {false, false}, pv_last[2] = {false, false};
-            uint64_t t_progress = global_timer_ns();
-            while (true) {
-                bool progress = false;
-                if (kobs < krel + C::NK && mbar_test(&sh->k_full[kobs % C::NK], (kobs / C::NK) & 1)) {
-                    ++kobs;
-                    progress = true;
-                }
-                if (vobs < vrel + C::NV && mbar_test(&sh->v_full[vobs % C::NV], (vobs / C::NV) & 1)) {
-                    ++vobs;
-                    progress = true;
-                }
+            int u = 0;  // merged step (K and V ring index)
+            int qcnt[2] = {0, 0}, pcnt[2] = {0, 0};
+            bool pend[2] = {false, false}, pfirst[2] = {false, false}, plast[2] = {false, false};
+            auto wait = [&](uint64_t *bar, int parity) {
+                if (ok && !mbar_wait(bar, parity, lim, abort)) ok = false;
+                return ok;
+            };
+            // O_s += P_s V_(u-1): the pending tile of slot s, issued at the step after its QK^T
+            auto pv = [&](int s) {
+                const int v = u - 1;
+                if (!wait(&sh->p_full[s], pcnt[s] & 1) || !wait(&sh->v_full[v % C::NV], (v / C::NV) & 1)) return;
+                tc_fence_after();
+                const uint32_t sV = smem_u32(smem + C::OFF_V + (v % C::NV) * C::TILE_BYTES);
 #pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    // PV of the pending tile once its P is in TMEM and its V tile landed
-                    if (pend[s] && pv_u[s] < vobs && mbar_test(&sh->p_full[s], pcnt[s] & 1)) {
-                        tc_fence_after();
-                        const uint32_t sV = smem_u32(smem + C::OFF_V + (pv_u[s] % C::NV) * C::TILE_BYTES);
+                for (int kk = 0; kk < kBN / 16; ++kk) {
+                    // B = V tile, MN-major: 16 keys per step (2 x 8-row groups of 128 B)
+                    umma_ts(tmem + C::COL_O + D * s, tmem + 128 * s + 8 * kk, sdesc(sV + kk * 2048, kBoxBytes, 1024),
+                            IDESC_PV, (!pfirst[s] || kk > 0) ? 1u : 0u);
+                }
+                if (plast[s]) umma_commit(&sh->o_full[s]);  // O_s of the item complete
+                pend[s] = false;
+                ++pcnt[s];
+            };
+            // S_s = Q_s K_u^T
+            auto qk = [&](int s, uint32_t f) {
+                if ((f & f_first(s)) && !wait(&sh->q_full[s], qcnt[s] & 1)) return;
+                tc_fence_after();
+                const uint32_t sQ = sQ0 + s * C::TILE_BYTES;
+                const uint32_t sK = smem_u32(smem + C::OFF_K + (u % C::NK) * C::TILE_BYTES);
 #pragma unroll
-                        for (int kk = 0; kk < kBN / 16; ++kk) {
-                            // B = V tile, MN-major: 16 keys per step (2 x 8-row groups of 128 B)
-                            const uint64_t bd = sdesc(sV + kk * 2048, kBoxBytes, 1024);
-                            umma_ts(tmem + C::COL_O + D * s, tmem + 128 * s + 8 * kk, bd, IDESC_PV,
-                                    (!pv_first[s] || kk > 0) ? 1u : 0u);
-                        }
-                        if (pv_last[s]) umma_commit(&sh->o_full[s]);  // O_s of the item complete
-                        pend[s] = false;
-                        ++pcnt[s];
-                        progress = true;
-                    }
-                    // QK^T of the slot's next tile (only after the PV that reads P_s, which
-                    // shares the S_s columns)
-                    if (!pend[s] && !fin[s] && qk_u[s] < kobs) {
-                        const uint32_t f = sh->kflags[qk_u[s] % C::NK];
-                        if (f & kStepEnd) {
-                            fin[s] = true;
-                            progress = true;
-                        } else if (!(f & f_in(s))) {
-                            ++qk_u[s];
-                            progress = true;
-                        } else if (!(f & f_first(s)) || mbar_test(&sh->q_full[s], qcnt[s] & 1)) {
-                            tc_fence_after();
-                            const uint32_t sQ = smem_u32(smem + C::OFF_Q + s * C::TILE_BYTES);
-                            const uint32_t sK = smem_u32(smem + C::OFF_K + (qk_u[s] % C::NK) * C::TILE_BYTES);
-#pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk) {
-                                // A = Q, B = K tile, both K-major: 16 elements = 32 B per step
-                                const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                                umma_ss(tmem + 128 * s, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024),
-                                        IDESC_QK, kk > 0 ? 1u : 0u);
-                            }
-                            umma_commit(&sh->s_full[s]);
-                            if (f & f_last(s)) umma_commit(&sh->q_empty[s]);  // Q_s no longer read
-                            if (f & f_first(s)) ++qcnt[s];
-                            pend[s] = true;
-                            pv_u[s] = qk_u[s];
-                            pv_first[s] = (f & f_first(s)) != 0;
-                            pv_last[s] = (f & f_last(s)) != 0;
-                            ++qk_u[s];
-                            progress = true;
-                        }
-                    }
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    // A = Q, B = K tile, both K-major: 16 elements = 32 B per step
+                    const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                    umma_ss(tmem + 128 * s, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), IDESC_QK,
+                            kk > 0 ? 1u : 0u);
                 }
-                // release stages no slot needs any more (each commit completes once the
-                // MMAs issued so far, which include every reader of the stage, are done)
-                const int kf = min(qk_u[0], qk_u[1]);
-                while (krel < kf) {
-                    umma_commit(&sh->k_empty[krel % C::NK]);
-                    ++krel;
-                }
-                const int vf = min(pend[0] ? pv_u[0] : qk_u[0], pend[1] ? pv_u[1] : qk_u[1]);
-                while (vrel < vf) {
-                    umma_commit(&sh->v_empty[vrel % C::NV]);
-                    ++vrel;
-                }
-                if (fin[0] && fin[1] && !pend[0] && !pend[1]) break;
-                if (progress) {
-                    t_progress = global_timer_ns();
-                    continue;
-                }
-                if (*abort || static_cast<int64_t>(global_timer_ns() - t_progress) >= lim) {
-                    ok = false;
-                    break;
-                }
+                umma_commit(&sh->s_full[s]);
+                if (f & f_last(s)) umma_commit(&sh->q_empty[s]);  // Q_s no longer read
+                if (f & f_first(s)) ++qcnt[s];
+                pend[s] = true;
+                pfirst[s] = (f & f_first(s)) != 0;
+                plast[s] = (f & f_last(s)) != 0;
+            };
+            while (ok) {
+                if (pend[0]) pv(0);
+                if (!wait(&sh->k_full[u % C::NK], (u / C::NK) & 1)) break;
+                const uint32_t f = sh->kflags[u % C::NK];
+                const bool end = (f & kStepEnd) != 0;
+                if (!end && (f & f_in(0))) qk(0, f);
+                if (pend[1]) pv(1);
+                if (!end && (f & f_in(1))) qk(1, f);
+                if (!ok) break;
+                // each commit completes once the MMAs issued so far, which include every
+                // reader of the stage, are done
+                if (u >= 1) umma_commit(&sh->v_empty[(u - 1) % C::NV]);
+                if (end) break;
+                umma_commit(&sh->k_empty[u % C::NK]);
+                ++u;
             }
             if (!ok) {
                 report(p.status, SSA_ERR_TIMEOUT);
