@@ -122,6 +122,8 @@ struct ItemDesc {
     int nb[2];   // band tiles
     int ns[2];   // stripe tiles
     int slo[2];  // stripe count of the previous block (columns < 128 qb)
+    int sc[2];   // stripe count of the block (columns <= min(S - 1, 128 qb + 127))
+    int vp;      // offset of the head's stripe columns in vert_cols
 };
 
 struct Shared {
@@ -251,17 +253,19 @@ __device__ ItemDesc make_pair(const AttnParams &p, int idx) {
     for (int s = 0; s < 2; ++s) {
         const int qb = 2 * pq + s;
         d.qb[s] = -1;
-        d.tp0[s] = d.nb[s] = d.ns[s] = d.slo[s] = 0;
+        d.tp0[s] = d.nb[s] = d.ns[s] = d.slo[s] = d.sc[s] = 0;
         if (qb >= p.nqb) continue;
         d.qb[s] = qb;
         const int it = d.h * p.nqb + qb;
         d.tp0[s] = __ldg(p.tile_ptr + it);
         d.slo[s] = qb > 0 ? __ldg(p.stripe_cnt + it - 1) : 0;
+        d.sc[s] = __ldg(p.stripe_cnt + it);
         if (!bad) {
             d.nb[s] = __ldg(p.tile_ptr + it + 1) - d.tp0[s];
-            d.ns[s] = (__ldg(p.stripe_cnt + it) + kBN - 1) / kBN;
+            d.ns[s] = (d.sc[s] + kBN - 1) / kBN;
         }
     }
+    d.vp = __ldg(p.vert_ptr + d.h);
     return d;
 }
 
@@ -273,7 +277,7 @@ struct Steps {
     const int32_t *kb[2];
     int nb[2], ns[2], i[2], a[2], an[2];
     int js;
-    bool started[2];
+    bool started[2], emitted;
 };
 
 __device__ __forceinline__ void steps_init(Steps &st, const AttnParams &p, const ItemDesc &d) {
@@ -288,12 +292,18 @@ __device__ __forceinline__ void steps_init(Steps &st, const AttnParams &p, const
         st.started[s] = false;
     }
     st.js = 0;
+    st.emitted = false;
 }
 
 // Next step of the sequence: key-tile row, whether it is a band tile (else a stripe
-// tile of K_C / V_C) and the slot flags.  Returns false after the last step.
+// tile of K_C / V_C) and the slot flags.  Returns false after the last step.  An item
+// without any tile yields one no-op step (row0 < 0, no slot, no data): the MMA issuer
+// then still passes a step boundary between the items around it, where it issues the
+// PVs the previous item's epilogue waits for.
 __device__ __forceinline__ bool steps_next(Steps &st, bool &band, int &row0, uint32_t &flags) {
     flags = 0;
+    const bool first = !st.emitted;
+    st.emitted = true;
     if (st.a[0] != INT_MAX || st.a[1] != INT_MAX) {
         const int kb = min(st.a[0], st.a[1]);
         band = true;
@@ -327,6 +337,11 @@ __device__ __forceinline__ bool steps_next(Steps &st, bool &band, int &row0, uin
             if (st.js == st.ns[s] - 1) flags |= f_last(s);
         }
         ++st.js;
+        return true;
+    }
+    if (first) {  // no tile at all
+        band = false;
+        row0 = -1;
         return true;
     }
     return false;
@@ -422,11 +437,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     sh->kflags[si] = fl;
-                    uint8_t *dst = smem + C::OFF_K + si * C::TILE_BYTES;
-                    mbar_arrive_expect_tx(&sh->k_full[si], C::TILE_BYTES);
-                    for (int b = 0; b < C::BOXES; ++b)
-                        tma_load_3d(dst + b * kBoxBytes, band ? &tmK : &tmKC, &sh->k_full[si], 64 * b, row0,
-                                    band ? d.g : d.h);
+                    if (row0 < 0) {  // no-op step: no data
+                        mbar_arrive(&sh->k_full[si]);
+                    } else {
+                        uint8_t *dst = smem + C::OFF_K + si * C::TILE_BYTES;
+                        mbar_arrive_expect_tx(&sh->k_full[si], C::TILE_BYTES);
+                        for (int b = 0; b < C::BOXES; ++b)
+                            tma_load_3d(dst + b * kBoxBytes, band ? &tmK : &tmKC, &sh->k_full[si], 64 * b, row0,
+                                        band ? d.g : d.h);
+                    }
                     ++tk;
                 }
             }
@@ -517,11 +536,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    uint8_t *dst = smem + C::OFF_V + si * C::TILE_BYTES;
-                    mbar_arrive_expect_tx(&sh->v_full[si], C::TILE_BYTES);
-                    for (int b = 0; b < C::BOXES; ++b)
-                        tma_load_3d(dst + b * kBoxBytes, band ? &tmV : &tmVC, &sh->v_full[si], 64 * b, row0,
-                                    band ? d.g : d.h);
+                    if (row0 < 0) {  // no-op step: no data
+                        mbar_arrive(&sh->v_full[si]);
+                    } else {
+                        uint8_t *dst = smem + C::OFF_V + si * C::TILE_BYTES;
+                        mbar_arrive_expect_tx(&sh->v_full[si], C::TILE_BYTES);
+                        for (int b = 0; b < C::BOXES; ++b)
+                            tma_load_3d(dst + b * kBoxBytes, band ? &tmV : &tmVC, &sh->v_full[si], 64 * b, row0,
+                                        band ? d.g : d.h);
+                    }
                     ++tv;
                 }
             }
@@ -591,6 +614,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             while (ok) {
                 if (pend[0]) pv(0);
+                // if K_u has not landed but slot 1's P has, its PV goes first (it needs no
+                // K, and an item's last PV completes the O its epilogue waits for)
+                if (pend[1] && !mbar_test(&sh->k_full[u % C::NK], (u / C::NK) & 1) &&
+                    mbar_test(&sh->p_full[1], pcnt[1] & 1))
+                    pv(1);
                 if (!wait(&sh->k_full[u % C::NK], (u / C::NK) & 1)) break;
                 const uint32_t f = sh->kflags[u % C::NK];
                 const bool end = (f & kStepEnd) != 0;
@@ -600,7 +628,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 // each commit completes once the MMAs issued so far, which include every
                 // reader of the stage, are done
-                if (u >= 1) umma_commit(&sh->v_empty[(u - 1) % C::NV]);
+                // V of step u-1 is observed before its release even when no PV read it
+                // (a no-op step), so every later wait on the stage sees its phases in order
+                if (u >= 1) {
+                    if (!wait(&sh->v_full[(u - 1) % C::NV], ((u - 1) / C::NV) & 1)) break;
+                    umma_commit(&sh->v_empty[(u - 1) % C::NV]);
+                }
                 if (end) break;
                 umma_commit(&sh->k_empty[u % C::NK]);
                 ++u;
@@ -667,11 +700,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 continue;
             }
             // stripe columns c <= i: between the counts of the previous and this block
+            // (usually none or a few: a short count, else a binary search)
             int n_i = 0;
             if (row_ok && ns > 0) {
-                const int32_t *Ch = p.vert_cols + __ldg(p.vert_ptr + d.h);
-                const int hi = __ldg(p.stripe_cnt + d.h * p.nqb + qb);
-                n_i = slo + lower_bound_i32(Ch + slo, hi - slo, i + 1);
+                const int32_t *Ch = p.vert_cols + d.vp + slo;
+                const int nc = (s ? d.sc[1] : d.sc[0]) - slo;
+                if (nc <= 8) {
+                    n_i = slo;
+                    for (int t = 0; t < nc; ++t) n_i += (__ldg(Ch + t) <= i) ? 1 : 0;
+                } else {
+                    n_i = slo + lower_bound_i32(Ch, nc, i + 1);
+                }
             }
             // plan data of band tile j: pulled into L1 one tile ahead, loaded at the tile
             auto prefetch_l1 = [&](int j) {
@@ -818,6 +857,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++tcnt;
             }
             if (!ok) break;
+            // The next item's descriptor is usually published already: pull its first
+            // band tile's plan data and its stripe columns into L1 while the epilogue
+            // waits for O.
+            if (mbar_test(&sh->item_full[m % kRing], (m / kRing) & 1)) {
+                const ItemDesc &dn = sh->items[m % kRing];
+                if (!dn.end && (s ? dn.qb[1] : dn.qb[0]) >= 0) {
+                    const size_t tt = static_cast<size_t>(s ? dn.tp0[1] : dn.tp0[0]);
+                    if ((s ? dn.nb[1] : dn.nb[0]) > 0) {
+                        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.tile_dmask + 4 * tt));
+                        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.tile_cmask + 2 * tt));
+                        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.tile_flags + tt));
+                    }
+                    if ((s ? dn.ns[1] : dn.ns[0]) > 0)
+                        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.vert_cols + dn.vp + (s ? dn.slo[1] : dn.slo[0])));
+                }
+            }
             // ---- epilogue: O / l, LSE ----
             if (!__all_sync(0xffffffffu, mbar_wait(&sh->o_full[s], icnt & 1, lim, abort))) {
                 ok = false;

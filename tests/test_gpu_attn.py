@@ -151,6 +151,22 @@ def test_long_context(ora, density):
     _run(diags, verts, S, 24, 8, 128, inputs.SEED_BASE + 5, rows=rows, ora=ora)
 
 
+def test_trailing_empty_items(ora):
+    """The first half of the query blocks of every head has no retained key, so the last
+    half of the work schedule (which runs from the last query blocks down) is items with
+    no tile at all, in long runs after every CTA's last non-empty item.  The step sequence
+    must still move past them: the last PVs of the preceding items (which their
+    epilogues wait for) may not depend on a later item being scheduled."""
+    S, Hq, Hkv, d = 8192, 48, 8, 128
+    g = np.random.default_rng(31)
+    diags = [np.arange(4096 + int(g.integers(0, 512)), 4096 + 600, dtype=np.int32) for _ in range(Hq)]
+    diags = [x[x < S] for x in diags]
+    verts = [np.sort(g.choice(np.arange(4096, S), size=3, replace=False)).astype(np.int32) for _ in range(Hq)]
+    rows = np.unique(np.concatenate([sample_rows(S, 96, 4), np.arange(4000, 4200)])).astype(np.int32)
+    for _ in range(3):  # several launches: the stall depended on timing
+        _run(diags, verts, S, Hq, Hkv, d, 41, rows=rows, ora=ora)
+
+
 def test_bad_kv_map_reports_invalid(ora):
     import structured_sparse_attention_b200 as ssa
     S, d = 256, 64
