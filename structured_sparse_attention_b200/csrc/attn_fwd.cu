@@ -572,6 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int u = 0;  // merged step (K and V ring index)
             int qcnt[2] = {0, 0}, pcnt[2] = {0, 0};
             bool pend[2] = {false, false}, pfirst[2] = {false, false}, plast[2] = {false, false};
+            bool v_seen = false;  // a PV of step u-1 has observed its V stage
             auto wait = [&](uint64_t *bar, int parity) {
                 if (ok && !mbar_wait(bar, parity, lim, abort)) ok = false;
                 return ok;
@@ -580,6 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto pv = [&](int s) {
                 const int v = u - 1;
                 if (!wait(&sh->p_full[s], pcnt[s] & 1) || !wait(&sh->v_full[v % C::NV], (v / C::NV) & 1)) return;
+                v_seen = true;
                 tc_fence_after();
                 const uint32_t sV = smem_u32(smem + C::OFF_V + (v % C::NV) * C::TILE_BYTES);
 #pragma unroll
@@ -614,11 +616,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             while (ok) {
                 if (pend[0]) pv(0);
-                // if K_u has not landed but slot 1's P has, its PV goes first (it needs no
-                // K, and an item's last PV completes the O its epilogue waits for)
-                if (pend[1] && !mbar_test(&sh->k_full[u % C::NK], (u / C::NK) & 1) &&
-                    mbar_test(&sh->p_full[1], pcnt[1] & 1))
-                    pv(1);
                 if (!wait(&sh->k_full[u % C::NK], (u / C::NK) & 1)) break;
                 const uint32_t f = sh->kflags[u % C::NK];
                 const bool end = (f & kStepEnd) != 0;
@@ -631,9 +628,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // V of step u-1 is observed before its release even when no PV read it
                 // (a no-op step), so every later wait on the stage sees its phases in order
                 if (u >= 1) {
-                    if (!wait(&sh->v_full[(u - 1) % C::NV], ((u - 1) / C::NV) & 1)) break;
+                    if (!v_seen && !wait(&sh->v_full[(u - 1) % C::NV], ((u - 1) / C::NV) & 1)) break;
                     umma_commit(&sh->v_empty[(u - 1) % C::NV]);
                 }
+                v_seen = false;
                 if (end) break;
                 umma_commit(&sh->k_empty[u % C::NK]);
                 ++u;
@@ -857,22 +855,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++tcnt;
             }
             if (!ok) break;
-            // The next item's descriptor is usually published already: pull its first
-            // band tile's plan data and its stripe columns into L1 while the epilogue
-            // waits for O.
-            if (mbar_test(&sh->item_full[m % kRing], (m / kRing) & 1)) {
-                const ItemDesc &dn = sh->items[m % kRing];
-                if (!dn.end && (s ? dn.qb[1] : dn.qb[0]) >= 0) {
-                    const size_t tt = static_cast<size_t>(s ? dn.tp0[1] : dn.tp0[0]);
-                    if ((s ? dn.nb[1] : dn.nb[0]) > 0) {
-                        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.tile_dmask + 4 * tt));
-                        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.tile_cmask + 2 * tt));
-                        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.tile_flags + tt));
-                    }
-                    if ((s ? dn.ns[1] : dn.ns[0]) > 0)
-                        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.vert_cols + dn.vp + (s ? dn.slo[1] : dn.slo[0])));
-                }
-            }
             // ---- epilogue: O / l, LSE ----
             if (!__all_sync(0xffffffffu, mbar_wait(&sh->o_full[s], icnt & 1, lim, abort))) {
                 ok = false;
