@@ -62,6 +62,30 @@ def load_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def profiled_traffic(workload):
+    """DRAM bytes per attention launch from the committed ncu summary of this workload,
+    if the attention sources are still the ones it was taken on (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"sparse_attn_fwd_{workload}_dram.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line and not line.startswith(("|", "#", " ")):
+            k, _, v = line.partition(":")
+            fields[k.strip()] = v.strip()
+    csrc = os.path.join(ROOT, "structured_sparse_attention_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("attn_fwd.cu", "common.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    if fields.get("source_sha256_16") != h.hexdigest()[:16]:
+        return None
+    try:
+        return float(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def nnz_per_head(diags, verts, S):
     """Retained pairs per head of the extended mask, from the list form (integer counting)."""
     out = []
@@ -346,7 +370,10 @@ def run_gpu(args, rank, world, local, dist):
         achieved = algo_bytes / (attn_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                 "frac": achieved / hbm_gbs}
-    roof.update({"traffic": args.traffic, "kernel": "sparse_attn_fwd (stripe gather + attention kernel)",
+    traffic = args.traffic if args.traffic is not None else profiled_traffic(args.workload)
+    roof.update({"traffic": traffic, "traffic_source": ("command line" if args.traffic is not None else
+                 "profiles/ summary (dram__bytes_read.sum + dram__bytes_write.sum, one launch)" if traffic else None),
+                 "kernel": "sparse_attn_fwd (stripe gather + attention kernel)",
                  "peak_source": f"{peak_kind} ({'burst' if bound == 'tensor' else 'copy'})",
                  "algorithmic": {"flops": flops, "bytes": algo_bytes},
                  "roofline_ms": max(t_tensor, t_hbm) * 1e3, "frac_of_roofline_time": max(t_tensor, t_hbm) * 1e3 / attn_ms})
