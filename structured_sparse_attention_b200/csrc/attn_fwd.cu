@@ -21,17 +21,18 @@
 //                    TMA producer of the K tiles of the merged sequence; each K stage
 //                    carries a flag word: which slot uses it, first/last tile of a
 //                    slot within the item, end of work
-//     warp 10        lane 0: TMA producer of the V tiles of the same sequence
-//     warp 11        lane 0: TMA producer of the two Q tiles of each item
+//     warp 10        lane 0: TMA producer of the two Q tiles of each item, then of the
+//                    V tiles of the same sequence
 //                    (each blocking role has a warp of its own: single-lane loops of one
 //                    warp would serialise on each other's waits)
-//     warp 9         allocates tensor memory; lane 0 issues tcgen05.mma for both slots
-//                    in a fixed order with blocking waits: for merged step u,
-//                    PV_0(u-1), QK_0(u), PV_1(u-1), QK_1(u).  S_s = Q_s K^T goes to TMEM,
-//                    O_s += P_s V with P_s read from TMEM.  P_s is written over the first
-//                    half of S_s, so a slot's QK^T always follows the PV of its previous
-//                    tile (tcgen05.mma operations of one thread execute in issue order);
-//                    while one slot's softmax works, the tensor core runs the other's MMAs.
+//     warps 9, 11    MMA issuers, one per slot (warp 9 allocates tensor memory).  For
+//                    merged step u, slot s issues PV_s of its tile at u-1, then QK_s(u).
+//                    S_s = Q_s K^T goes to TMEM, O_s += P_s V with P_s read from TMEM.
+//                    P_s is written over the first half of S_s, so a slot's QK^T always
+//                    follows the PV of its previous tile (tcgen05.mma operations of one
+//                    thread execute in issue order).  Two issuers keep the tensor pipe
+//                    fed while either one waits or commits; while one slot's softmax
+//                    works, the tensor core runs the other's MMAs.
 //     warps 0-3      softmax of slot 0 (query block 2p), one thread per query row
 //     warps 4-7      softmax of slot 1 (query block 2p+1)
 //                    tcgen05.ld S (128 columns), element mask from the plan (FULL
@@ -65,8 +66,8 @@ constexpr int kBN = SSA_BLOCK;
 constexpr int kThreads = 384;
 constexpr int kSlotThreads = 128;
 constexpr int kSoftmaxWarps = 8;
-constexpr int kWarpTma = 8, kWarpMma = 9, kWarpV = 10, kWarpQ = 11;
-constexpr int kLaunchRegs = 168, kCtrlRegs = 88, kSoftmaxRegs = 208;
+constexpr int kWarpTma = 8, kWarpMma0 = 9, kWarpV = 10, kWarpMma1 = 11;
+constexpr int kLaunchRegs = 168, kCtrlRegs = 104, kSoftmaxRegs = 200;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kCtrlRegs <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr int kRing = 4;  // work-item descriptors in flight
@@ -79,7 +80,10 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if the ma
 // logits is computed by exp2_fma2 instead of the MUFU ex2, which alone would take as
 // long as the tile's MMAs.  Coefficients: degree-4 minimax fit of 2^f on [-1/2, 1/2]
 // (Remez exchange; printed by exp2_poly.py), relative error <= 2.7e-6 in fp32.
-constexpr int kEmuEvery = 0;  // 0: every exponential on the MUFU
+#ifndef SSA_EMU_EVERY
+#define SSA_EMU_EVERY 0
+#endif
+constexpr int kEmuEvery = SSA_EMU_EVERY;  // 0: every exponential on the MUFU
 __host__ __device__ constexpr bool emulated_pair(int k) {
     return kEmuEvery > 0 && (k % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1;
 }
@@ -137,6 +141,7 @@ struct Shared {
     uint32_t kflags[kMaxStages];
     uint32_t tmem_base;
     int abort;
+    int turn;  // MMA issue order: bracket 2u + s (step u, slot s) may issue when turn == 2u + s
 };
 static_assert(sizeof(Shared) <= 1024, "barrier block too large");
 
@@ -157,6 +162,7 @@ struct AttnParams {
     float *LSE;
     int32_t *status;
     int64_t wait_ns;
+    int o_align32;  // O is 32-byte aligned (rows are then too: d * 2 bytes is a multiple of 32)
 };
 
 __device__ __forceinline__ int kv_head(const AttnParams &p, int h) {
@@ -366,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int r = 0; r < kRing; ++r) {
             mbar_init(&sh->item_full[r], 1);
-            mbar_init(&sh->item_empty[r], 2 + kSoftmaxWarps);  // Q and V producers, softmax warps
+            mbar_init(&sh->item_empty[r], 1 + kSoftmaxWarps);  // Q/V producer, softmax warps
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sh->q_full[s], 1);
@@ -377,18 +383,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int st = 0; st < C::NK; ++st) {
             mbar_init(&sh->k_full[st], 1);
-            mbar_init(&sh->k_empty[st], 1);
+            mbar_init(&sh->k_empty[st], 2);  // one arrival per slot's MMA issuer
         }
         for (int st = 0; st < C::NV; ++st) {
             mbar_init(&sh->v_full[st], 1);
-            mbar_init(&sh->v_empty[st], 1);
+            mbar_init(&sh->v_empty[st], 2);
         }
-        mbar_init(&sh->mma_drain, 1);
+        mbar_init(&sh->mma_drain, 2);
         mbar_init(&sh->softmax_done, 2 * kSlotThreads);
         sh->abort = 0;
+        sh->turn = 0;
         fence_barrier_init();
     }
-    if (warp == kWarpMma) {
+    if (warp == kWarpMma0) {
         tmem_alloc(&sh->tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -467,14 +474,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int u = (tk > C::NK ? tk - C::NK : 0); u < tk; ++u)
                 mbar_wait(&sh->k_full[u % C::NK], (u / C::NK) & 1, kDrainLimitNs, nullptr);
         }
-      } else if (warp == kWarpQ) {
+      } else if (warp == kWarpV) {
         if (lane == 0) {
-            // ------------------------------ Q producer ------------------------------
-            // Its own warp, so a Q tile that waits for the previous item's last QK^T of its
-            // slot never holds back the K and V loads of the next item.
+            // ------------------------- Q and V producer -------------------------
+            // The two Q tiles of an item, then its V tiles.  A Q tile waits for the
+            // last QK^T of its slot in the previous item; the V tiles of the previous
+            // item are all issued by then, so that wait never holds back a PV.
             prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmV);
+            prefetch_tmap(&tmVC);
             bool ok = true;
-            int m = 0;
+            int m = 0, tv = 0;
             int qn[2] = {0, 0};
             while (ok) {
                 const int slot = m % kRing;
@@ -499,32 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_3d(sQ + b * kBoxBytes, &tmQ, &sh->q_full[s], 64 * b, d.qb[s] * kBM, d.h);
                     ++qn[s];
                 }
-            }
-            if (!ok) {
-                report(p.status, SSA_ERR_TIMEOUT);
-                *abort = 1;
-            }
-            // Drain: never leave the CTA with a copy still writing shared memory.
-            for (int s = 0; s < 2; ++s)
-                if (qn[s] >= 1) mbar_wait(&sh->q_full[s], (qn[s] - 1) & 1, kDrainLimitNs, nullptr);
-        }
-      } else if (warp == kWarpV) {
-        if (lane == 0) {
-            // ----------------------------- V producer ----------------------------
-            prefetch_tmap(&tmV);
-            prefetch_tmap(&tmVC);
-            bool ok = true;
-            int m = 0, tv = 0;
-            while (ok) {
-                const int slot = m % kRing;
-                if (!mbar_wait(&sh->item_full[slot], (m / kRing) & 1, lim, abort)) {
-                    ok = false;
-                    break;
-                }
-                const ItemDesc d = sh->items[slot];
-                mbar_arrive(&sh->item_empty[slot]);
-                ++m;
-                if (d.end) break;
+                if (!ok) break;
                 Steps st;
                 steps_init(st, p, d);
                 bool band;
@@ -552,105 +537,138 @@ __global__ void __launch_bounds__(kThreads, 1)
                 report(p.status, SSA_ERR_TIMEOUT);
                 *abort = 1;
             }
+            // Drain: never leave the CTA with a copy still writing shared memory.
             for (int u = (tv > C::NV ? tv - C::NV : 0); u < tv; ++u)
                 mbar_wait(&sh->v_full[u % C::NV], (u / C::NV) & 1, kDrainLimitNs, nullptr);
+            for (int s = 0; s < 2; ++s)
+                if (qn[s] >= 1) mbar_wait(&sh->q_full[s], (qn[s] - 1) & 1, kDrainLimitNs, nullptr);
         }
-      } else if (warp == kWarpMma) {
-        // --------------------------------- MMA issuer ---------------------------------
-        // A fixed issue order with blocking waits (the warp sleeps in mbarrier.try_wait
-        // instead of taking issue slots from the softmax warps on its SM sub-partition).
-        // For merged step u:  PV_0(u-1) | wait K_u | QK_0(u) | PV_1(u-1) | QK_1(u) |
-        // release K_u and V_(u-1).  A slot's QK^T is issued after the PV of its previous
-        // tile (P shares the S columns), and while one slot's softmax works the tensor
-        // core runs the other slot's PV and QK^T.  Every PV is issued at the step after
-        // its QK^T, so no V tile is held longer than one step.
+      } else if (warp == kWarpMma0 || warp == kWarpMma1) {
+        // ------------------------------ MMA issuers ------------------------------
+        // One thread per slot (warps 9 and 11, on different SM sub-partitions), each
+        // issuing only its own slot's tcgen05.mma.  A tcgen05.mma blocks its thread while
+        // the tensor pipe's short queue is full, so a single issuer leaves the pipe idle
+        // whenever it does its waits and commits; with two, one slot's MMAs run while
+        // the other's issuer does its bookkeeping.  Per merged step u, slot s:
+        //   PV_s of its tile at u-1 (if any) | wait K_u | QK_s(u) (if s uses K_u)
+        // A slot's QK^T always follows the PV of its previous tile (P_s shares the S_s
+        // columns; tcgen05.mma of one thread execute in issue order).  Every PV is issued
+        // at the step after its QK^T, so no V tile is held longer than one step.  Each
+        // issuer releases every K and V stage once (a commit after its own MMAs on it,
+        // else a plain arrival), so each stage's empty barrier takes two arrivals; the
+        // K ring bounds the distance between the two issuers to NK steps, and NV > NK
+        // keeps every arrival in the phase it belongs to.  Every release of a stage
+        // (commit or plain arrival) comes after the issuer observed that stage's fill for
+        // the step, so no release can complete the stage's previous phase early, and a
+        // producer never waits more than one phase behind.
         if (lane == 0) {
+            const int s = (warp == kWarpMma1) ? 1 : 0;
             constexpr uint32_t IDESC_QK = idesc_bf16(kBM, kBN, false);
             constexpr uint32_t IDESC_PV = idesc_bf16(kBM, D, true);
-            const uint32_t sQ0 = smem_u32(smem + C::OFF_Q);
+            const uint32_t sQ = smem_u32(smem + C::OFF_Q + s * C::TILE_BYTES);
+            const uint32_t tS = tmem + 128 * s, tO = tmem + C::COL_O + D * s;
             bool ok = true;
             int u = 0;  // merged step (K and V ring index)
-            int qcnt[2] = {0, 0}, pcnt[2] = {0, 0};
-            bool pend[2] = {false, false}, pfirst[2] = {false, false}, plast[2] = {false, false};
-            bool v_seen = false;  // a PV of step u-1 has observed its V stage
+            int qcnt = 0, pcnt = 0;
+            bool pend = false, pfirst = false, plast = false;
+            // The issuer polls (mbar_wait_poll): mbarrier.try_wait in a thread with MMAs
+            // in flight costs about their drain time even when the phase is complete.
             auto wait = [&](uint64_t *bar, int parity) {
-                if (ok && !mbar_wait(bar, parity, lim, abort)) ok = false;
+                if (ok && !mbar_wait_poll(bar, parity, lim, abort)) ok = false;
                 return ok;
             };
-            // O_s += P_s V_(u-1): the pending tile of slot s, issued at the step after its QK^T
-            auto pv = [&](int s) {
-                const int v = u - 1;
-                if (!wait(&sh->p_full[s], pcnt[s] & 1) || !wait(&sh->v_full[v % C::NV], (v / C::NV) & 1)) return;
-                v_seen = true;
-                tc_fence_after();
-                const uint32_t sV = smem_u32(smem + C::OFF_V + (v % C::NV) * C::TILE_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {
-                    // B = V tile, MN-major: 16 keys per step (2 x 8-row groups of 128 B)
-                    umma_ts(tmem + C::COL_O + D * s, tmem + 128 * s + 8 * kk, sdesc(sV + kk * 2048, kBoxBytes, 1024),
-                            IDESC_PV, (!pfirst[s] || kk > 0) ? 1u : 0u);
+            volatile int *turn = &sh->turn;
+            // the issue order of the single-issuer schedule: brackets (u, 0), (u, 1), (u+1, 0) ...
+            auto wait_turn = [&](int t) {
+                if (!ok) return false;
+                if (*turn == t) return true;
+                const uint64_t t0 = global_timer_ns();
+                while (*turn != t) {
+                    if (*abort || static_cast<int64_t>(global_timer_ns() - t0) >= lim) {
+                        ok = false;
+                        return false;
+                    }
                 }
-                if (plast[s]) umma_commit(&sh->o_full[s]);  // O_s of the item complete
-                pend[s] = false;
-                ++pcnt[s];
-            };
-            // S_s = Q_s K_u^T
-            auto qk = [&](int s, uint32_t f) {
-                if ((f & f_first(s)) && !wait(&sh->q_full[s], qcnt[s] & 1)) return;
-                tc_fence_after();
-                const uint32_t sQ = sQ0 + s * C::TILE_BYTES;
-                const uint32_t sK = smem_u32(smem + C::OFF_K + (u % C::NK) * C::TILE_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    // A = Q, B = K tile, both K-major: 16 elements = 32 B per step
-                    const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                    umma_ss(tmem + 128 * s, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), IDESC_QK,
-                            kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&sh->s_full[s]);
-                if (f & f_last(s)) umma_commit(&sh->q_empty[s]);  // Q_s no longer read
-                if (f & f_first(s)) ++qcnt[s];
-                pend[s] = true;
-                pfirst[s] = (f & f_first(s)) != 0;
-                plast[s] = (f & f_last(s)) != 0;
+                return true;
             };
             while (ok) {
-                if (pend[0]) pv(0);
+                // 1. every wait of this step's bracket, while the other slot's MMAs run
+                const int v = u - 1;
+                if (u >= 1 && !wait(&sh->v_full[v % C::NV], (v / C::NV) & 1)) break;
+                if (pend && !wait(&sh->p_full[s], pcnt & 1)) break;
                 if (!wait(&sh->k_full[u % C::NK], (u / C::NK) & 1)) break;
                 const uint32_t f = sh->kflags[u % C::NK];
                 const bool end = (f & kStepEnd) != 0;
-                if (!end && (f & f_in(0))) qk(0, f);
-                if (pend[1]) pv(1);
-                if (!end && (f & f_in(1))) qk(1, f);
-                if (!ok) break;
-                // each commit completes once the MMAs issued so far, which include every
-                // reader of the stage, are done
-                // V of step u-1 is observed before its release even when no PV read it
-                // (a no-op step), so every later wait on the stage sees its phases in order
-                if (u >= 1) {
-                    if (!v_seen && !wait(&sh->v_full[(u - 1) % C::NV], ((u - 1) / C::NV) & 1)) break;
-                    umma_commit(&sh->v_empty[(u - 1) % C::NV]);
+                const bool in = !end && (f & f_in(s));
+                if (in && (f & f_first(s)) && !wait(&sh->q_full[s], qcnt & 1)) break;
+                // 2. this slot's turn: PV_s of its tile at u-1, then QK_s(u)
+                if (!wait_turn(2 * u + s)) break;
+                tc_fence_after();
+                if (pend) {
+                    const uint32_t sV = smem_u32(smem + C::OFF_V + (v % C::NV) * C::TILE_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk) {
+                        // B = V tile, MN-major: 16 keys per step (2 x 8-row groups of 128 B)
+                        umma_ts(tO, tS + 8 * kk, sdesc(sV + kk * 2048, kBoxBytes, 1024), IDESC_PV,
+                                (!pfirst || kk > 0) ? 1u : 0u);
+                    }
                 }
-                v_seen = false;
+                if (in) {
+                    const uint32_t sK = smem_u32(smem + C::OFF_K + (u % C::NK) * C::TILE_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        // A = Q, B = K tile, both K-major: 16 elements = 32 B per step
+                        const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                        umma_ss(tS, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), IDESC_QK,
+                                kk > 0 ? 1u : 0u);
+                    }
+                }
+                *turn = 2 * u + s + 1;
+                // 3. completions.  A release of V_(u-1) by a slot that did not read it comes
+                // after its fill was observed above: the fill of step u-1 follows the
+                // completion of the stage's previous phase, so the release lands in the
+                // phase of step u-1 (never in the previous one, where it would stand in
+                // for the other slot's PV still reading the stage, and never a phase
+                // ahead of the producer, as for a no-op step that no slot reads).
+                if (pend) {
+                    if (plast) umma_commit(&sh->o_full[s]);  // O_s of the item complete
+                    umma_commit(&sh->v_empty[v % C::NV]);    // completes once the PV has read V
+                    pend = false;
+                    ++pcnt;
+                } else if (u >= 1) {
+                    mbar_arrive(&sh->v_empty[v % C::NV]);
+                }
                 if (end) break;
-                umma_commit(&sh->k_empty[u % C::NK]);
+                if (in) {
+                    umma_commit(&sh->s_full[s]);
+                    if (f & f_last(s)) umma_commit(&sh->q_empty[s]);  // Q_s no longer read
+                    umma_commit(&sh->k_empty[u % C::NK]);
+                    if (f & f_first(s)) ++qcnt;
+                    pend = true;
+                    pfirst = (f & f_first(s)) != 0;
+                    plast = (f & f_last(s)) != 0;
+                } else {
+                    mbar_arrive(&sh->k_empty[u % C::NK]);
+                }
                 ++u;
             }
             if (!ok) {
                 report(p.status, SSA_ERR_TIMEOUT);
                 *abort = 1;
             }
-            umma_commit(&sh->mma_drain);  // completes once every issued MMA is done
+            umma_commit(&sh->mma_drain);  // completes once every MMA this thread issued is done
         }
         __syncwarp();
         // Free tensor memory after the softmax warps are done and every MMA has finished.
-        if (lane == 0) {
-            mbar_wait(&sh->softmax_done, 0, kDrainLimitNs, nullptr);
-            mbar_wait(&sh->mma_drain, 0, kDrainLimitNs, nullptr);
+        if (warp == kWarpMma0) {
+            if (lane == 0) {
+                mbar_wait(&sh->softmax_done, 0, kDrainLimitNs, nullptr);
+                mbar_wait(&sh->mma_drain, 0, kDrainLimitNs, nullptr);
+            }
+            __syncwarp();
+            tc_fence_after();
+            tmem_dealloc(tmem, kTmemCols);
         }
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
       }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
@@ -872,16 +890,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool empty = !(m_run > -INFINITY) || !(l_run > 0.0f);
             const float inv = empty ? 0.0f : 1.0f / l_run;
             if (row_ok) {
+                // the row as bf16, 16 columns (32 bytes) per store when O allows it: half the
+                // store instructions of 16-byte stores for the same bytes
+                uint32_t w[D / 2];
 #pragma unroll
-                for (int k = 0; k < D / 8; ++k) {
-                    uint32_t w[4];
+                for (int q = 0; q < D / 2; ++q) {
+                    const __nv_bfloat162 v2 =
+                        __floats2bfloat162_rn(__uint_as_float(ro[2 * q]) * inv, __uint_as_float(ro[2 * q + 1]) * inv);
+                    w[q] = *reinterpret_cast<const uint32_t *>(&v2);
+                }
+                if (p.o_align32) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(ro[8 * k + 2 * q]) * inv,
-                                                                        __uint_as_float(ro[8 * k + 2 * q + 1]) * inv);
-                        w[q] = *reinterpret_cast<const uint32_t *>(&v2);
-                    }
-                    orow[k] = make_uint4(w[0], w[1], w[2], w[3]);
+                    for (int k = 0; k < D / 16; ++k) st_global_v8(orow + 2 * k, w + 8 * k);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < D / 8; ++k) orow[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
                 }
                 p.LSE[static_cast<size_t>(d.h) * p.S + i] =
                     empty ? -INFINITY : (m_run + log2f(l_run)) * 0.69314718055994531f;
@@ -1056,6 +1079,7 @@ extern "C" int sparse_attn_fwd(const void *Q, const void *K, const void *V, int 
     p.work_counter = static_cast<int *>(ws);
     p.scale_log2 = scale * 1.4426950408889634f;
     p.O = static_cast<uint16_t *>(O);
+    p.o_align32 = (reinterpret_cast<uintptr_t>(O) & 31u) == 0;
     p.LSE = LSE;
     p.status = dev_status;
     p.wait_ns = wait_limit_ns();
