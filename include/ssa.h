@@ -142,17 +142,23 @@ typedef struct ssa_plan_sizes {
  * device buffer owned by the caller and sized from ssa_plan_sizes:
  *   ext_diag_ptr [n_heads+1], ext_diag_offsets [max(n_diag,1)],
  *   ext_vert_ptr [n_heads+1], ext_vert_cols [max(n_vert,1)],
- *   tile_ptr [n_heads*nqb + 1], tile_kb [max(n_tiles,1)],
+ *   tile_ptr [n_heads*nqb + 1], tile_key0 [max(n_tiles,1)],
  *   tile_dmask [max(n_tiles,1)][4] (uint64), tile_cmask [max(n_tiles,1)][2] (uint64),
  *   tile_flags [max(n_tiles,1)], stripe_cnt [n_heads*nqb].
- * Tile semantics, for head h, query block qb (rows 128qb..128qb+127), key tile kb:
- *   dmask bit t (0..254) set  iff  r = 128(qb-kb) + t - 127 is an extended diagonal
- *   cmask bit jl (0..127) set iff  column 128kb + jl is an extended column
- *   a tile is listed, in ascending kb, iff some (i, j) in it has i < S, j <= i,
- *   i - j a diagonal and j not a column; tile_flags bit 0 (FULL) iff kb < qb,
- *   128(qb+1) <= S, all 255 dmask bits set and cmask == 0;
+ * Tile semantics, for head h and query block qb (rows lo = 128qb .. hi = 128qb+127):
+ *   needed keys: j in [0, hi] such that some extended diagonal r has lo-j <= r <= hi-j
+ *   (all 128 rows count, even in a ragged last block); the band tiles are key windows
+ *   key0 .. key0+127, chosen greedily: the first starts at the smallest needed key,
+ *   each next one at the smallest needed key >= previous key0 + 128 (so a band whose
+ *   keys do not start at a multiple of 128 still takes ceil(width / 128) windows);
+ *   dmask bit t (0..254) set  iff  r = 128qb - key0 + t - 127 is an extended diagonal
+ *   cmask bit jl (0..127) set iff  column key0 + jl is an extended column
+ *   a window is listed, in ascending key0, iff some (i, j) in it has i < S,
+ *   i - j a diagonal and j not a column; tile_flags bit 0 (FULL) iff 128(qb+1) <= S,
+ *   all 255 dmask bits set and cmask == 0;
  *   stripe_cnt[h*nqb+qb] = #{extended columns c <= min(S-1, 128qb+127)}.
- * Columns are owned by the stripe phase only, so each retained pair is used once.
+ * The windows are disjoint and cover every needed key, and columns are owned by the
+ * stripe phase only, so each retained pair is used once.
  */
 typedef struct ssa_plan {
     int32_t n_heads;
@@ -165,14 +171,15 @@ typedef struct ssa_plan {
     int32_t *ext_vert_ptr;
     int32_t *ext_vert_cols;
     int32_t *tile_ptr;
-    int32_t *tile_kb;
+    int32_t *tile_key0;
     uint64_t *tile_dmask;
     uint64_t *tile_cmask;
     uint32_t *tile_flags;
     int32_t *stripe_cnt;
 } ssa_plan;
 
-/* Workspace bytes of either pass of sparse_pattern_extend. */
+/* Workspace bytes of either pass of sparse_pattern_extend (about 4 * n_heads * S for
+ * the per-diagonal run starts, plus small per-block counters). */
 SSA_API size_t sparse_pattern_extend_ws_bytes(int n_heads, int S);
 
 /*

@@ -156,14 +156,14 @@ def plan(ext, S, routine="brute"):
     nqb = (S + TILE - 1) // TILE
     f = getattr(lib(), "ora_plan_" + routine)
     n = _check(f(H, _p(dp), _p(do), _p(vp), _p(vo), S, 0, None, None, None, None, None, None), "plan")
-    out = dict(tile_ptr=np.zeros(H * nqb + 1, np.int32), tile_kb=np.zeros(max(n, 1), np.int32),
+    out = dict(tile_ptr=np.zeros(H * nqb + 1, np.int32), tile_key0=np.zeros(max(n, 1), np.int32),
                tile_dmask=np.zeros((max(n, 1), 4), np.uint64), tile_cmask=np.zeros((max(n, 1), 2), np.uint64),
                tile_flags=np.zeros(max(n, 1), np.uint32), stripe_cnt=np.zeros(H * nqb, np.int32))
-    n2 = _check(f(H, _p(dp), _p(do), _p(vp), _p(vo), S, n, _p(out["tile_ptr"]), _p(out["tile_kb"]),
+    n2 = _check(f(H, _p(dp), _p(do), _p(vp), _p(vo), S, n, _p(out["tile_ptr"]), _p(out["tile_key0"]),
                   _p(out["tile_dmask"]), _p(out["tile_cmask"]), _p(out["tile_flags"]),
                   _p(out["stripe_cnt"])), "plan")
     assert n2 == n
-    for k in ("tile_kb", "tile_dmask", "tile_cmask", "tile_flags"):
+    for k in ("tile_key0", "tile_dmask", "tile_cmask", "tile_flags"):
         out[k] = out[k][:n].copy()
     out["n_tiles"] = n
     out["nqb"] = nqb
@@ -179,13 +179,13 @@ def plan_items(ext, S, items):
     f = lib().ora_plan_items
     n = _check(f(H, _p(dp), _p(do), _p(vp), _p(vo), S, ni, _p(items), 0, None, None, None, None, None,
                  None), "plan_items")
-    out = dict(item_ptr=np.zeros(ni + 1, np.int32), tile_kb=np.zeros(max(n, 1), np.int32),
+    out = dict(item_ptr=np.zeros(ni + 1, np.int32), tile_key0=np.zeros(max(n, 1), np.int32),
                tile_dmask=np.zeros((max(n, 1), 4), np.uint64), tile_cmask=np.zeros((max(n, 1), 2), np.uint64),
                tile_flags=np.zeros(max(n, 1), np.uint32), stripe_cnt=np.zeros(ni, np.int32))
-    _check(f(H, _p(dp), _p(do), _p(vp), _p(vo), S, ni, _p(items), n, _p(out["item_ptr"]), _p(out["tile_kb"]),
+    _check(f(H, _p(dp), _p(do), _p(vp), _p(vo), S, ni, _p(items), n, _p(out["item_ptr"]), _p(out["tile_key0"]),
              _p(out["tile_dmask"]), _p(out["tile_cmask"]), _p(out["tile_flags"]), _p(out["stripe_cnt"])),
            "plan_items")
-    for k in ("tile_kb", "tile_dmask", "tile_cmask", "tile_flags"):
+    for k in ("tile_key0", "tile_dmask", "tile_cmask", "tile_flags"):
         out[k] = out[k][:n].copy()
     return out
 

@@ -218,16 +218,24 @@ int ora_extend(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offsets
 }
 
 /* ----------------------------------------------------------------------------------
- * Canonical tile plan.  For head h, query block qb (rows 128qb..128qb+127) and key
- * tile kb (columns 128kb..128kb+127):
- *   dmask bit t (0..254) set  iff  r = 128(qb-kb) + t - 127 is in D_h
- *   cmask bit jl (0..127) set iff  128kb + jl is in C_h
- *   listed (ascending kb)     iff  some (i, j) of the tile has i < S, j <= i,
- *                                  i - j in D_h and j not in C_h
- *   FULL flag (bit 0)         iff  kb < qb, 128(qb+1) <= S, all 255 dmask bits set
- *                                  and cmask == 0
+ * Canonical tile plan (this library's own layout of the extended mask).  For head h
+ * and query block qb (rows lo = 128qb .. hi = 128qb + 127; rows >= S hold no pair):
+ *   needed keys      j in [0, hi] such that some r in D_h has lo - j <= r <= hi - j
+ *                    (the keys some diagonal reaches from some row of the block,
+ *                    counting all 128 rows even in a ragged last block)
+ *   key windows      greedy: the first starts at the smallest needed key, each next
+ *                    one at the smallest needed key >= (previous start + 128); a
+ *                    window with start key0 covers keys key0 .. key0 + 127
+ *   dmask bit t (0..254) set  iff  r = 128qb - key0 + t - 127 is in D_h
+ *   cmask bit jl (0..127) set iff  key0 + jl is in C_h
+ *   a window is listed (ascending key0) iff some (i, j) of it has i < S,
+ *                    i - j in D_h and j not in C_h (j <= i follows from r >= 0)
+ *   FULL flag (bit 0)         iff  128(qb+1) <= S, all 255 dmask bits set and
+ *                                  cmask == 0
  *   stripe_cnt[h][qb]          =   #{c in C_h : c <= min(S-1, 128qb+127)}
- * Two independent routines compute it; the tests require them to agree.
+ * The windows are disjoint and cover every needed key, so each retained pair of the
+ * band lies in exactly one listed window.  Two independent routines compute the
+ * plan; the tests require them to agree.
  * -------------------------------------------------------------------------------- */
 
 static void set_bit(uint64_t *w, int b) { w[b >> 6] |= (uint64_t)1 << (b & 63); }
@@ -252,12 +260,12 @@ static int32_t count_le(const int32_t *a, int n, int32_t x) {
     return c;
 }
 
-/* Routine 1: brute force over every (i, j) of every candidate tile (small S only).
+/* Routine 1: brute force over every (i, j) of the block (small S only).
  * With tile arrays NULL it only counts.  Returns the number of listed tiles, or a
  * negative error (capacity exceeded / bad input). */
 long long ora_plan_brute(int n_heads, const int32_t *ext_diag_ptr, const int32_t *ext_diag_offsets,
                          const int32_t *ext_vert_ptr, const int32_t *ext_vert_cols, int S,
-                         long long capacity, int32_t *tile_ptr, int32_t *tile_kb,
+                         long long capacity, int32_t *tile_ptr, int32_t *tile_key0,
                          uint64_t *tile_dmask, uint64_t *tile_cmask, uint32_t *tile_flags,
                          int32_t *stripe_cnt) {
     if (n_heads < 0 || S <= 0) return ORA_ERR_INVALID;
@@ -265,9 +273,11 @@ long long ora_plan_brute(int n_heads, const int32_t *ext_diag_ptr, const int32_t
     int nqb = (S + T - 1) / T;
     uint8_t *isD = (uint8_t *)malloc((size_t)S);
     uint8_t *isC = (uint8_t *)malloc((size_t)S);
-    if (!isD || !isC) {
+    uint8_t *need = (uint8_t *)malloc((size_t)nqb * T);
+    if (!isD || !isC || !need) {
         free(isD);
         free(isC);
+        free(need);
         return ORA_ERR_NOMEM;
     }
     long long n = 0;
@@ -282,24 +292,40 @@ long long ora_plan_brute(int n_heads, const int32_t *ext_diag_ptr, const int32_t
         for (int k = 0; k < nc; ++k) isC[C[k]] = 1;
         for (int qb = 0; qb < nqb; ++qb) {
             if (tile_ptr) tile_ptr[h * nqb + qb] = (int32_t)n;
-            int last_row = (T * qb + T - 1 < S - 1) ? T * qb + T - 1 : S - 1;
+            const long lo = (long)T * qb, hi = lo + T - 1;
+            int last_row = (hi < S - 1) ? (int)hi : S - 1;
             if (stripe_cnt) stripe_cnt[h * nqb + qb] = count_le(C, nc, last_row);
-            for (int kb = 0; kb <= qb; ++kb) {
+            /* needed keys, cell by cell over the 128 rows of the block */
+            memset(need, 0, (size_t)(hi + 1));
+            for (long j = 0; j <= hi; ++j)
+                for (int il = 0; il < T; ++il) {
+                    long r = lo + il - j;
+                    if (r >= 0 && r < S && isD[r]) {
+                        need[j] = 1;
+                        break;
+                    }
+                }
+            long next = 0; /* smallest allowed start of the next window */
+            while (1) {
+                long key0 = next;
+                while (key0 <= hi && !need[key0]) ++key0;
+                if (key0 > hi) break;
+                next = key0 + T;
                 uint64_t dm[4] = {0, 0, 0, 0}, cm[2] = {0, 0};
                 for (int t = 0; t < 2 * T - 1; ++t) {
-                    long r = (long)T * (qb - kb) + t - (T - 1);
+                    long r = lo - key0 + t - (T - 1);
                     if (r >= 0 && r < S && isD[r]) set_bit(dm, t);
                 }
                 for (int jl = 0; jl < T; ++jl) {
-                    long j = (long)T * kb + jl;
+                    long j = key0 + jl;
                     if (j < S && isC[j]) set_bit(cm, jl);
                 }
                 int listed = 0;
                 for (int il = 0; il < T && !listed; ++il) {
-                    long i = (long)T * qb + il;
+                    long i = lo + il;
                     if (i >= S) break;
                     for (int jl = 0; jl < T; ++jl) {
-                        long j = (long)T * kb + jl;
+                        long j = key0 + jl;
                         if (j <= i && isD[i - j] && !isC[j]) {
                             listed = 1;
                             break;
@@ -307,15 +333,16 @@ long long ora_plan_brute(int n_heads, const int32_t *ext_diag_ptr, const int32_t
                     }
                 }
                 if (!listed) continue;
-                int full = (kb < qb) && ((long)T * (qb + 1) <= S) && popcount256(dm) == 2 * T - 1 &&
-                           cm[0] == 0 && cm[1] == 0;
-                if (tile_kb) {
+                int full = ((long)T * (qb + 1) <= S) && popcount256(dm) == 2 * T - 1 && cm[0] == 0 &&
+                           cm[1] == 0;
+                if (tile_key0) {
                     if (n >= capacity) {
                         free(isD);
                         free(isC);
+                        free(need);
                         return ORA_ERR_CAPACITY;
                     }
-                    tile_kb[n] = kb;
+                    tile_key0[n] = (int32_t)key0;
                     memcpy(tile_dmask + 4 * n, dm, sizeof dm);
                     memcpy(tile_cmask + 2 * n, cm, sizeof cm);
                     tile_flags[n] = full ? 1u : 0u;
@@ -327,6 +354,7 @@ long long ora_plan_brute(int n_heads, const int32_t *ext_diag_ptr, const int32_t
     if (tile_ptr) tile_ptr[n_heads * nqb] = (int32_t)n;
     free(isD);
     free(isC);
+    free(need);
     return n;
 }
 
@@ -342,91 +370,101 @@ static int first_ge(const int32_t *a, int n, long x) {
 }
 
 /* Routine 2 for one (head, query block): interval arithmetic over the offsets.
- * Candidate tiles are those a diagonal r in D_h crosses within the valid rows;
- * dmask / cmask are range queries on the sorted lists; "listed" checks, per set dmask
- * bit, whether the diagonal's cells in valid rows reach a column outside cmask.
- * Appends the block's tiles at out index n; returns the new n or a negative error. */
-static long long interval_block(const int32_t *D, int nd, const int32_t *C, int nc, int S, int qb,
-                                uint8_t *cand, long long n, long long capacity, int32_t *tile_kb,
+ * The diagonals r <= hi split into runs whose consecutive offsets differ by <= 128;
+ * a run [ra, rb] reaches exactly the contiguous keys [max(0, lo - rb), hi - ra] from
+ * the block's 128 rows, and runs further apart leave a gap of unreached keys (run0[k]
+ * is the first index of the run holding D[k]).  The
+ * runs, taken from the largest offset down (ascending keys), give the windows by
+ * stepping 128 keys at a time from max(run start, next allowed start).  dmask / cmask
+ * are range queries on the sorted lists; "listed" checks, per set dmask bit, whether
+ * the diagonal's cells in valid rows reach a column outside cmask.  Appends the
+ * block's tiles at out index n; returns the new n or a negative error. */
+static long long interval_block(const int32_t *D, const int32_t *run0, int nd, const int32_t *C,
+                                int nc, int S, int qb, long long n, long long capacity,
+                                int32_t *tile_key0,
                                 uint64_t *tile_dmask, uint64_t *tile_cmask, uint32_t *tile_flags) {
     const int T = ORA_TILE;
-    int nqb = (S + T - 1) / T;
-    long lo_i = (long)T * qb;
-    long hi_i = lo_i + T - 1 < S - 1 ? lo_i + T - 1 : S - 1;
-    int nrows = (int)(hi_i - lo_i + 1);
-    memset(cand, 0, (size_t)nqb);
-    for (int k = 0; k < nd; ++k) {
-        long r = D[k];
-        if (r > hi_i) break;
-        long jlo = lo_i - r > 0 ? lo_i - r : 0;
-        long jhi = hi_i - r;
-        for (long kb = jlo / T; kb <= jhi / T; ++kb) cand[kb] = 1;
-    }
-    for (int kb = 0; kb <= qb; ++kb) {
-        if (!cand[kb]) continue;
-        long base = (long)T * (qb - kb) - (T - 1); /* r of dmask bit 0 */
-        uint64_t dm[4] = {0, 0, 0, 0}, cm[2] = {0, 0};
-        for (int k = first_ge(D, nd, base); k < nd && D[k] <= base + 2 * T - 2; ++k)
-            set_bit(dm, (int)(D[k] - base));
-        for (int k = first_ge(C, nc, (long)T * kb); k < nc && C[k] < (long)T * (kb + 1); ++k)
-            set_bit(cm, (int)(C[k] - (long)T * kb));
-        int listed = 0;
-        for (int t = 0; t <= 2 * T - 2 && !listed; ++t) {
-            if (!get_bit(dm, t)) continue;
-            int delta = t - (T - 1); /* il - jl */
-            int il_lo = delta > 0 ? delta : 0;
-            int il_hi = T - 1;
-            if (T - 1 + delta < il_hi) il_hi = T - 1 + delta;
-            if (nrows - 1 < il_hi) il_hi = nrows - 1;
-            for (int il = il_lo; il <= il_hi; ++il) {
-                if (!get_bit(cm, il - delta)) {
-                    listed = 1;
-                    break;
+    long lo = (long)T * qb, hi = lo + T - 1;
+    long hi_valid = hi < S - 1 ? hi : S - 1;
+    int nrows = (int)(hi_valid - lo + 1);
+    int k = first_ge(D, nd, hi + 1) - 1; /* largest offset <= hi */
+    long next = 0;                          /* smallest allowed start of the next window */
+    while (k >= 0) {
+        int ks = run0[k];
+        long a = lo - D[k] > 0 ? lo - D[k] : 0, b = hi - D[ks];
+        for (long key0 = a > next ? a : next; key0 <= b; key0 += T) {
+            next = key0 + T;
+            long base = lo - key0 - (T - 1); /* r of dmask bit 0 */
+            uint64_t dm[4] = {0, 0, 0, 0}, cm[2] = {0, 0};
+            for (int q = first_ge(D, nd, base); q < nd && D[q] <= base + 2 * T - 2; ++q)
+                set_bit(dm, (int)(D[q] - base));
+            for (int q = first_ge(C, nc, key0); q < nc && C[q] < key0 + T; ++q)
+                set_bit(cm, (int)(C[q] - key0));
+            int listed = 0;
+            for (int t = 0; t <= 2 * T - 2 && !listed; ++t) {
+                if (!get_bit(dm, t)) continue;
+                int delta = t - (T - 1); /* il - jl */
+                int il_lo = delta > 0 ? delta : 0;
+                int il_hi = T - 1;
+                if (T - 1 + delta < il_hi) il_hi = T - 1 + delta;
+                if (nrows - 1 < il_hi) il_hi = nrows - 1;
+                for (int il = il_lo; il <= il_hi; ++il) {
+                    if (!get_bit(cm, il - delta)) {
+                        listed = 1;
+                        break;
+                    }
                 }
             }
+            if (!listed) continue;
+            int full = ((long)T * (qb + 1) <= S) && popcount256(dm) == 2 * T - 1 && cm[0] == 0 &&
+                       cm[1] == 0;
+            if (tile_key0) {
+                if (n >= capacity) return ORA_ERR_CAPACITY;
+                tile_key0[n] = (int32_t)key0;
+                memcpy(tile_dmask + 4 * n, dm, sizeof dm);
+                memcpy(tile_cmask + 2 * n, cm, sizeof cm);
+                tile_flags[n] = full ? 1u : 0u;
+            }
+            ++n;
         }
-        if (!listed) continue;
-        int full = (kb < qb) && ((long)T * (qb + 1) <= S) && popcount256(dm) == 2 * T - 1 &&
-                   cm[0] == 0 && cm[1] == 0;
-        if (tile_kb) {
-            if (n >= capacity) return ORA_ERR_CAPACITY;
-            tile_kb[n] = kb;
-            memcpy(tile_dmask + 4 * n, dm, sizeof dm);
-            memcpy(tile_cmask + 2 * n, cm, sizeof cm);
-            tile_flags[n] = full ? 1u : 0u;
-        }
-        ++n;
+        k = ks - 1;
     }
     return n;
+}
+
+/* run0[k] = first index of the run of D (consecutive offsets <= 128 apart) holding D[k]. */
+static void run_starts(const int32_t *D, int nd, int32_t *run0) {
+    for (int k = 0; k < nd; ++k) run0[k] = (k > 0 && D[k] - D[k - 1] <= ORA_TILE) ? run0[k - 1] : k;
 }
 
 /* Routine 2 over every (head, query block); same outputs as routine 1. */
 long long ora_plan_interval(int n_heads, const int32_t *ext_diag_ptr,
                             const int32_t *ext_diag_offsets, const int32_t *ext_vert_ptr,
                             const int32_t *ext_vert_cols, int S, long long capacity,
-                            int32_t *tile_ptr, int32_t *tile_kb, uint64_t *tile_dmask,
+                            int32_t *tile_ptr, int32_t *tile_key0, uint64_t *tile_dmask,
                             uint64_t *tile_cmask, uint32_t *tile_flags, int32_t *stripe_cnt) {
     if (n_heads < 0 || S <= 0) return ORA_ERR_INVALID;
     const int T = ORA_TILE;
     int nqb = (S + T - 1) / T;
-    uint8_t *cand = (uint8_t *)malloc((size_t)nqb);
-    if (!cand) return ORA_ERR_NOMEM;
+    int32_t *run0 = (int32_t *)malloc(sizeof(int32_t) * (size_t)(S + 1));
+    if (!run0) return ORA_ERR_NOMEM;
     long long n = 0;
     for (int h = 0; h < n_heads && n >= 0; ++h) {
         const int32_t *D = ext_diag_offsets + ext_diag_ptr[h];
         int nd = ext_diag_ptr[h + 1] - ext_diag_ptr[h];
         const int32_t *C = ext_vert_cols + ext_vert_ptr[h];
         int nc = ext_vert_ptr[h + 1] - ext_vert_ptr[h];
+        run_starts(D, nd, run0);
         for (int qb = 0; qb < nqb && n >= 0; ++qb) {
             if (tile_ptr) tile_ptr[h * nqb + qb] = (int32_t)n;
             long hi_i = (long)T * qb + T - 1 < S - 1 ? (long)T * qb + T - 1 : S - 1;
             if (stripe_cnt) stripe_cnt[h * nqb + qb] = count_le(C, nc, (int32_t)hi_i);
-            n = interval_block(D, nd, C, nc, S, qb, cand, n, capacity, tile_kb, tile_dmask,
+            n = interval_block(D, run0, nd, C, nc, S, qb, n, capacity, tile_key0, tile_dmask,
                                tile_cmask, tile_flags);
         }
     }
     if (tile_ptr && n >= 0) tile_ptr[n_heads * nqb] = (int32_t)n;
-    free(cand);
+    free(run0);
     return n;
 }
 
@@ -435,13 +473,13 @@ long long ora_plan_interval(int n_heads, const int32_t *ext_diag_ptr,
 long long ora_plan_items(int n_heads, const int32_t *ext_diag_ptr, const int32_t *ext_diag_offsets,
                          const int32_t *ext_vert_ptr, const int32_t *ext_vert_cols, int S,
                          int n_items, const int32_t *items, long long capacity, int32_t *item_ptr,
-                         int32_t *tile_kb, uint64_t *tile_dmask, uint64_t *tile_cmask,
+                         int32_t *tile_key0, uint64_t *tile_dmask, uint64_t *tile_cmask,
                          uint32_t *tile_flags, int32_t *stripe_cnt) {
     if (n_heads < 0 || S <= 0 || n_items < 0) return ORA_ERR_INVALID;
     const int T = ORA_TILE;
     int nqb = (S + T - 1) / T;
-    uint8_t *cand = (uint8_t *)malloc((size_t)nqb);
-    if (!cand) return ORA_ERR_NOMEM;
+    int32_t *run0 = (int32_t *)malloc(sizeof(int32_t) * (size_t)(S + 1));
+    if (!run0) return ORA_ERR_NOMEM;
     long long n = 0;
     for (int a = 0; a < n_items && n >= 0; ++a) {
         int h = items[2 * a], qb = items[2 * a + 1];
@@ -456,11 +494,12 @@ long long ora_plan_items(int n_heads, const int32_t *ext_diag_ptr, const int32_t
         if (item_ptr) item_ptr[a] = (int32_t)n;
         long hi_i = (long)T * qb + T - 1 < S - 1 ? (long)T * qb + T - 1 : S - 1;
         if (stripe_cnt) stripe_cnt[a] = count_le(C, nc, (int32_t)hi_i);
-        n = interval_block(D, nd, C, nc, S, qb, cand, n, capacity, tile_kb, tile_dmask, tile_cmask,
+        run_starts(D, nd, run0);
+        n = interval_block(D, run0, nd, C, nc, S, qb, n, capacity, tile_key0, tile_dmask, tile_cmask,
                            tile_flags);
     }
     if (item_ptr && n >= 0) item_ptr[n_items] = (int32_t)n;
-    free(cand);
+    free(run0);
     return n;
 }
 

@@ -47,7 +47,7 @@ class PlanStruct(C.Structure):
                 ("max_vert", C.c_int32), ("n_tiles", C.c_int64),
                 ("ext_diag_ptr", C.c_void_p), ("ext_diag_offsets", C.c_void_p),
                 ("ext_vert_ptr", C.c_void_p), ("ext_vert_cols", C.c_void_p),
-                ("tile_ptr", C.c_void_p), ("tile_kb", C.c_void_p), ("tile_dmask", C.c_void_p),
+                ("tile_ptr", C.c_void_p), ("tile_key0", C.c_void_p), ("tile_dmask", C.c_void_p),
                 ("tile_cmask", C.c_void_p), ("tile_flags", C.c_void_p), ("stripe_cnt", C.c_void_p)]
 
 
@@ -168,7 +168,7 @@ class Plan:
         self.ext_vert_ptr = torch.empty(H + 1, **i32)
         self.ext_vert_cols = torch.empty(max(sizes.n_vert, 1), **i32)
         self.tile_ptr = torch.empty(H * nqb + 1, **i32)
-        self.tile_kb = torch.empty(T, **i32)
+        self.tile_key0 = torch.empty(T, **i32)
         self.tile_dmask = torch.empty((T, 4), dtype=torch.int64, device=device)
         self.tile_cmask = torch.empty((T, 2), dtype=torch.int64, device=device)
         self.tile_flags = torch.empty(T, **i32)
@@ -177,7 +177,7 @@ class Plan:
         st.n_heads, st.S, st.nqb, st.max_vert = H, sizes.S, nqb, sizes.max_vert
         st.n_tiles = int(sizes.n_tiles)
         for name in ("ext_diag_ptr", "ext_diag_offsets", "ext_vert_ptr", "ext_vert_cols", "tile_ptr",
-                     "tile_kb", "tile_dmask", "tile_cmask", "tile_flags", "stripe_cnt"):
+                     "tile_key0", "tile_dmask", "tile_cmask", "tile_flags", "stripe_cnt"):
             setattr(st, name, getattr(self, name).data_ptr())
         self.struct = st
 
@@ -196,7 +196,7 @@ class Plan:
     def to_numpy(self):
         """Host copies in the oracle's layout (uint64 masks, uint32 flags)."""
         T = self.n_tiles
-        out = dict(tile_ptr=self.tile_ptr.cpu().numpy(), tile_kb=self.tile_kb[:T].cpu().numpy(),
+        out = dict(tile_ptr=self.tile_ptr.cpu().numpy(), tile_key0=self.tile_key0[:T].cpu().numpy(),
                    tile_dmask=self.tile_dmask[:T].cpu().numpy().view("uint64"),
                    tile_cmask=self.tile_cmask[:T].cpu().numpy().view("uint64"),
                    tile_flags=self.tile_flags[:T].cpu().numpy().view("uint32"),

@@ -14,8 +14,8 @@
 //   sparse_attn_fwd_kernel   persistent: one CTA per SM takes work items from a global
 //                            counter.  An item is a PAIR of consecutive 128-row query
 //                            blocks (2p, 2p+1) of one head; the CTA walks the merged
-//                            key-tile sequence of the two blocks (band tiles in
-//                            ascending key-tile order, then stripe tiles), so a key/value
+//                            key-tile sequence of the two blocks (band windows in
+//                            ascending order of their first key, then stripe tiles), so a key/value
 //                            tile wanted by both blocks is staged once and feeds both.
 //     warp 8         lane 0: scheduler (work counter -> ring of item descriptors) and
 //                    TMA producer of the K tiles of the merged sequence; each K stage
@@ -148,7 +148,7 @@ static_assert(sizeof(Shared) <= 1024, "barrier block too large");
 struct AttnParams {
     int S, H, Hkv, nqb, npad;
     const int32_t *tile_ptr;
-    const int32_t *tile_kb;
+    const int32_t *tile_key0;
     const uint64_t *tile_dmask;
     const uint64_t *tile_cmask;
     const uint32_t *tile_flags;
@@ -275,12 +275,12 @@ __device__ ItemDesc make_pair(const AttnParams &p, int idx) {
     return d;
 }
 
-// The merged key-tile sequence of an item: band tiles of both blocks in ascending key
-// tile (a tile listed by both is one step), then the stripe tiles (block 2p+1 holds at
-// least as many stripe columns as block 2p).  The next band entry of each block is
+// The merged key-tile sequence of an item: band tiles of both blocks in ascending order
+// of their first key (a window listed by both, same start, is one step), then the
+// stripe tiles (block 2p+1 holds at least as many stripe columns as block 2p).  The next band entry of each block is
 // loaded one step ahead so the producers do not wait on it.
 struct Steps {
-    const int32_t *kb[2];
+    const int32_t *key0[2];  // window start keys of each block's band tiles
     int nb[2], ns[2], i[2], a[2], an[2];
     int js;
     bool started[2], emitted;
@@ -289,12 +289,12 @@ struct Steps {
 __device__ __forceinline__ void steps_init(Steps &st, const AttnParams &p, const ItemDesc &d) {
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
-        st.kb[s] = p.tile_kb + d.tp0[s];
+        st.key0[s] = p.tile_key0 + d.tp0[s];
         st.nb[s] = d.nb[s];
         st.ns[s] = d.ns[s];
         st.i[s] = 0;
-        st.a[s] = d.nb[s] > 0 ? __ldg(st.kb[s]) : INT_MAX;
-        st.an[s] = d.nb[s] > 1 ? __ldg(st.kb[s] + 1) : INT_MAX;
+        st.a[s] = d.nb[s] > 0 ? __ldg(st.key0[s]) : INT_MAX;
+        st.an[s] = d.nb[s] > 1 ? __ldg(st.key0[s] + 1) : INT_MAX;
         st.started[s] = false;
     }
     st.js = 0;
@@ -311,12 +311,12 @@ __device__ __forceinline__ bool steps_next(Steps &st, bool &band, int &row0, uin
     const bool first = !st.emitted;
     st.emitted = true;
     if (st.a[0] != INT_MAX || st.a[1] != INT_MAX) {
-        const int kb = min(st.a[0], st.a[1]);
+        const int key0 = min(st.a[0], st.a[1]);
         band = true;
-        row0 = kb * kBN;
+        row0 = key0;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
-            if (st.a[s] != kb) continue;
+            if (st.a[s] != key0) continue;
             flags |= f_in(s);
             if (!st.started[s]) {
                 flags |= f_first(s);
@@ -324,7 +324,7 @@ __device__ __forceinline__ bool steps_next(Steps &st, bool &band, int &row0, uin
             }
             ++st.i[s];
             st.a[s] = st.an[s];
-            st.an[s] = (st.i[s] + 1 < st.nb[s]) ? __ldg(st.kb[s] + st.i[s] + 1) : INT_MAX;
+            st.an[s] = (st.i[s] + 1 < st.nb[s]) ? __ldg(st.key0[s] + st.i[s] + 1) : INT_MAX;
             if (st.i[s] == st.nb[s] && st.ns[s] == 0) flags |= f_last(s);
         }
         return true;
@@ -1044,7 +1044,7 @@ extern "C" int sparse_attn_fwd(const void *Q, const void *K, const void *V, int 
     SSA_CHECK_ARG(plan->S == S && plan->n_heads == H_q && plan->nqb == (S + kBM - 1) / kBM,
                   "sparse_attn_fwd: plan (S=%d heads=%d) does not match S=%d H_q=%d", plan->S,
                   plan->n_heads, S, H_q);
-    SSA_CHECK_ARG(plan->tile_ptr && plan->tile_kb && plan->tile_dmask && plan->tile_cmask &&
+    SSA_CHECK_ARG(plan->tile_ptr && plan->tile_key0 && plan->tile_dmask && plan->tile_cmask &&
                       plan->tile_flags && plan->stripe_cnt && plan->ext_vert_ptr &&
                       plan->ext_vert_cols,
                   "sparse_attn_fwd: null plan array");
@@ -1068,7 +1068,7 @@ extern "C" int sparse_attn_fwd(const void *Q, const void *K, const void *V, int 
     p.nqb = plan->nqb;
     p.npad = static_cast<int>(round_up128(static_cast<size_t>(plan->max_vert)));
     p.tile_ptr = plan->tile_ptr;
-    p.tile_kb = plan->tile_kb;
+    p.tile_key0 = plan->tile_key0;
     p.tile_dmask = plan->tile_dmask;
     p.tile_cmask = plan->tile_cmask;
     p.tile_flags = plan->tile_flags;

@@ -5,7 +5,8 @@
 //
 // In list form the extension keeps every diagonal r < S and every column c < S.  The
 // tile plan is this library's own layout of that mask for the attention kernel:
-// for each (head, query block) the ascending key tiles the band touches, each with a
+// for each (head, query block) the ascending 128-key windows the band reaches (each
+// starting where the band's keys start, not at a multiple of 128), each with a
 // 255-bit local-diagonal mask, a 128-bit column-exclusion mask and a FULL flag, plus
 // the number of columns the stripe phase covers (exact semantics in ssa.h).
 //
@@ -13,7 +14,9 @@
 //   validate_lists_kernel  lists sorted, unique, non-negative; kept counts r < S, c < S
 //   exclusive_scan_kernel  single-block scan (list offsets, tile offsets)
 //   extend_copy_kernel     the extended CSR lists
-//   plan_tiles_kernel      count pass / fill pass of the band tiles + stripe counts
+//   run_start_kernel       per head: first index of the run (offsets <= 128 apart)
+//                          holding each kept diagonal
+//   plan_tiles_kernel      count pass / fill pass of the band windows + stripe counts
 //   plan_totals_kernel     totals for the sizing pass
 #include "common.cuh"
 
@@ -37,13 +40,14 @@ struct PlanParams {
     int32_t *ext_counts;   // [2H]: kept diagonals, kept columns per head
     int32_t *ext_scan;     // [2 (H+1)]: exclusive scans of the two count arrays
     int32_t *tile_counts;  // [H*nqb]
+    int32_t *run0;         // [H][S]: run start index of each kept diagonal
     int32_t *tile_ptr;     // [H*nqb + 1] (workspace in the sizing pass, plan in the fill pass)
     Totals *totals;
     int32_t *ws_status;
     int32_t *dev_status;
     // fill pass outputs
     int64_t capacity;
-    int32_t *tile_kb;
+    int32_t *tile_key0;
     uint64_t *tile_dmask;
     uint64_t *tile_cmask;
     uint32_t *tile_flags;
@@ -128,6 +132,39 @@ __global__ void extend_copy_kernel(PlanParams p) {
     }
 }
 
+// run0[k] = the largest k' <= k with k' == 0 or D[k'] - D[k'-1] > 128: the first index of
+// the run of offsets (each within 128 of the previous one) that holds D[k].  A run
+// reaches one contiguous range of keys from the 128 rows of a query block.  One block
+// per head: an inclusive max-scan of the run boundaries.
+__global__ void __launch_bounds__(kScanThreads) run_start_kernel(PlanParams p) {
+    __shared__ int32_t s_warp[kScanThreads / 32];
+    __shared__ int32_t s_carry;
+    const int h = blockIdx.x;
+    const int32_t *D = p.doff + p.dptr[h];
+    const int nd = p.ext_counts[2 * h];
+    int32_t *run0 = p.run0 + static_cast<size_t>(h) * p.S;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) s_carry = 0;
+    __syncthreads();
+    for (int start = 0; start < nd; start += kScanThreads) {
+        const int k = start + threadIdx.x;
+        int x = (k < nd && (k == 0 || __ldg(D + k) - __ldg(D + k - 1) > kTile)) ? k : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) x = max(x, __shfl_up_sync(0xffffffffu, x, o) * (lane >= o ? 1 : 0));
+        if (lane == 31) s_warp[warp] = x;
+        __syncthreads();
+        int before = s_carry, total = s_carry;
+        for (int w = 0; w < kScanThreads / 32; ++w) {
+            if (w < warp) before = max(before, s_warp[w]);
+            total = max(total, s_warp[w]);
+        }
+        if (k < nd) run0[k] = max(x, before);
+        __syncthreads();
+        if (threadIdx.x == 0) s_carry = total;
+        __syncthreads();
+    }
+}
+
 __device__ __forceinline__ void set_bit_range(uint64_t (&w)[4], int a, int b) {  // inclusive
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -140,10 +177,11 @@ __device__ __forceinline__ void set_bit_range(uint64_t (&w)[4], int a, int b) { 
     }
 }
 
-// Evaluate tile (qb, kb) of one head.  Returns 0 (not listed), 1 (listed), 2 (FULL).
-__device__ int eval_tile(const int32_t *D, int nD, const int32_t *C, int nC, int S, int qb, int kb,
-                         uint64_t (&dm)[4], uint64_t (&cm)[2]) {
-    const int base = kTile * (qb - kb) - (kTile - 1);  // r of dmask bit 0
+// Evaluate the window of keys key0 .. key0+127 for query block qb of one head.
+// Returns 0 (not listed), 1 (listed), 2 (FULL).
+__device__ int eval_window(const int32_t *D, int nD, const int32_t *C, int nC, int S, int qb, int key0,
+                           uint64_t (&dm)[4], uint64_t (&cm)[2]) {
+    const int base = kTile * qb - key0 - (kTile - 1);  // r of dmask bit 0
     const int lb = lower_bound_i32(D, nD, max(base, 0));
     const int ub = lower_bound_i32(D, nD, base + 2 * kTile - 1);
     if (lb == ub) return 0;
@@ -158,9 +196,9 @@ __device__ int eval_tile(const int32_t *D, int nD, const int32_t *C, int nC, int
         }
     }
     cm[0] = cm[1] = 0;
-    const int cl = lower_bound_i32(C, nC, kTile * kb);
+    const int cl = lower_bound_i32(C, nC, key0);
     for (int k = cl; k < nC; ++k) {
-        const int jl = __ldg(C + k) - kTile * kb;
+        const int jl = __ldg(C + k) - key0;
         if (jl >= kTile) break;
         cm[jl >> 6] |= 1ull << (jl & 63);
     }
@@ -180,7 +218,8 @@ __device__ int eval_tile(const int32_t *D, int nD, const int32_t *C, int nC, int
     }
     if (!listed) return 0;
     const bool all = dm[0] == ~0ull && dm[1] == ~0ull && dm[2] == ~0ull && dm[3] == (~0ull >> 1);
-    const bool full = kb < qb && kTile * (qb + 1) <= S && all && (cm[0] | cm[1]) == 0;
+    // all 255 offsets present implies r >= 0 everywhere, i.e. the window is left of the diagonal
+    const bool full = kTile * (qb + 1) <= S && all && (cm[0] | cm[1]) == 0;
     return full ? 2 : 1;
 }
 
@@ -194,41 +233,52 @@ __global__ void __launch_bounds__(128) plan_tiles_kernel(PlanParams p) {
     const int32_t *D = p.doff + p.dptr[h];
     const int32_t *C = p.vcol + p.vptr[h];
     const int nD = p.ext_counts[2 * h], nC = p.ext_counts[2 * h + 1];
-    const int lo_i = kTile * qb, hi_i = min(kTile * qb + kTile - 1, p.S - 1);
-    if (FILL && lane == 0) p.stripe_cnt[item] = lower_bound_i32(C, nC, hi_i + 1);
-    // key tiles reachable by some diagonal r <= hi_i
-    const int nvalid = lower_bound_i32(D, nD, hi_i + 1);
+    // windows are chosen over all 128 rows of the block (lo .. hi), even past S
+    const int lo = kTile * qb, hi = lo + kTile - 1;
+    if (FILL && lane == 0) p.stripe_cnt[item] = lower_bound_i32(C, nC, min(hi, p.S - 1) + 1);
+    const int32_t *run0 = p.run0 + static_cast<size_t>(h) * p.S;
+    // Runs of offsets from the largest r <= hi down, i.e. in ascending keys: run [ra, rb]
+    // reaches keys [max(0, lo - rb), hi - ra]; windows step 128 keys from the larger of
+    // that start and the end of the previous window.
+    int k = lower_bound_i32(D, nD, hi + 1) - 1;
+    int next = 0;
     int count = 0;
-    if (nvalid > 0) {
-        const int rmin = __ldg(D), rmax = __ldg(D + nvalid - 1);
-        const int kb_lo = max(0, lo_i - rmax) / kTile;
-        const int kb_hi = (hi_i - rmin) / kTile;
-        int64_t pos = FILL ? p.tile_ptr[item] : 0;
-        for (int kb0 = kb_lo; kb0 <= kb_hi; kb0 += 32) {
-            const int kb = kb0 + lane;
-            uint64_t dm[4], cm[2];
-            int r = 0;
-            if (kb <= kb_hi) r = eval_tile(D, nD, C, nC, p.S, qb, kb, dm, cm);
-            const uint32_t ball = __ballot_sync(0xffffffffu, r != 0);
-            if (FILL && r) {
-                const int64_t t = pos + __popc(ball & ((1u << lane) - 1u));
-                if (t < p.capacity) {
-                    p.tile_kb[t] = kb;
-                    uint64_t *dst = p.tile_dmask + 4 * t;
-                    dst[0] = dm[0];
-                    dst[1] = dm[1];
-                    dst[2] = dm[2];
-                    dst[3] = dm[3];
-                    p.tile_cmask[2 * t] = cm[0];
-                    p.tile_cmask[2 * t + 1] = cm[1];
-                    p.tile_flags[t] = (r == 2) ? 1u : 0u;
-                } else {
-                    report(p.dev_status, SSA_ERR_CAPACITY);
+    int64_t pos = FILL ? p.tile_ptr[item] : 0;
+    while (k >= 0) {
+        const int ks = run0[k];
+        const int a = max(0, lo - __ldg(D + k)), b = hi - __ldg(D + ks);
+        const int s0 = max(a, next);
+        if (s0 <= b) {
+            const int nw = (b - s0) / kTile + 1;
+            for (int w0 = 0; w0 < nw; w0 += 32) {
+                const int w = w0 + lane;
+                const int key0 = s0 + kTile * w;
+                uint64_t dm[4], cm[2];
+                int r = 0;
+                if (w < nw) r = eval_window(D, nD, C, nC, p.S, qb, key0, dm, cm);
+                const uint32_t ball = __ballot_sync(0xffffffffu, r != 0);
+                if (FILL && r) {
+                    const int64_t t = pos + __popc(ball & ((1u << lane) - 1u));
+                    if (t < p.capacity) {
+                        p.tile_key0[t] = key0;
+                        uint64_t *dst = p.tile_dmask + 4 * t;
+                        dst[0] = dm[0];
+                        dst[1] = dm[1];
+                        dst[2] = dm[2];
+                        dst[3] = dm[3];
+                        p.tile_cmask[2 * t] = cm[0];
+                        p.tile_cmask[2 * t + 1] = cm[1];
+                        p.tile_flags[t] = (r == 2) ? 1u : 0u;
+                    } else {
+                        report(p.dev_status, SSA_ERR_CAPACITY);
+                    }
                 }
+                pos += __popc(ball);
+                count += __popc(ball);
             }
-            pos += __popc(ball);
-            count += __popc(ball);
+            next = s0 + kTile * nw;
         }
+        k = ks - 1;
     }
     if (!FILL && lane == 0) p.tile_counts[item] = count;
 }
@@ -282,7 +332,8 @@ extern "C" size_t sparse_pattern_extend_ws_bytes(int n_heads, int S) {
     const size_t items = static_cast<size_t>(n_heads) * nqb;
     return align_up(sizeof(Totals)) + align_up(sizeof(int32_t) * 2 * n_heads) +
            align_up(sizeof(int32_t) * 2 * (n_heads + 1)) + align_up(sizeof(int32_t) * items) +
-           align_up(sizeof(int32_t) * (items + 1)) + 256;
+           align_up(sizeof(int32_t) * (items + 1)) +
+           align_up(sizeof(int32_t) * static_cast<size_t>(n_heads) * static_cast<size_t>(S)) + 256;
 }
 
 extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
@@ -323,6 +374,8 @@ extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
     p.tile_counts = reinterpret_cast<int32_t *>(w);
     w += align_up(sizeof(int32_t) * n_heads * nqb);
     int32_t *ws_tile_ptr = reinterpret_cast<int32_t *>(w);
+    w += align_up(sizeof(int32_t) * (n_heads * nqb + 1));
+    p.run0 = reinterpret_cast<int32_t *>(w);
     p.dev_status = dev_status;
 
     const int items = n_heads * nqb;
@@ -333,6 +386,8 @@ extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
         SSA_CHECK_ARG(sizes, "sparse_pattern_extend: sizes must not be NULL in the sizing pass");
         p.tile_ptr = ws_tile_ptr;
         validate_lists_kernel<<<n_heads, 128, 0, s>>>(p);
+        SSA_LAUNCH_CHECK();
+        run_start_kernel<<<n_heads, kScanThreads, 0, s>>>(p);
         SSA_LAUNCH_CHECK();
         plan_tiles_kernel<false><<<tile_grid, 128, 0, s>>>(p);
         SSA_LAUNCH_CHECK();
@@ -362,14 +417,14 @@ extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
                   "(%d, %d, %d)",
                   plan->n_heads, plan->S, plan->nqb, n_heads, S, nqb);
     SSA_CHECK_ARG(plan->ext_diag_ptr && plan->ext_diag_offsets && plan->ext_vert_ptr &&
-                      plan->ext_vert_cols && plan->tile_ptr && plan->tile_kb &&
+                      plan->ext_vert_cols && plan->tile_ptr && plan->tile_key0 &&
                       plan->tile_dmask && plan->tile_cmask && plan->tile_flags &&
                       plan->stripe_cnt,
                   "sparse_pattern_extend: null plan array");
     SSA_CHECK_ARG(plan->n_tiles >= 0, "sparse_pattern_extend: negative tile capacity");
     p.tile_ptr = plan->tile_ptr;
     p.capacity = plan->n_tiles;
-    p.tile_kb = plan->tile_kb;
+    p.tile_key0 = plan->tile_key0;
     p.tile_dmask = plan->tile_dmask;
     p.tile_cmask = plan->tile_cmask;
     p.tile_flags = plan->tile_flags;
@@ -387,6 +442,8 @@ extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
                                                      p.ext_scan + (n_heads + 1));
     SSA_LAUNCH_CHECK();
     extend_copy_kernel<<<n_heads, 128, 0, s>>>(p);
+    SSA_LAUNCH_CHECK();
+    run_start_kernel<<<n_heads, kScanThreads, 0, s>>>(p);
     SSA_LAUNCH_CHECK();
     plan_tiles_kernel<false><<<tile_grid, 128, 0, s>>>(p);
     SSA_LAUNCH_CHECK();

@@ -9,7 +9,7 @@ from structured_sparse_attention_b200 import inputs
 
 pytestmark = pytest.mark.gpu
 
-FIELDS = ("tile_ptr", "tile_kb", "tile_dmask", "tile_cmask", "tile_flags", "stripe_cnt")
+FIELDS = ("tile_ptr", "tile_key0", "tile_dmask", "tile_cmask", "tile_flags", "stripe_cnt")
 
 
 def _gpu_plan(diags, verts, S):
@@ -73,7 +73,7 @@ def _sampled(ora, plan, ext, S, seed, n=48):
     for a, (h, qb) in enumerate(items):
         g0, g1 = got["tile_ptr"][h * nqb + qb], got["tile_ptr"][h * nqb + qb + 1]
         r0, r1 = ref["item_ptr"][a], ref["item_ptr"][a + 1]
-        for k in ("tile_kb", "tile_dmask", "tile_cmask", "tile_flags"):
+        for k in ("tile_key0", "tile_dmask", "tile_cmask", "tile_flags"):
             np.testing.assert_array_equal(got[k][g0:g1], ref[k][r0:r1], err_msg=f"{k} h={h} qb={qb}")
         assert got["stripe_cnt"][h * nqb + qb] == ref["stripe_cnt"][a]
 

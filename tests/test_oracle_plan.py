@@ -78,14 +78,14 @@ def test_extend_filters_and_validates(ora):
 
 
 def test_plan_main_diagonal_only(ora):
-    # D = {0}: each query block has exactly its own diagonal tile, holding only the
-    # local diagonal t = 127; never FULL; no stripes.
+    # D = {0}: each query block has exactly one window, starting at its own first row
+    # and holding only the local diagonal t = 127; never FULL; no stripes.
     for S in (256, 300):
         ext = _ext(ora, [np.array([0], np.int32)], [np.array([], np.int32)], S)
         p = ora.plan(ext, S)
         nqb = (S + T - 1) // T
         assert p["n_tiles"] == nqb
-        assert p["tile_kb"].tolist() == list(range(nqb))
+        assert p["tile_key0"].tolist() == [T * qb for qb in range(nqb)]
         for t in range(nqb):
             assert p["tile_dmask"][t].tolist() == [0, 1 << 63, 0, 0]
             assert p["tile_cmask"][t].tolist() == [0, 0]
@@ -100,9 +100,9 @@ def test_plan_full_causal(ora):
     assert p["n_tiles"] == 4 * 5 // 2
     for qb in range(4):
         a, b = p["tile_ptr"][qb], p["tile_ptr"][qb + 1]
-        assert p["tile_kb"][a:b].tolist() == list(range(qb + 1))
+        assert p["tile_key0"][a:b].tolist() == [T * kb for kb in range(qb + 1)]
         for t in range(a, b):
-            kb = p["tile_kb"][t]
+            kb = p["tile_key0"][t] // T
             assert p["tile_flags"][t] == (1 if kb < qb else 0)
             if kb == qb:
                 # only r >= 0, i.e. t >= 127
@@ -111,8 +111,8 @@ def test_plan_full_causal(ora):
 
 
 def test_plan_column_owned_by_stripes(ora):
-    # D = {128}, C = {0..127}: every band element of tile (qb=1, kb=0) sits in a column
-    # of C, so the tile is not listed; the stripe phase owns those pairs.
+    # D = {128}, C = {0..127}: the only window of block 1 (keys 0..127) holds band
+    # elements in columns of C only, so it is not listed; the stripe phase owns them.
     S = 256
     ext = _ext(ora, [np.array([128], np.int32)], [np.arange(128, dtype=np.int32)], S)
     p = ora.plan(ext, S)
@@ -122,7 +122,7 @@ def test_plan_column_owned_by_stripes(ora):
     ext = _ext(ora, [np.arange(S, dtype=np.int32)], [np.array([5], np.int32)], S)
     p = ora.plan(ext, S)
     t = p["tile_ptr"][1]
-    assert p["tile_kb"][t] == 0 and p["tile_flags"][t] == 0
+    assert p["tile_key0"][t] == 0 and p["tile_flags"][t] == 0
     assert p["tile_cmask"][t].tolist() == [1 << 5, 0]
 
 
@@ -131,7 +131,7 @@ def test_plan_ragged_tail_is_not_full(ora):
     ext = _ext(ora, [np.arange(S, dtype=np.int32)], [np.array([], np.int32)], S)
     p = ora.plan(ext, S)
     a, b = p["tile_ptr"][1], p["tile_ptr"][2]
-    assert p["tile_kb"][a:b].tolist() == [0, 1]
+    assert p["tile_key0"][a:b].tolist() == [0, T]
     assert p["tile_flags"][a:b].tolist() == [0, 0]
 
 
@@ -144,7 +144,7 @@ def test_plan_routines_agree_and_count_pairs(ora, seed):
     ext = _ext(ora, diags, verts, S)
     pb = ora.plan(ext, S, "brute")
     pi = ora.plan(ext, S, "interval")
-    for k in ("tile_ptr", "tile_kb", "tile_dmask", "tile_cmask", "tile_flags", "stripe_cnt"):
+    for k in ("tile_ptr", "tile_key0", "tile_dmask", "tile_cmask", "tile_flags", "stripe_cnt"):
         np.testing.assert_array_equal(pb[k], pi[k], err_msg=k)
     nnz = ora.nnz(ext, S)
     for h in range(H):
@@ -165,6 +165,42 @@ def test_plan_items_equals_full_plan(ora):
     for a, (h, qb) in enumerate(items):
         f0, f1 = full["tile_ptr"][h * nqb + qb], full["tile_ptr"][h * nqb + qb + 1]
         s0, s1 = sel["item_ptr"][a], sel["item_ptr"][a + 1]
-        for k in ("tile_kb", "tile_dmask", "tile_cmask", "tile_flags"):
+        for k in ("tile_key0", "tile_dmask", "tile_cmask", "tile_flags"):
             np.testing.assert_array_equal(full[k][f0:f1], sel[k][s0:s1])
         assert full["stripe_cnt"][h * nqb + qb] == sel["stripe_cnt"][a]
+
+
+def test_plan_windows_follow_an_unaligned_band(ora):
+    # D = {100..399} (300 contiguous offsets).  Block 5 (rows 640..767) reaches keys
+    # 640 - 399 = 241 .. 767 - 100 = 667, i.e. 427 keys: four windows starting at 241,
+    # 369, 497, 625 (key tiles aligned to multiples of 128 would need five: 1..5).
+    S = 1024
+    ext = _ext(ora, [np.arange(100, 400, dtype=np.int32)], [np.array([], np.int32)], S)
+    for routine in ("brute", "interval"):
+        p = ora.plan(ext, S, routine)
+        a, b = p["tile_ptr"][5], p["tile_ptr"][6]
+        assert p["tile_key0"][a:b].tolist() == [241, 369, 497, 625]
+        # window 241: r = 640 - 241 + t - 127 = 272 + t, so bits t = 0..127 (r 272..399)
+        assert p["tile_dmask"][a].tolist() == [2**64 - 1, 2**64 - 1, 0, 0]
+        # window 625: r = t - 112, so bits t = 212..254 (r 100..142)
+        want = 0
+        for t in range(212, 255):
+            want |= 1 << t
+        assert p["tile_dmask"][a + 3].tolist() == [(want >> (64 * w)) & (2**64 - 1) for w in range(4)]
+        # window 369 sees r = 144..398, all in D: FULL; windows 241 (r 272..526), 497
+        # (r 16..270) and 625 (r -112..142) see D only partly
+        assert p["tile_flags"][a:b].tolist() == [0, 1, 0, 0]
+        # block 0 (rows 0..127) reaches keys 0..27 only (r = 100 from rows 100..127)
+        assert p["tile_key0"][p["tile_ptr"][0]:p["tile_ptr"][1]].tolist() == [0]
+
+
+def test_plan_windows_skip_gaps_between_diagonal_runs(ora):
+    # Two runs far apart, D = {0, 1} and {700}: block 7 (rows 896..1023) reaches keys
+    # 196..323 from r = 700 and 895..1023 from the first run; nothing is listed in the
+    # gap, and the 129 keys of the first run take two windows (895 and 1023).
+    S = 1024
+    ext = _ext(ora, [np.array([0, 1, 700], np.int32)], [np.array([], np.int32)], S)
+    for routine in ("brute", "interval"):
+        p = ora.plan(ext, S, routine)
+        a, b = p["tile_ptr"][7], p["tile_ptr"][8]
+        assert p["tile_key0"][a:b].tolist() == [196, 895, 1023]
