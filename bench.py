@@ -34,7 +34,7 @@ METRIC = "sparse-attn prefill tokens/s & effective TFLOP/s vs roofline, per mask
 UNIT = "tokens/s"
 
 # Kernels launched per call (the library's own kernels).
-LAUNCHES = {"capture": 3, "extend_fill": 7, "attn": 2}
+LAUNCHES = {"capture": 3, "extend_fill": 8, "attn": 2}
 
 WORKLOADS = {
     # name: (H_q, H_kv, S, d, pattern builder)
