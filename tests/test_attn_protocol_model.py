@@ -1,0 +1,402 @@
+"""Discrete-event model of the barrier protocol of sparse_attn_fwd_kernel (CPU only).
+
+The attention kernel's roles (scheduler + K producer, Q/V producer, one MMA issuer per
+slot with the turn token, one softmax per slot) are re-enacted here with the same loop
+structure, barrier counts and phase counters, over random work items (items without
+tiles, items where one slot has no tile, windows shared by both slots, stripe tiles)
+and random latencies for the copies, the MMAs, the softmax and the epilogue.  The
+tensor pipe executes MMA groups in issue order; a commit completes when every group
+issued before it has completed.
+
+Checked in every run:
+  * no deadlock: every role finishes;
+  * every parity wait targets the barrier's current or previous phase, never one that
+    has already come round again (a waiter two phases behind would wait forever);
+  * a K or V stage is refilled only after every MMA that reads its previous content
+    has completed, and a Q buffer only after the last QK^T that reads it;
+  * the first PV of an item (which overwrites O) is issued only after the epilogue of
+    the slot's previous item has read O;
+  * every tile the producers stage is consumed by exactly the slots that list it.
+The model also shows that releasing a V stage without first observing its fill (the
+rule the issuers follow) breaks the phase invariant for runs of tile-less items.
+"""
+
+import heapq
+import random
+
+import pytest
+
+NK, NV, RING = 2, 3, 4
+
+
+class ProtocolError(AssertionError):
+    pass
+
+
+class Barrier:
+    def __init__(self, sim, name, count):
+        self.sim, self.name, self.count = sim, name, count
+        self.pending = count
+        self.completions = 0
+        self.waiters = []  # (agent, phase)
+
+    def arrive(self, n=1):
+        self.pending -= n
+        if self.pending < 0:
+            raise ProtocolError(f"{self.name}: more arrivals than the count in one phase")
+        if self.pending == 0:
+            self.completions += 1
+            self.pending = self.count
+            woken, self.waiters = self.waiters, []
+            for agent, phase in woken:
+                self.sim.wait_on(agent, self, phase)
+
+
+class Sim:
+    def __init__(self, seed, items, release_without_fill=False):
+        self.rng = random.Random(seed)
+        self.t = 0
+        self.q = []
+        self.seq = 0
+        self.items = items
+        self.release_without_fill = release_without_fill
+        B = lambda n, c: Barrier(self, n, c)
+        self.item_full = [B(f"item_full{r}", 1) for r in range(RING)]
+        self.item_empty = [B(f"item_empty{r}", 1 + 2) for r in range(RING)]  # Q/V producer + 2 softmax
+        self.q_full = [B(f"q_full{s}", 1) for s in range(2)]
+        self.q_empty = [B(f"q_empty{s}", 1) for s in range(2)]
+        self.k_full = [B(f"k_full{i}", 1) for i in range(NK)]
+        self.k_empty = [B(f"k_empty{i}", 2) for i in range(NK)]
+        self.v_full = [B(f"v_full{i}", 1) for i in range(NV)]
+        self.v_empty = [B(f"v_empty{i}", 2) for i in range(NV)]
+        self.s_full = [B(f"s_full{s}", 1) for s in range(2)]
+        self.p_full = [B(f"p_full{s}", 1) for s in range(2)]
+        self.o_full = [B(f"o_full{s}", 1) for s in range(2)]
+        self.ring = [None] * RING
+        self.kflags = [None] * NK
+        self.turn = 0
+        self.turn_waiters = []
+        self.pipe_free_at = 0
+        self.readers = {}  # buffer -> completion time of the last MMA reading it
+        self.epi_done = [0, 0]   # epilogues that have read O, per slot
+        self.first_pv = [0, 0]   # first PVs of items issued, per slot
+        self.waiting = {}        # agent -> (barrier, phase) of its last wait
+        self.k_content, self.v_content = [None] * NK, [None] * NV
+        self.consumed = []
+        self.done = set()
+        self.agents = {}
+
+    # -- scheduling -------------------------------------------------------------------
+    def at(self, t, agent, value=None):
+        self.seq += 1
+        heapq.heappush(self.q, (t, self.seq, agent, value))
+
+    def wait_on(self, agent, bar, phase):
+        # parity wait for completion of `phase` (an explicit phase index)
+        self.waiting[agent] = (bar, phase)
+        if bar.completions >= phase + 2:
+            raise ProtocolError(f"{bar.name}: waiter {agent} targets phase {phase}, "
+                                f"but {bar.completions} phases have completed")
+        if bar.completions >= phase + 1:
+            self.at(self.t + self.rng.randint(1, 20), agent)
+        else:
+            bar.waiters.append((agent, phase))
+
+    def later(self, dt, fn):
+        self.seq += 1
+        heapq.heappush(self.q, (self.t + dt, self.seq, None, fn))
+
+    # -- tensor pipe ------------------------------------------------------------------
+    def mma(self, duration, reads):
+        start = max(self.t, self.pipe_free_at)
+        self.pipe_free_at = start + duration
+        for buf in reads:
+            self.readers[buf] = max(self.readers.get(buf, 0), self.pipe_free_at)
+        return self.pipe_free_at
+
+    def commit(self, bar):
+        done = max(self.t, self.pipe_free_at)
+        self.later(done - self.t + 1, lambda: bar.arrive())
+
+    def tma(self, bar, buf):
+        if self.readers.get(buf, 0) > self.t:
+            raise ProtocolError(f"{buf} refilled at {self.t} while an MMA reads it until {self.readers[buf]}")
+        self.later(self.rng.randint(200, 3000), lambda: bar.arrive())
+
+    def run(self, limit=10 ** 9):
+        self.agents = {"kprod": k_producer(self), "qvprod": qv_producer(self),
+                       "mma0": mma_issuer(self, 0), "mma1": mma_issuer(self, 1),
+                       "sm0": softmax(self, 0), "sm1": softmax(self, 1)}
+        for name in self.agents:
+            self.at(0, name)
+        while self.q:
+            t, _, agent, value = heapq.heappop(self.q)
+            self.t = t
+            if t > limit:
+                break
+            if agent is None:
+                value()
+                continue
+            gen = self.agents[agent]
+            if agent in self.waiting:
+                bar, phase = self.waiting.pop(agent)
+                if bar.completions != phase + 1:  # a poll here would see the wrong parity
+                    raise ProtocolError(f"{bar.name}: {agent} resumes for phase {phase} after "
+                                        f"{bar.completions} completions")
+            try:
+                cmd = next(gen)
+            except StopIteration:
+                self.done.add(agent)
+                continue
+            kind = cmd[0]
+            if kind == "wait":
+                self.wait_on(agent, cmd[1], cmd[2])
+            elif kind == "delay":
+                self.at(self.t + cmd[1], agent)
+            elif kind == "turn":
+                if self.turn == cmd[1]:
+                    self.at(self.t + 1, agent)
+                else:
+                    self.turn_waiters.append((agent, cmd[1]))
+        if len(self.done) != len(self.agents):
+            stuck = sorted(set(self.agents) - self.done)
+            raise ProtocolError(f"deadlock: {stuck} never finished")
+
+    def pass_turn(self, value):
+        self.turn = value
+        keep = []
+        for agent, want in self.turn_waiters:
+            if want == value:
+                self.at(self.t + 1, agent)
+            else:
+                keep.append((agent, want))
+        self.turn_waiters = keep
+
+
+# ---------------------------------------------------------------------------------------
+# Work items and their merged step sequence (the rule of the kernel's steps_next)
+# ---------------------------------------------------------------------------------------
+
+def random_item(rng):
+    kind = rng.random()
+    if kind < 0.15:
+        return ([], 0, [], 0)  # no tile at all
+    keys = sorted(rng.sample(range(0, 40), rng.randint(0, 10)))
+    k0 = [k for k in keys if rng.random() < 0.8]
+    k1 = [k for k in keys if rng.random() < 0.8] + [k for k in range(41, 41 + rng.randint(0, 2))]
+    ns0 = rng.randint(0, 2)
+    ns1 = max(ns0, rng.randint(0, 2))
+    if kind < 0.3:
+        k0, ns0 = [], 0  # slot 0 without tiles
+    return (k0, ns0, k1, ns1)
+
+
+def steps(item):
+    """Merged steps: (tile id or None, flags) with flags {slot: (first, last)}."""
+    k0, ns0, k1, ns1 = item
+    lists, ns = [list(k0), list(k1)], [ns0, ns1]
+    out, started = [], [False, False]
+    nb = [len(k0), len(k1)]
+    idx = [0, 0]
+    while idx[0] < nb[0] or idx[1] < nb[1]:
+        key = min(lists[s][idx[s]] for s in range(2) if idx[s] < nb[s])
+        fl = {}
+        for s in range(2):
+            if idx[s] < nb[s] and lists[s][idx[s]] == key:
+                first = not started[s]
+                started[s] = True
+                idx[s] += 1
+                fl[s] = (first, idx[s] == nb[s] and ns[s] == 0)
+        out.append((("band", key), fl))
+    for js in range(max(ns)):
+        fl = {}
+        for s in range(2):
+            if js < ns[s]:
+                first = not started[s]
+                started[s] = True
+                fl[s] = (first, js == ns[s] - 1)
+        out.append((("stripe", js), fl))
+    if not out:
+        out.append((None, {}))  # no-op step
+    return out
+
+
+def tiles_of(item, s):
+    k0, ns0, k1, ns1 = item
+    keys, ns = (k0, ns0) if s == 0 else (k1, ns1)
+    return [("band", k) for k in keys] + [("stripe", j) for j in range(ns)]
+
+
+# ---------------------------------------------------------------------------------------
+# Roles
+# ---------------------------------------------------------------------------------------
+
+def k_producer(sim):
+    tk = 0
+    for m, item in enumerate(sim.items + [None]):
+        slot = m % RING
+        if m >= RING:
+            yield ("wait", sim.item_empty[slot], m // RING - 1)
+        sim.ring[slot] = item
+        sim.item_full[slot].arrive()
+        if item is None:
+            break
+        for tile, fl in steps(item):
+            si = tk % NK
+            if tk >= NK:
+                yield ("wait", sim.k_empty[si], tk // NK - 1)
+            sim.kflags[si] = (tile, fl, False)
+            if tile is None:
+                sim.k_full[si].arrive()
+            else:
+                sim.k_content[si] = tile
+                sim.tma(sim.k_full[si], f"K{si}")
+            tk += 1
+            yield ("delay", sim.rng.randint(1, 400))  # issue cost of a step
+    si = tk % NK
+    if tk >= NK:
+        yield ("wait", sim.k_empty[si], tk // NK - 1)
+    sim.kflags[si] = (None, {}, True)
+    sim.k_full[si].arrive()
+
+
+def qv_producer(sim):
+    tv, qn = 0, [0, 0]
+    m = 0
+    while True:
+        slot = m % RING
+        yield ("wait", sim.item_full[slot], m // RING)
+        item = sim.ring[slot]
+        sim.item_empty[slot].arrive()
+        m += 1
+        if item is None:
+            return
+        for s in range(2):
+            if not tiles_of(item, s):
+                continue
+            if qn[s] >= 1:
+                yield ("wait", sim.q_empty[s], qn[s] - 1)
+            sim.tma(sim.q_full[s], f"Q{s}")
+            qn[s] += 1
+        for tile, fl in steps(item):
+            si = tv % NV
+            if tv >= NV:
+                yield ("wait", sim.v_empty[si], tv // NV - 1)
+            if tile is None:
+                sim.v_full[si].arrive()
+            else:
+                sim.v_content[si] = tile
+                sim.tma(sim.v_full[si], f"V{si}")
+            tv += 1
+            yield ("delay", sim.rng.randint(1, 400))  # issue cost of a step
+
+
+def mma_issuer(sim, s):
+    u, qcnt, pcnt = 0, 0, 0
+    pend = pfirst = plast = False
+    ptile = None
+    while True:
+        v = u - 1
+        if u >= 1 and not (sim.release_without_fill and not pend):
+            yield ("wait", sim.v_full[v % NV], v // NV)
+        if pend:
+            yield ("wait", sim.p_full[s], pcnt)
+        yield ("wait", sim.k_full[u % NK], u // NK)
+        tile, fl, end = sim.kflags[u % NK]
+        inn = (not end) and s in fl
+        if inn and fl[s][0]:
+            yield ("wait", sim.q_full[s], qcnt)
+        yield ("turn", 2 * u + s)
+        if pend:
+            if pfirst:
+                if sim.first_pv[s] > sim.epi_done[s]:
+                    raise ProtocolError(f"slot {s}: first PV of an item before the epilogue read O")
+                sim.first_pv[s] += 1
+            if sim.v_content[v % NV] != ptile:
+                raise ProtocolError(f"slot {s}: PV reads {sim.v_content[v % NV]}, wants {ptile}")
+            sim.mma(512, [f"V{v % NV}"])
+        if inn:
+            if sim.k_content[u % NK] != tile:
+                raise ProtocolError(f"slot {s}: QK reads {sim.k_content[u % NK]}, wants {tile}")
+            sim.consumed.append((s, tile))
+            sim.mma(512, [f"K{u % NK}", f"Q{s}"])
+        sim.pass_turn(2 * u + s + 1)
+        if pend:
+            if plast:
+                sim.commit(sim.o_full[s])
+            sim.commit(sim.v_empty[v % NV])
+            pend = False
+            pcnt += 1
+        elif u >= 1:
+            sim.v_empty[v % NV].arrive()
+        if end:
+            return
+        if inn:
+            sim.commit(sim.s_full[s])
+            if fl[s][1]:
+                sim.commit(sim.q_empty[s])
+            sim.commit(sim.k_empty[u % NK])
+            if fl[s][0]:
+                qcnt += 1
+            pend, pfirst, plast, ptile = True, fl[s][0], fl[s][1], tile
+        else:
+            sim.k_empty[u % NK].arrive()
+        u += 1
+        yield ("delay", sim.rng.randint(1, 50))
+
+
+def softmax(sim, s):
+    m, tcnt, icnt = 0, 0, 0
+    while True:
+        slot = m % RING
+        yield ("wait", sim.item_full[slot], m // RING)
+        item = sim.ring[slot]
+        sim.item_empty[slot].arrive()
+        m += 1
+        if item is None:
+            return
+        n = len(tiles_of(item, s))
+        if n == 0:
+            continue
+        for _ in range(n):
+            yield ("wait", sim.s_full[s], tcnt)
+            yield ("delay", sim.rng.randint(800, 3000))
+            sim.p_full[s].arrive()
+            tcnt += 1
+        yield ("wait", sim.o_full[s], icnt)
+        icnt += 1
+        yield ("delay", sim.rng.randint(100, 600))  # O read from tensor memory
+        sim.epi_done[s] += 1
+        yield ("delay", sim.rng.randint(100, 1500))  # normalise and store
+
+
+def _items(seed, n):
+    rng = random.Random(seed)
+    items = [random_item(rng) for _ in range(n)]
+    if seed % 3 == 0:  # long runs of items without tiles, as at the end of a schedule
+        items += [([], 0, [], 0)] * rng.randint(5, 20)
+    return items
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_protocol_random_schedules(seed):
+    items = _items(seed, 30)
+    sim = Sim(seed, items)
+    sim.run()
+    # every tile was consumed by exactly the slots that list it, in order
+    want = [(s, t) for it in items for t, fl in steps(it) for s in sorted(fl)]
+    assert sorted(sim.consumed, key=str) == sorted(want, key=str)
+
+
+def test_release_without_observed_fill_breaks_phases():
+    # Releasing a V stage that no slot reads without first observing its fill lets the
+    # releases of a run of no-op steps race ahead of the producer.
+    broken = 0
+    for seed in range(40):
+        items = [([], 0, [], 0)] * 12 + [([1, 2], 0, [1, 2, 3], 1)] + [([], 0, [], 0)] * 12
+        sim = Sim(seed, items, release_without_fill=True)
+        try:
+            sim.run()
+        except ProtocolError:
+            broken += 1
+    assert broken > 0
