@@ -48,6 +48,12 @@ WORKLOADS = {
     "long-104k-10pct": (24, 8, 104000, 128, lambda: inputs.patterns_density(inputs.SEED_BASE + 5, "10")),
     "long-104k-100pct": (24, 8, 104000, 128, lambda: inputs.patterns_density(inputs.SEED_BASE + 5, "100")),
 }
+# Decoding step (one new query per sequence at the last position of its cache):
+# name: (B, H_q, H_kv, S_cache, d, pattern builder)
+DECODE_WORKLOADS = {
+    "decode-llama3-8b-16k-b16": (16, 32, 8, 16384, 128,
+                                 lambda: inputs.patterns_band_random(inputs.SEED_BASE + 7, S=16384)),
+}
 SEEDS = {"llama3-8b-layer-64k": inputs.SEED_BASE + 4, "llama3.2-1b-layer-16k": inputs.SEED_BASE + 3,
          "llama3-8b-layer-16k": inputs.SEED_BASE + 6}
 CAPTURE_MAPS = 32  # one layer's heads
@@ -398,13 +404,99 @@ def run_gpu(args, rank, world, local, dist):
     return line
 
 
+def run_decode(args):
+    """Time sparse_attn_decode on one GPU: tokens/s (B new tokens per step) and the
+    achieved HBM bandwidth of the gathered key/value rows against the measured copy peak."""
+    import torch
+
+    import structured_sparse_attention_b200 as ssa
+    B, Hq, Hkv, S, d, builder = DECODE_WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    diags, verts = builder()
+    dp, do = inputs.to_csr(diags)
+    vp, vo = inputs.to_csr(verts)
+    lists = [torch.from_numpy(a.astype(np.int32)).to(dev) for a in (dp, do, vp, vo)]
+    plan = ssa.extend(*lists, S)
+    base = inputs.SEED_BASE + 8
+    kc = torch.from_numpy(np.stack([inputs.normal_bf16(base + 2 * b, Hkv, S, d) for b in range(B)]).view(np.int16))
+    vc = torch.from_numpy(np.stack([inputs.normal_bf16(base + 2 * b + 1, Hkv, S, d) for b in range(B)]).view(np.int16))
+    kc, vc = kc.to(dev).view(torch.bfloat16), vc.to(dev).view(torch.bfloat16)
+    h_q = torch.from_numpy(inputs.normal_bf16(base - 1, B, Hq, d).view(np.int16)).view(torch.bfloat16).pin_memory()
+    q = h_q.to(dev)
+    pos_h = np.full(B, S - 1, np.int32)
+    pos = torch.from_numpy(pos_h).to(dev)
+    O = torch.empty_like(q)
+    LSE = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(ssa.load().sparse_attn_decode_ws_bytes(B, Hq, d), 16), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # larger than the 126 MB L2
+
+    def call():
+        ssa.attn_decode(q, kc, vc, pos, plan, out=O, lse=LSE, ws=ws, status=status, check=False)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0")
+    sampler.start()
+    time.sleep(0.3)
+    for e0, e1 in ev:
+        flush.fill_(1)  # evict the previous step's rows from L2 (not timed)
+        e0.record()
+        call()
+        e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())}")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    # end to end: the step's queries in from pinned host memory, O and LSE back
+    h_O = torch.empty(O.shape, dtype=torch.bfloat16).pin_memory()
+    h_L = torch.empty(LSE.shape, dtype=torch.float32).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        q.copy_(h_q, non_blocking=True)
+        call()
+        h_O.copy_(O, non_blocking=True)
+        h_L.copy_(LSE, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1) / args.steps
+    # retained keys of row S-1 per head (integer counting from the lists)
+    keys = 0
+    for Dh, Ch in zip(diags, verts):
+        Dh, Ch = np.asarray(Dh, np.int64), np.asarray(Ch, np.int64)
+        band = set((S - 1 - Dh[Dh <= S - 1]).tolist())
+        keys += len(band | set(Ch[Ch <= S - 1].tolist()))
+    algo_bytes = B * keys * d * 2 * 2 + 2 * B * Hq * d * 2 + B * Hq * 4
+    hbm_gbs, _, _, peak_kind = load_peaks()
+    achieved = algo_bytes / (ms / 1e3) / 1e9
+    line = {"metric": "sparse-attn decode tokens/s & achieved HBM GB/s vs roofline", "value": B / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "B": B, "H_q": Hq, "H_kv": Hkv, "S_cache": S, "d": d,
+                       "keys_per_sequence": keys, "l2": "flushed between timed steps (256 MB write)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": achieved / hbm_gbs, "traffic": None, "kernel": "sparse_attn_decode (partial + combine)",
+                         "peak_source": f"{peak_kind} (copy)", "algorithmic": {"bytes": algo_bytes}},
+            "clocks": clocks,
+            "e2e": {"value": B / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h_q.numel() * 2),
+                    "d2h_bytes_per_step": int(h_O.numel() * 2 + h_L.numel() * 4), "ms_per_step": e_ms},
+            "gpu_launches": 2 * args.steps, "cpu_baseline": None}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ssa", choices=["ssa", "reference"])
-    ap.add_argument("--workload", default="llama3-8b-layer-64k", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="llama3-8b-layer-64k", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle attention work")
@@ -414,6 +506,11 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if args.workload in DECODE_WORKLOADS:
+        if args.impl != "ssa" or args.gpus != 1:
+            ap.error("decode workloads run the library on one GPU")
+        run_decode(args)
+        return
     rank, world, local, dist = dist_setup(args.gpus)
     if args.impl == "reference":
         if rank == 0:

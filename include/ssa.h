@@ -243,6 +243,45 @@ SSA_API int sparse_attn_fwd(const void *Q, const void *K, const void *V, int H_q
                     void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
 
 /* ------------------------------------------------------------------------------ */
+/* Decoding step                                                                   */
+/* ------------------------------------------------------------------------------ */
+
+/* Workspace bytes of sparse_attn_decode: the per-split partial results
+ * ((2 + d) floats per split, 1 to 16 splits per sequence and head). */
+SSA_API size_t sparse_attn_decode_ws_bytes(int B, int H_q, int d);
+
+/*
+ * sparse_attn_decode -- one decoding step over the same extended mask: the new query
+ * of sequence b sits at position pos[b] and attends to row pos[b] of the mask ("What
+ * carries the argument": the kept patterns are pasted over the whole S x S square;
+ * Referee Report summary: the mask is applied to the scaled logits before the
+ * softmax), i.e. for head h with KV head g:
+ *   J = {pos - r : r an extended diagonal, r <= pos} U {c an extended column, c <= pos}
+ *   O[b][h]   = sum_{j in J} softmax_j(scale * q . K[b][g][j]) V[b][g][j]
+ *   LSE[b][h] = log sum_{j in J} exp(scale * q . K[b][g][j])      (natural log)
+ * which is row pos[b] of sparse_attn_fwd over the same cache.  An empty J gives O = 0
+ * and LSE = -inf.  bf16 inputs, fp32 accumulation, bf16 O.  Bound by the HBM traffic
+ * of the gathered key and value rows.
+ *
+ *   Q, O         device bf16 [B][H_q][d], contiguous
+ *   K, V         device bf16 [B][H_kv][S_cache][d]: the key/value cache of each sequence
+ *   B, H_q, H_kv >= 1 (B, H_q <= 65535); H_q % H_kv == 0 when kv_map is NULL
+ *   S_cache      must equal plan->S;  d in {64, 128} (else SSA_ERR_UNSUPPORTED)
+ *   pos          device int32 [B], 0 <= pos[b] < S_cache; a position outside that range
+ *                (or a kv_map entry outside [0, H_kv)) sets SSA_ERR_INVALID in
+ *                dev_status and gives that sequence O = 0, LSE = -inf
+ *   plan         from sparse_pattern_extend with S = S_cache and n_heads = H_q (only its
+ *                extended lists are read)
+ *   LSE          device float32 [B][H_q]
+ *   ws           device workspace of at least sparse_attn_decode_ws_bytes(B, H_q, d);
+ *                Q, K, V, O and ws 16-byte aligned
+ */
+SSA_API int sparse_attn_decode(const void *Q, const void *K, const void *V, int B, int H_q, int H_kv,
+                               int S_cache, int d, const int32_t *pos, const ssa_plan *plan,
+                               const int32_t *kv_map, float scale, void *O, float *LSE, void *ws,
+                               size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------------ */
 /* Diagnostics                                                                     */
 /* ------------------------------------------------------------------------------ */
 

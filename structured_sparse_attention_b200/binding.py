@@ -27,6 +27,7 @@ BLOCK = 128
 EXPORTS = ("sparse_pattern_capture_ws_bytes", "sparse_pattern_capture", "sparse_pattern_capture_noalloc",
            "sparse_pattern_extend_ws_bytes", "sparse_pattern_extend",
            "sparse_attn_fwd_ws_bytes", "sparse_attn_fwd",
+           "sparse_attn_decode_ws_bytes", "sparse_attn_decode",
            "ssa_last_error", "ssa_version", "ssa_set_wait_limit_ns")
 
 
@@ -76,6 +77,11 @@ def load():
         lib.sparse_attn_fwd.argtypes = [V, V, V, I, I, I, I, C.POINTER(PlanStruct), V, C.c_float,
                                         V, V, V, SZ, V, V]
         lib.sparse_attn_fwd.restype = I
+        lib.sparse_attn_decode_ws_bytes.argtypes = [I, I, I]
+        lib.sparse_attn_decode_ws_bytes.restype = SZ
+        lib.sparse_attn_decode.argtypes = [V, V, V, I, I, I, I, I, V, C.POINTER(PlanStruct), V, C.c_float,
+                                           V, V, V, SZ, V, V]
+        lib.sparse_attn_decode.restype = I
         lib.ssa_last_error.argtypes = []
         lib.ssa_last_error.restype = C.c_char_p
         lib.ssa_version.restype = I
@@ -288,6 +294,48 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan, *, k
     _check(lib.sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, S, d, C.byref(plan.struct),
                                _ptr(kv_map), float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                _ptr(status), cs))
+    if check:
+        _check_status(status, s)
+    return out, lse
+
+
+# ------------------------------------------------------------------------------------
+# Decoding step
+# ------------------------------------------------------------------------------------
+
+def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, pos: torch.Tensor,
+                plan: Plan, *, kv_map=None, scale: float | None = None, out=None, lse=None, ws=None,
+                stream=None, check: bool = True, status=None):
+    """sparse_attn_decode.  q [B,H_q,d], caches [B,H_kv,S,d] bf16, pos [B] int32 (CUDA).
+    Returns (O [B,H_q,d] bf16, LSE [B,H_q] fp32)."""
+    lib = load()
+    for t, nm in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need_cuda(t, nm, torch.bfloat16)
+    _need_cuda(pos, "pos", torch.int32)
+    B, Hq, d = q.shape
+    Hkv, S = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (B, Hkv, S, d) or v_cache.shape != k_cache.shape:
+        raise SSAError(-1, "k_cache and v_cache must be [B, H_kv, S, d] matching q")
+    if pos.numel() != B:
+        raise SSAError(-1, "pos must hold one position per sequence")
+    dev = q.device
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    need = lib.sparse_attn_decode_ws_bytes(B, Hq, d)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    if kv_map is not None:
+        _need_cuda(kv_map, "kv_map", torch.int32)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    cs, s = _stream(stream)
+    _check(lib.sparse_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), B, Hq, Hkv, S, d, _ptr(pos),
+                                  C.byref(plan.struct), _ptr(kv_map), float(scale), _ptr(out), _ptr(lse),
+                                  _ptr(ws), ws.numel(), _ptr(status), cs))
     if check:
         _check_status(status, s)
     return out, lse
