@@ -357,6 +357,32 @@ def run_gpu(args, rank, world, local, dist):
         e2e = {"value": world * S / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms}
 
+    # ---------------- dense reference point (context, not the target) ----------------
+    dense = None
+    if args.dense_ref:
+        import torch.nn.functional as F
+        qd = q.unsqueeze(0)
+        kd, vd = k.unsqueeze(0), v.unsqueeze(0)
+        scale = d ** -0.5
+
+        def sdpa():
+            return F.scaled_dot_product_attention(qd, kd, vd, is_causal=True, scale=scale, enable_gqa=True)
+
+        for _ in range(3):
+            sdpa()
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        d0.record()
+        for _ in range(reps):
+            sdpa()
+        d1.record()
+        torch.cuda.synchronize()
+        dms = d0.elapsed_time(d1) / reps
+        dense = {"what": "torch scaled_dot_product_attention, causal, bf16, same Q/K/V (GQA), all causal pairs",
+                 "ms": dms, "tokens_per_s": S / (dms / 1e3),
+                 "effective_tflops_of_causal_pairs": 4.0 * d * Hq * S * (S + 1) / 2 / (dms / 1e3) / 1e12}
+
     # ---------------- metrics ----------------
     nnz = nnz_per_head(diags, verts, S)
     flops = 4.0 * d * float(nnz.sum())
@@ -400,6 +426,7 @@ def run_gpu(args, rank, world, local, dist):
         "clocks": clocks,
         "e2e": e2e,
         "gpu_launches": args.steps * sum(LAUNCHES.values()),
+        "dense_reference": dense,
     }
     return line
 
@@ -500,6 +527,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle attention work")
+    ap.add_argument("--dense-ref", action="store_true",
+                    help="also time torch's causal SDPA on the same inputs (dense reference point)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of the same kernel")
     args = ap.parse_args()

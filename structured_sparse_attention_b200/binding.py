@@ -225,6 +225,12 @@ def extend(diag_ptr, diag_offsets, vert_ptr, vert_cols, S: int, *, stream=None, 
     if vert_ptr.numel() != H + 1:
         raise SSAError(-1, "diag_ptr and vert_ptr must describe the same number of heads")
     dev = diag_ptr.device
+    # an empty value list is a zero-size tensor without storage; the C ABI wants a
+    # valid pointer even when no entry is read
+    if diag_offsets.numel() == 0:
+        diag_offsets = torch.zeros(1, dtype=torch.int32, device=dev)
+    if vert_cols.numel() == 0:
+        vert_cols = torch.zeros(1, dtype=torch.int32, device=dev)
     need = lib.sparse_pattern_extend_ws_bytes(H, S)
     if ws is None or ws.numel() < need:
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
@@ -251,6 +257,10 @@ def refill(plan: Plan, diag_ptr, diag_offsets, vert_ptr, vert_cols, *, stream=No
     """Re-run only the fill pass of sparse_pattern_extend into an existing plan (same sizes)."""
     lib = load()
     H, S = plan.n_heads, plan.S
+    if diag_offsets.numel() == 0:
+        diag_offsets = torch.zeros(1, dtype=torch.int32, device=diag_ptr.device)
+    if vert_cols.numel() == 0:
+        vert_cols = torch.zeros(1, dtype=torch.int32, device=diag_ptr.device)
     cs, _ = _stream(stream)
     _check(lib.sparse_pattern_extend(H, _ptr(diag_ptr), _ptr(diag_offsets), _ptr(vert_ptr),
                                      _ptr(vert_cols), S, C.byref(plan.sizes), C.byref(plan.struct),
