@@ -57,6 +57,15 @@ DECODE_WORKLOADS = {
 SEEDS = {"llama3-8b-layer-64k": inputs.SEED_BASE + 4, "llama3.2-1b-layer-16k": inputs.SEED_BASE + 3,
          "llama3-8b-layer-16k": inputs.SEED_BASE + 6}
 CAPTURE_MAPS = 32  # one layer's heads
+MUFU_EX2_PER_CLK_SM = 16  # B200: ex2.approx results per clock per SM (microbenchmark: 15.99)
+
+
+def sm_max_mhz():
+    """clocks.max.sm of the machine's B200s (MEASURED_PEAKS.json, else the nominal 1965 MHz)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return float(json.load(open(p)).get("sm_max_mhz", 1965.0))
+    return 1965.0
 CAPTURE_L = 512
 
 
@@ -393,8 +402,17 @@ def run_gpu(args, rank, world, local, dist):
     algo_bytes = (2 * Hq * S * d * 2) + (2 * Hkv * S * d * 2) + Hq * S * 4
     t_tensor = flops / (tf_burst * 1e12)
     t_hbm = algo_bytes / (hbm_gbs * 1e9)
-    bound = "tensor" if t_tensor >= t_hbm else "hbm"
-    if bound == "tensor":
+    # one ex2 per retained pair on the MUFU: 16 per clock per SM (measured 15.99) at the
+    # maximum SM clock; at d = 64 this, not the tensor pipe, bounds the kernel
+    n_exp = float(nnz.sum())  # nnz holds one entry per Q head
+    mufu_peak = MUFU_EX2_PER_CLK_SM * props.multi_processor_count * sm_max_mhz() * 1e6
+    t_mufu = n_exp / mufu_peak
+    bound = max((t_tensor, "tensor"), (t_hbm, "hbm"), (t_mufu, "alu"))[1]
+    if bound == "alu":
+        achieved = n_exp / (attn_ms / 1e3) / 1e9
+        roof = {"bound": "alu", "achieved": achieved, "peak": mufu_peak / 1e9, "unit": "Gex2/s",
+                "frac": achieved / (mufu_peak / 1e9), "pipe": "MUFU ex2 (one per retained pair)"}
+    elif bound == "tensor":
         achieved = flops / (attn_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
                 "frac": achieved / tf_burst}
@@ -408,7 +426,9 @@ def run_gpu(args, rank, world, local, dist):
                  "kernel": "sparse_attn_fwd (stripe gather + attention kernel)",
                  "peak_source": f"{peak_kind} ({'burst' if bound == 'tensor' else 'copy'})",
                  "algorithmic": {"flops": flops, "bytes": algo_bytes},
-                 "roofline_ms": max(t_tensor, t_hbm) * 1e3, "frac_of_roofline_time": max(t_tensor, t_hbm) * 1e3 / attn_ms})
+                 "roofline_ms": max(t_tensor, t_hbm, t_mufu) * 1e3,
+                 "frac_of_roofline_time": max(t_tensor, t_hbm, t_mufu) * 1e3 / attn_ms,
+                 "bounds_ms": {"tensor": t_tensor * 1e3, "hbm": t_hbm * 1e3, "mufu": t_mufu * 1e3}})
 
     line = {
         "metric": METRIC, "value": world * S / (ms_step / 1e3), "unit": UNIT, "n_gpus": world,
