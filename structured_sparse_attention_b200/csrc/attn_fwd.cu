@@ -21,8 +21,8 @@
 //                    TMA producer of the K tiles of the merged sequence; each K stage
 //                    carries a flag word: which slot uses it, first/last tile of a
 //                    slot within the item, end of work
-//     warp 10        lane 0: TMA producer of the two Q tiles of each item, then of the
-//                    V tiles of the same sequence
+//     warp 10        lane 0: TMA producer of the V tiles of the same sequence, and of
+//                    each slot's Q tile at the slot's first step of the item
 //                    (each blocking role has a warp of its own: single-lane loops of one
 //                    warp would serialise on each other's waits)
 //     warps 9, 11    MMA issuers, one per slot (warp 9 allocates tensor memory).  For
@@ -38,7 +38,11 @@
 //                    tcgen05.ld S (128 columns), element mask from the plan (FULL
 //                    tiles skip it), online max/sum in fp32 (log2 domain, packed f32x2
 //                    arithmetic), P as bf16 into TMEM, lazy O rescale (only when the
-//                    max grows by > 2^8); epilogue O / l -> bf16 and LSE.
+//                    max grows by > 2^8); epilogue O / l -> bf16 and LSE.  A slot's
+//                    epilogue runs after it has handed over the P of its first tile of
+//                    the next item: the tensor pipe gets that P without waiting for the
+//                    epilogue, and the first PV of the next item (which overwrites O_s)
+//                    waits on o_empty until the epilogue has read O_s.
 // Tensor memory (512 columns): S0 0..127, S1 128..255, O0 256.., O1 256+d...
 //
 // Every barrier is waited on with a counter of its own completions, and every wait
@@ -135,7 +139,7 @@ struct Shared {
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[kMaxStages], k_empty[kMaxStages];
     uint64_t v_full[kMaxStages], v_empty[kMaxStages];
-    uint64_t s_full[2], p_full[2], o_full[2];
+    uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
     uint64_t mma_drain, softmax_done;
     ItemDesc items[kRing];
     uint32_t kflags[kMaxStages];
@@ -380,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sh->s_full[s], 1);
             mbar_init(&sh->p_full[s], kSlotThreads);
             mbar_init(&sh->o_full[s], 1);
+            mbar_init(&sh->o_empty[s], kSlotThreads);
         }
         for (int st = 0; st < C::NK; ++st) {
             mbar_init(&sh->k_full[st], 1);
@@ -477,9 +482,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (warp == kWarpV) {
         if (lane == 0) {
             // ------------------------- Q and V producer -------------------------
-            // The two Q tiles of an item, then its V tiles.  A Q tile waits for the
-            // last QK^T of its slot in the previous item; the V tiles of the previous
-            // item are all issued by then, so that wait never holds back a PV.
+            // The V tiles of the merged sequence, and each slot's Q tile at the slot's
+            // first step of the item.  A Q tile waits for the last QK^T of its slot in
+            // the previous item; loading it only at the slot's first step keeps the V
+            // tiles of the steps before it from waiting on that QK^T.
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmV);
             prefetch_tmap(&tmVC);
@@ -496,26 +502,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&sh->item_empty[slot]);
                 ++m;
                 if (d.end) break;
-#pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    if (!ok || d.nb[s] + d.ns[s] == 0) continue;
-                    if (qn[s] >= 1 && !mbar_wait(&sh->q_empty[s], (qn[s] - 1) & 1, lim, abort)) {
-                        ok = false;
-                        continue;
-                    }
-                    uint8_t *sQ = smem + C::OFF_Q + s * C::TILE_BYTES;
-                    mbar_arrive_expect_tx(&sh->q_full[s], C::TILE_BYTES);
-                    for (int b = 0; b < C::BOXES; ++b)
-                        tma_load_3d(sQ + b * kBoxBytes, &tmQ, &sh->q_full[s], 64 * b, d.qb[s] * kBM, d.h);
-                    ++qn[s];
-                }
-                if (!ok) break;
                 Steps st;
                 steps_init(st, p, d);
                 bool band;
                 int row0;
                 uint32_t fl;
                 while (steps_next(st, band, row0, fl)) {
+#pragma unroll
+                    for (int s = 0; s < 2; ++s) {
+                        if (!ok || !(fl & f_first(s))) continue;
+                        if (qn[s] >= 1 && !mbar_wait(&sh->q_empty[s], (qn[s] - 1) & 1, lim, abort)) {
+                            ok = false;
+                            continue;
+                        }
+                        uint8_t *sQ = smem + C::OFF_Q + s * C::TILE_BYTES;
+                        mbar_arrive_expect_tx(&sh->q_full[s], C::TILE_BYTES);
+                        for (int b = 0; b < C::BOXES; ++b)
+                            tma_load_3d(sQ + b * kBoxBytes, &tmQ, &sh->q_full[s], 64 * b, d.qb[s] * kBM, d.h);
+                        ++qn[s];
+                    }
+                    if (!ok) break;
                     const int si = tv % C::NV;
                     if (tv >= C::NV && !mbar_wait(&sh->v_empty[si], ((tv / C::NV) - 1) & 1, lim, abort)) {
                         ok = false;
@@ -569,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tS = tmem + 128 * s, tO = tmem + C::COL_O + D * s;
             bool ok = true;
             int u = 0;  // merged step (K and V ring index)
-            int qcnt = 0, pcnt = 0;
+            int qcnt = 0, pcnt = 0, ocnt = 0;  // ocnt: first PVs of items issued
             bool pend = false, pfirst = false, plast = false;
             // The issuer polls (mbar_wait_poll): mbarrier.try_wait in a thread with MMAs
             // in flight costs about their drain time even when the phase is complete.
@@ -596,6 +602,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int v = u - 1;
                 if (u >= 1 && !wait(&sh->v_full[v % C::NV], (v / C::NV) & 1)) break;
                 if (pend && !wait(&sh->p_full[s], pcnt & 1)) break;
+                // the first PV of an item overwrites O_s: the previous item's epilogue
+                // must have read it
+                if (pend && pfirst && ocnt >= 1 && !wait(&sh->o_empty[s], (ocnt - 1) & 1)) break;
                 if (!wait(&sh->k_full[u % C::NK], (u / C::NK) & 1)) break;
                 const uint32_t f = sh->kflags[u % C::NK];
                 const bool end = (f & kStepEnd) != 0;
@@ -633,6 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (pend) {
                     if (plast) umma_commit(&sh->o_full[s]);  // O_s of the item complete
                     umma_commit(&sh->v_empty[v % C::NV]);    // completes once the PV has read V
+                    if (pfirst) ++ocnt;
                     pend = false;
                     ++pcnt;
                 } else if (u >= 1) {
@@ -686,6 +696,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t kNegInf = 0xff800000u;
         bool ok = true;
         int m = 0, tcnt = 0, icnt = 0;
+        // The epilogue of the slot's last item with tiles, owed until the P of the first
+        // tile of the slot's next such item (or the end of work): row e_i of head e_h,
+        // with its running max and sum.
+        bool owed = false;
+        int e_h = 0, e_i = 0;
+        float e_m = 0.0f, e_l = 0.0f;
+        auto epilogue = [&]() -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(&sh->o_full[s], icnt & 1, lim, abort))) return false;
+            ++icnt;
+            tc_fence_after();
+            uint32_t ro[D];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + 32 * c, ro + 32 * c);
+            tmem_wait_ld();
+            // O_s is read: the next item's first PV may overwrite it
+            tc_fence_before();
+            mbar_arrive(&sh->o_empty[s]);
+            // a row whose max stayed -inf has no retained key: O = 0, LSE = -inf
+            const bool empty = !(e_m > -INFINITY) || !(e_l > 0.0f);
+            const float inv = empty ? 0.0f : 1.0f / e_l;
+            if (e_i < p.S) {
+                const size_t row = static_cast<size_t>(e_h) * p.S + e_i;
+                uint4 *orow = reinterpret_cast<uint4 *>(p.O + row * D);
+                // the row as bf16, 16 columns (32 bytes) per store when O allows it: half the
+                // store instructions of 16-byte stores for the same bytes
+                uint32_t w[D / 2];
+#pragma unroll
+                for (int q = 0; q < D / 2; ++q) {
+                    const __nv_bfloat162 v2 =
+                        __floats2bfloat162_rn(__uint_as_float(ro[2 * q]) * inv, __uint_as_float(ro[2 * q + 1]) * inv);
+                    w[q] = *reinterpret_cast<const uint32_t *>(&v2);
+                }
+                if (p.o_align32) {
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) st_global_v8(orow + 2 * k, w + 8 * k);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < D / 8; ++k) orow[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                }
+                p.LSE[row] =
+                    empty ? -INFINITY : (e_m + log2f(e_l)) * 0.69314718055994531f;
+            }
+            return true;
+        };
         while (true) {
             const int slot = m % kRing;
             if (!__all_sync(0xffffffffu, mbar_wait(&sh->item_full[slot], (m / kRing) & 1, lim, abort))) {
@@ -706,9 +760,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n = nb + ns;
             const int i = qb * kBM + il;
             const bool row_ok = i < p.S;
-            uint4 *orow = reinterpret_cast<uint4 *>(p.O + (static_cast<size_t>(d.h) * p.S + (row_ok ? i : 0)) * D);
             if (n == 0) {  // no retained key in this block: O = 0, LSE = -inf
                 if (row_ok) {
+                    uint4 *orow = reinterpret_cast<uint4 *>(p.O + (static_cast<size_t>(d.h) * p.S + i) * D);
 #pragma unroll
                     for (int k = 0; k < D / 8; ++k) orow[k] = make_uint4(0, 0, 0, 0);
                     p.LSE[static_cast<size_t>(d.h) * p.S + i] = -INFINITY;
@@ -871,45 +925,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&sh->p_full[s]);
                 ++tcnt;
+                // the previous item's epilogue, now that the tensor pipe has this P
+                if (j == 0 && owed) {
+                    if (!epilogue()) {
+                        ok = false;
+                        break;
+                    }
+                    owed = false;
+                }
             }
             if (!ok) break;
-            // ---- epilogue: O / l, LSE ----
-            if (!__all_sync(0xffffffffu, mbar_wait(&sh->o_full[s], icnt & 1, lim, abort))) {
-                ok = false;
-                break;
-            }
-            ++icnt;
-            tc_fence_after();
-            uint32_t ro[D];
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + 32 * c, ro + 32 * c);
-            tmem_wait_ld();
-            // the next item's first PV may overwrite O_s once this slot's next P is handed
-            // over, which this thread does only after the load above has completed
-            // a row whose max stayed -inf has no retained key: O = 0, LSE = -inf
-            const bool empty = !(m_run > -INFINITY) || !(l_run > 0.0f);
-            const float inv = empty ? 0.0f : 1.0f / l_run;
-            if (row_ok) {
-                // the row as bf16, 16 columns (32 bytes) per store when O allows it: half the
-                // store instructions of 16-byte stores for the same bytes
-                uint32_t w[D / 2];
-#pragma unroll
-                for (int q = 0; q < D / 2; ++q) {
-                    const __nv_bfloat162 v2 =
-                        __floats2bfloat162_rn(__uint_as_float(ro[2 * q]) * inv, __uint_as_float(ro[2 * q + 1]) * inv);
-                    w[q] = *reinterpret_cast<const uint32_t *>(&v2);
-                }
-                if (p.o_align32) {
-#pragma unroll
-                    for (int k = 0; k < D / 16; ++k) st_global_v8(orow + 2 * k, w + 8 * k);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < D / 8; ++k) orow[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-                }
-                p.LSE[static_cast<size_t>(d.h) * p.S + i] =
-                    empty ? -INFINITY : (m_run + log2f(l_run)) * 0.69314718055994531f;
-            }
+            owed = true;
+            e_h = d.h;
+            e_i = i;
+            e_m = m_run;
+            e_l = l_run;
         }
+        if (ok && owed && !epilogue()) ok = false;
         if (!ok) {
             report(p.status, SSA_ERR_TIMEOUT);
             *abort = 1;

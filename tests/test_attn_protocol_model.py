@@ -15,7 +15,9 @@ Checked in every run:
   * a K or V stage is refilled only after every MMA that reads its previous content
     has completed, and a Q buffer only after the last QK^T that reads it;
   * the first PV of an item (which overwrites O) is issued only after the epilogue of
-    the slot's previous item has read O;
+    the slot's previous item has read O.  That epilogue runs after the softmax of the
+    slot's first tile of the next item (it is deferred so the tensor pipe gets the next
+    item's first P sooner); the issuer waits for it on o_empty;
   * every tile the producers stage is consumed by exactly the slots that list it.
 The model also shows that releasing a V stage without first observing its fill (the
 rule the issuers follow) breaks the phase invariant for runs of tile-less items.
@@ -72,6 +74,7 @@ class Sim:
         self.s_full = [B(f"s_full{s}", 1) for s in range(2)]
         self.p_full = [B(f"p_full{s}", 1) for s in range(2)]
         self.o_full = [B(f"o_full{s}", 1) for s in range(2)]
+        self.o_empty = [B(f"o_empty{s}", 1) for s in range(2)]
         self.ring = [None] * RING
         self.kflags = [None] * NK
         self.turn = 0
@@ -271,14 +274,16 @@ def qv_producer(sim):
         m += 1
         if item is None:
             return
-        for s in range(2):
-            if not tiles_of(item, s):
-                continue
-            if qn[s] >= 1:
-                yield ("wait", sim.q_empty[s], qn[s] - 1)
-            sim.tma(sim.q_full[s], f"Q{s}")
-            qn[s] += 1
         for tile, fl in steps(item):
+            # the Q tile of a slot is loaded at the slot's first step of the item, so
+            # the V tiles of steps before it never wait on the slot's previous item
+            for s in sorted(fl):
+                if not fl[s][0]:
+                    continue
+                if qn[s] >= 1:
+                    yield ("wait", sim.q_empty[s], qn[s] - 1)
+                sim.tma(sim.q_full[s], f"Q{s}")
+                qn[s] += 1
             si = tv % NV
             if tv >= NV:
                 yield ("wait", sim.v_empty[si], tv // NV - 1)
@@ -292,7 +297,7 @@ def qv_producer(sim):
 
 
 def mma_issuer(sim, s):
-    u, qcnt, pcnt = 0, 0, 0
+    u, qcnt, pcnt, ocnt = 0, 0, 0, 0
     pend = pfirst = plast = False
     ptile = None
     while True:
@@ -301,6 +306,8 @@ def mma_issuer(sim, s):
             yield ("wait", sim.v_full[v % NV], v // NV)
         if pend:
             yield ("wait", sim.p_full[s], pcnt)
+            if pfirst and ocnt >= 1:
+                yield ("wait", sim.o_empty[s], ocnt - 1)
         yield ("wait", sim.k_full[u % NK], u // NK)
         tile, fl, end = sim.kflags[u % NK]
         inn = (not end) and s in fl
@@ -312,6 +319,7 @@ def mma_issuer(sim, s):
                 if sim.first_pv[s] > sim.epi_done[s]:
                     raise ProtocolError(f"slot {s}: first PV of an item before the epilogue read O")
                 sim.first_pv[s] += 1
+                ocnt += 1
             if sim.v_content[v % NV] != ptile:
                 raise ProtocolError(f"slot {s}: PV reads {sim.v_content[v % NV]}, wants {ptile}")
             sim.mma(512, [f"V{v % NV}"])
@@ -347,6 +355,17 @@ def mma_issuer(sim, s):
 
 def softmax(sim, s):
     m, tcnt, icnt = 0, 0, 0
+    owed = False  # the epilogue of the slot's last item with tiles is still to do
+
+    def epilogue():
+        nonlocal icnt
+        yield ("wait", sim.o_full[s], icnt)
+        icnt += 1
+        yield ("delay", sim.rng.randint(100, 600))  # O read from tensor memory
+        sim.epi_done[s] += 1
+        sim.o_empty[s].arrive()
+        yield ("delay", sim.rng.randint(100, 1500))  # normalise and store
+
     while True:
         slot = m % RING
         yield ("wait", sim.item_full[slot], m // RING)
@@ -354,20 +373,21 @@ def softmax(sim, s):
         sim.item_empty[slot].arrive()
         m += 1
         if item is None:
-            return
+            break
         n = len(tiles_of(item, s))
         if n == 0:
             continue
-        for _ in range(n):
+        for j in range(n):
             yield ("wait", sim.s_full[s], tcnt)
             yield ("delay", sim.rng.randint(800, 3000))
             sim.p_full[s].arrive()
             tcnt += 1
-        yield ("wait", sim.o_full[s], icnt)
-        icnt += 1
-        yield ("delay", sim.rng.randint(100, 600))  # O read from tensor memory
-        sim.epi_done[s] += 1
-        yield ("delay", sim.rng.randint(100, 1500))  # normalise and store
+            if j == 0 and owed:
+                yield from epilogue()
+                owed = False
+        owed = True
+    if owed:
+        yield from epilogue()
 
 
 def _items(seed, n):
