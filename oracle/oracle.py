@@ -66,7 +66,8 @@ def _setup(L):
     L.ora_attn_dense.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int, P, P, P, P, P,
                                  C.c_double, P, P]
     L.ora_nnz.argtypes = [C.c_int, P, P, P, P, C.c_int, P]
-    for name in ("ora_true_mask", "ora_gamma", "ora_select", "ora_capture", "ora_extend",
+    L.ora_attn_maps.argtypes = [P, P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_double, P]
+    for name in ("ora_attn_maps", "ora_true_mask", "ora_gamma", "ora_select", "ora_capture", "ora_extend",
                  "ora_attn_rows", "ora_attn_dense", "ora_nnz"):
         getattr(L, name).restype = C.c_int
 
@@ -88,6 +89,18 @@ def _check(rc, what):
 # ------------------------------------------------------------------------------------
 # Stage one
 # ------------------------------------------------------------------------------------
+
+def attn_maps(q, k, scale):
+    """Averaged causal attention maps in fp64.  q, k: bf16 bits uint16 [n_maps, B, L, d]
+    -> [n_maps, L, L] (zeros above the diagonal)."""
+    q, k = _c(q, np.uint16), _c(k, np.uint16)
+    n, B, L, d = q.shape
+    if k.shape != q.shape:
+        raise ValueError("q and k must have the same shape")
+    out = np.zeros((n, L, L), np.float64)
+    _check(lib().ora_attn_maps(_p(q), _p(k), n, B, L, d, float(scale), _p(out)), "attn_maps")
+    return out
+
 
 def true_mask(amap, lam=0.5, eps=1e-8, tau=0.3):
     """Binary true mask uint8 [L, L] of one averaged map (row min-max of Box-Cox, t >= tau)."""

@@ -670,3 +670,48 @@ int ora_nnz(int n_heads, const int32_t *ext_diag_ptr, const int32_t *ext_diag_of
     }
     return ORA_OK;
 }
+
+/* Averaged attention maps, the input of stage one ("What carries the argument":
+ * attention maps averaged over a calibration corpus at capture length L).  For map m,
+ * sample b and row i: the causal logits s_j = scale * <q_i, k_j> (j <= i), their
+ * softmax p_j = exp(s_j - max) / sum_j' exp(s_j' - max), and
+ *   maps[m][i][j] = (1/B) sum_b p_j  (j <= i),   0 above the diagonal.
+ * Q, K bf16 bits [n_maps][B][L][d]; maps [n_maps][L][L] in fp64. */
+int ora_attn_maps(const uint16_t *Q, const uint16_t *K, int n_maps, int B, int L, int d, double scale,
+                  double *maps) {
+    if (!Q || !K || !maps || n_maps <= 0 || B <= 0 || L <= 0 || d <= 0) return ORA_ERR_INVALID;
+    int err = ORA_OK;
+    memset(maps, 0, sizeof(double) * (size_t)n_maps * L * L);
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)L);
+        if (!s) err = ORA_ERR_NOMEM;
+#pragma omp for schedule(dynamic, 1)
+        for (int m = 0; m < n_maps; ++m) {
+            if (!s) continue;
+            for (int b = 0; b < B; ++b) {
+                const uint16_t *q = Q + ((size_t)m * B + b) * L * d;
+                const uint16_t *k = K + ((size_t)m * B + b) * L * d;
+                for (int i = 0; i < L; ++i) {
+                    double mx = -INFINITY;
+                    for (int j = 0; j <= i; ++j) {
+                        double dot = 0.0;
+                        for (int c = 0; c < d; ++c)
+                            dot += bf16_bits_to_double(q[(size_t)i * d + c]) * bf16_bits_to_double(k[(size_t)j * d + c]);
+                        s[j] = scale * dot;
+                        if (s[j] > mx) mx = s[j];
+                    }
+                    double sum = 0.0;
+                    for (int j = 0; j <= i; ++j) {
+                        s[j] = exp(s[j] - mx);
+                        sum += s[j];
+                    }
+                    double *row = maps + ((size_t)m * L + i) * L;
+                    for (int j = 0; j <= i; ++j) row[j] += s[j] / sum / B;
+                }
+            }
+        }
+        free(s);
+    }
+    return err;
+}

@@ -236,3 +236,42 @@ def averaged_maps(seed: int, n_maps: int, L: int = 512, n_samples: int = 16, boo
 
     _pmap(one, list(range(len(ids))))
     return out
+
+
+# --------------------------------------------------------------------------------------
+# Per-head query/key samples for producing the averaged maps on the GPU
+# --------------------------------------------------------------------------------------
+
+def qk_samples(seed: int, n_maps: int, B: int, L: int = 512, d: int = 64, planted: bool = True,
+               map_ids=None):
+    """Query and key rows of B calibration samples per map, bf16 bits [n, B, L, d] each.
+
+    Entries are N(0, 1).  With `planted`, map m gets its planted columns
+    (`planted_map_patterns`) as keys that every query favours: a unit direction u_m is
+    added (x 4.5) to every query row and to the key rows of those columns; and a local
+    diagonal: each key row also gets 0.35 x its own query row.  Each map has its own
+    random stream, so a subset (`map_ids`) reproduces the same rows as the full set.
+    """
+    ids = list(range(n_maps)) if map_ids is None else list(map_ids)
+    pl = planted_map_patterns(seed, n_maps, L)
+    streams = np.random.SeedSequence(seed + 104729).spawn(n_maps)
+    q_out = np.empty((len(ids), B, L, d), np.uint16)
+    k_out = np.empty((len(ids), B, L, d), np.uint16)
+
+    def one(o):
+        m = ids[o]
+        g = _gen(streams[m])
+        u = g.standard_normal(d).astype(np.float32)
+        u /= np.float32(np.linalg.norm(u))
+        for b in range(B):
+            q = g.standard_normal((L, d), dtype=np.float32)
+            k = g.standard_normal((L, d), dtype=np.float32)
+            if planted:
+                q += np.float32(4.5) * u
+                k[pl[m][1]] += np.float32(4.5) * u
+                k += np.float32(0.35) * q
+            q_out[o, b] = bf16_bits_from_f32(q)
+            k_out[o, b] = bf16_bits_from_f32(k)
+
+    _pmap(one, list(range(len(ids))))
+    return q_out, k_out
