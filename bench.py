@@ -57,6 +57,10 @@ DECODE_WORKLOADS = {
 SEEDS = {"llama3-8b-layer-64k": inputs.SEED_BASE + 4, "llama3.2-1b-layer-16k": inputs.SEED_BASE + 3,
          "llama3-8b-layer-16k": inputs.SEED_BASE + 6}
 CAPTURE_MAPS = 32  # one layer's heads
+# Stage-one map production: n_maps (layers x heads), samples B, capture length L, d
+MAPS_WORKLOADS = {
+    "maps-llama3.2-1b-l512-b16": (512, 16, 512, 64),
+}
 MUFU_EX2_PER_CLK_SM = 16  # B200: ex2.approx results per clock per SM (microbenchmark: 15.99)
 
 
@@ -537,13 +541,106 @@ def run_decode(args):
     print(json.dumps(line), flush=True)
 
 
+def run_maps(args):
+    """Time sparse_attn_maps on one GPU: averaged maps per second and the roofline of the
+    kernel (HBM bytes, one exponential and 2 d FLOPs per causal pair per sample)."""
+    import torch
+
+    import structured_sparse_attention_b200 as ssa
+    n, B, L, d = MAPS_WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    q_h, k_h = inputs.qk_samples(inputs.SEED_BASE + 9, n, B, L=L, d=d)
+    h_q = torch.from_numpy(q_h.view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_k = torch.from_numpy(k_h.view(np.int16)).view(torch.bfloat16).pin_memory()
+    q, k = h_q.to(dev), h_k.to(dev)
+    maps = torch.empty((n, L, L), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    scale = d ** -0.5
+
+    def call():
+        ssa.attn_maps(q, k, scale, out=maps, status=status, check=False)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0")
+    sampler.start()
+    time.sleep(0.3)
+    for e0, e1 in ev:
+        flush.fill_(1)  # inputs (1.07 GB) exceed L2 anyway; flushed for symmetry (not timed)
+        e0.record()
+        call()
+        e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())}")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    # end to end: Q and K in from pinned host memory, the maps back
+    h_m = torch.empty(maps.shape, dtype=torch.float32).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(3, min(args.steps, 10))
+    e0.record()
+    for _ in range(e_steps):
+        q.copy_(h_q, non_blocking=True)
+        k.copy_(h_k, non_blocking=True)
+        call()
+        h_m.copy_(maps, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1) / e_steps
+    pairs = n * B * L * (L + 1) // 2  # causal (i, j) pairs over all samples
+    algo_bytes = 2 * n * B * L * d * 2 + n * L * L * 4
+    algo_flops = 2 * d * pairs
+    hbm_gbs, tflops, _, peak_kind = load_peaks()
+    mufu = MUFU_EX2_PER_CLK_SM * props.multi_processor_count * sm_max_mhz() * 1e6
+    bounds = {"hbm": algo_bytes / (hbm_gbs * 1e9) * 1e3, "mufu": pairs / mufu * 1e3,
+              "tensor": algo_flops / (tflops * 1e12) * 1e3}
+    bound = max(bounds, key=bounds.get)
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": algo_bytes / (ms / 1e3) / 1e9, "peak": hbm_gbs, "unit": "GB/s"}
+    elif bound == "mufu":
+        roof = {"bound": "alu", "achieved": pairs / (ms / 1e3) / 1e9, "peak": mufu / 1e9, "unit": "Gex2/s",
+                "pipe": "MUFU ex2 (one per causal pair per sample)"}
+    else:
+        roof = {"bound": "tensor", "achieved": algo_flops / (ms / 1e3) / 1e12, "peak": tflops, "unit": "TFLOP/s"}
+    roof.update({"frac": bounds[bound] / ms, "traffic": None, "kernel": "attn_maps_kernel",
+                 "peak_source": f"{peak_kind}", "roofline_ms": bounds[bound], "bounds_ms": bounds,
+                 "algorithmic": {"bytes": algo_bytes, "flops": algo_flops, "ex2": pairs}})
+    line = {"metric": "stage-one averaged attention maps/s vs roofline", "value": n / (ms / 1e3), "unit": "maps/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "n_maps": n, "B": B, "L": L, "d": d,
+                       "l2": "inputs larger than L2 (Q+K 1.07 GB)"},
+            "roofline": roof, "clocks": clocks,
+            "e2e": {"value": n / (e_ms / 1e3), "unit": "maps/s", "h2d_bytes_per_step": int(2 * h_q.numel() * 2),
+                    "d2h_bytes_per_step": int(h_m.numel() * 4), "ms_per_step": e_ms},
+            "gpu_launches": args.steps, "cpu_baseline": None}
+    if not args.no_cpu_baseline:
+        from oracle import oracle as ora
+        ora.build()
+        cores = len(os.sched_getaffinity(0))
+        n_cpu = min(n, max(2, cores))  # one map per OpenMP thread
+        t0 = time.perf_counter()
+        ora.attn_maps(q_h[:n_cpu], k_h[:n_cpu], scale)
+        cpu_s = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": n_cpu / cpu_s, "unit": "maps/s", "cores": min(cores, n_cpu),
+                                "kind": "oracle", "sample": f"the first {n_cpu} of the {n} maps, all {B} samples "
+                                "each, fp64, one map per thread"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ssa", choices=["ssa", "reference"])
-    ap.add_argument("--workload", default="llama3-8b-layer-64k", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS))
+    ap.add_argument("--workload", default="llama3-8b-layer-64k", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(MAPS_WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle attention work")
@@ -555,6 +652,11 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if args.workload in MAPS_WORKLOADS:
+        if args.impl != "ssa" or args.gpus != 1:
+            ap.error("map workloads run the library on one GPU")
+        run_maps(args)
+        return
     if args.workload in DECODE_WORKLOADS:
         if args.impl != "ssa" or args.gpus != 1:
             ap.error("decode workloads run the library on one GPU")

@@ -54,6 +54,39 @@ extern "C" {
 #define SSA_BLOCK 128
 
 /* ------------------------------------------------------------------------------ */
+/* Stage one: averaged attention maps                                              */
+/* ------------------------------------------------------------------------------ */
+
+#define SSA_MAPS_MAX_B 32   /* samples averaged per call */
+#define SSA_MAPS_MAX_L 4096
+
+/*
+ * sparse_attn_maps -- the averaged attention maps stage one starts from ("What carries
+ * the argument": maps averaged over a calibration corpus; "Assumptions & free
+ * parameters": capture length L = 512), produced on the GPU from B samples of each
+ * map's query and key rows:
+ *   maps[m][i][j] = (1/B) sum_b softmax_j( scale * Q[m][b][i] . K[m][b][j] )   j <= i
+ *   maps[m][i][j] = 0                                                          j > i
+ * (causal row softmax per sample, then the mean over the samples), in the layout
+ * sparse_pattern_capture reads.  Arithmetic: bf16 inputs, fp32 logits (tensor cores),
+ * fp32 softmax with hardware 2^x, fp32 mean; each row sums to 1 up to fp32 rounding.
+ *
+ *   Q, K     device, bf16 [n_maps][B][L][d] contiguous (sample b of map m at
+ *            (m * B + b) * L * d), 16-byte aligned
+ *   n_maps   >= 1;  B in [1, SSA_MAPS_MAX_B];  L a multiple of 128 in [128, SSA_MAPS_MAX_L]
+ *   d        64 or 128 (else SSA_ERR_UNSUPPORTED)
+ *   scale    > 0, usually 1 / sqrt(d)
+ *   maps     device, float32 [n_maps][L][L] row-major, 16-byte aligned; every entry
+ *            is written
+ * Errors: SSA_ERR_INVALID for a null or misaligned pointer or a size out of range; an
+ * expired bounded wait sets SSA_ERR_TIMEOUT in dev_status (maps then unspecified).
+ * For B larger than SSA_MAPS_MAX_B, average the maps of several calls weighted by
+ * their sample counts.
+ */
+SSA_API int sparse_attn_maps(const void *Q, const void *K, int n_maps, int B, int L, int d, float scale,
+                             float *maps, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------------ */
 /* Stage one: pattern capture                                                      */
 /* ------------------------------------------------------------------------------ */
 

@@ -6,7 +6,7 @@ The binding is imported lazily so that the seeded input generator (``inputs``)
 can be used without loading the CUDA library.
 """
 
-_BINDING_NAMES = ("capture", "extend", "refill", "attn_fwd", "attn_ws_bytes", "attn_decode", "set_wait_limit_ns",
+_BINDING_NAMES = ("attn_maps", "capture", "extend", "refill", "attn_fwd", "attn_ws_bytes", "attn_decode", "set_wait_limit_ns",
                   "SSAError", "Plan", "load")
 
 

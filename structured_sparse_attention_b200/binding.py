@@ -11,6 +11,7 @@ caller zeroes it and reads it (the functions read it themselves when ``check``).
 from __future__ import annotations
 
 import ctypes as C
+import math
 import os
 
 import torch
@@ -24,7 +25,7 @@ ERRORS = {-1: "SSA_ERR_INVALID", -2: "SSA_ERR_UNSUPPORTED", -3: "SSA_ERR_CAPACIT
 BLOCK = 128
 
 #: Every symbol include/ssa.h declares.
-EXPORTS = ("sparse_pattern_capture_ws_bytes", "sparse_pattern_capture", "sparse_pattern_capture_noalloc",
+EXPORTS = ("sparse_attn_maps", "sparse_pattern_capture_ws_bytes", "sparse_pattern_capture", "sparse_pattern_capture_noalloc",
            "sparse_pattern_extend_ws_bytes", "sparse_pattern_extend",
            "sparse_attn_fwd_ws_bytes", "sparse_attn_fwd",
            "sparse_attn_decode_ws_bytes", "sparse_attn_decode",
@@ -63,6 +64,8 @@ def load():
             raise SSAError(-4, f"{LIB_PATH} is not built; run __graft_entry__.build()")
         lib = C.CDLL(LIB_PATH)
         V, I, D, SZ = C.c_void_p, C.c_int, C.c_double, C.c_size_t
+        lib.sparse_attn_maps.argtypes = [V, V, I, I, I, I, C.c_float, V, V, V]
+        lib.sparse_attn_maps.restype = I
         lib.sparse_pattern_capture_ws_bytes.argtypes = [I, I]
         lib.sparse_pattern_capture_ws_bytes.restype = SZ
         lib.sparse_pattern_capture.argtypes = [V, I, I, D, D, D, D, V, V, V, V, V, SZ, V, V]
@@ -128,6 +131,30 @@ def set_wait_limit_ns(ns: int) -> int:
 # ------------------------------------------------------------------------------------
 # Stage one
 # ------------------------------------------------------------------------------------
+
+def attn_maps(q: torch.Tensor, k: torch.Tensor, scale: float = None, *, stream=None, check: bool = True,
+              out=None, status=None):
+    """sparse_attn_maps: q, k bf16 [n_maps, B, L, d] (CUDA) -> averaged causal attention
+    maps float32 [n_maps, L, L] (entries above the diagonal are 0)."""
+    lib = load()
+    _need_cuda(q, "q", torch.bfloat16)
+    _need_cuda(k, "k", torch.bfloat16)
+    if q.dim() != 4 or q.shape != k.shape:
+        raise SSAError(-1, "q and k must both be [n_maps, B, L, d]")
+    n, B, L, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((n, L, L), dtype=torch.float32, device=q.device)
+    _need_cuda(out, "out", torch.float32)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=q.device)
+    cs, s = _stream(stream)
+    _check(lib.sparse_attn_maps(_ptr(q), _ptr(k), n, B, L, d, float(scale), _ptr(out), _ptr(status), cs))
+    if check:
+        _check_status(status, s)
+    return out
+
 
 def capture(maps: torch.Tensor, lam: float = 0.5, tau: float = 0.3, mu: float = 0.8,
             eps: float = 1e-8, *, stream=None, check: bool = True, out=None, ws=None, status=None):
