@@ -17,12 +17,13 @@
 // Each exponential is taken twice (once per pass): accumulating a whole row block over
 // all its chunks at once would need (rb + 1) x 128 fp32 values per row.
 //
-// Roles (320 threads): warps 0-7 softmax, two warpgroups splitting each tile's columns
-// (warpgroup h takes columns 64h..64h+63; thread il of a warpgroup owns row 128 rb + il,
-// TMEM lane il), so two warps per SM sub-partition share the MUFU; the halves' running
-// max and sum are combined through shared memory at the end of each sample.  Warp 8
-// lane 0: TMA producer of the Q block and K chunk of each tile.  Warp 9: tensor memory
-// (two S buffers of 128 columns) and lane 0 issues the MMAs.
+// Roles (576 threads): warps 0-15 softmax, four warpgroups splitting each tile's columns
+// (part h takes columns 32h..32h+31; thread il of a warpgroup owns row 128 rb + il,
+// TMEM lane il), so four warps per SM sub-partition share the MUFU and hide each
+// other's latencies; the parts' running max and sum are combined through shared memory
+// at the end of each sample, and part 0 keeps (m_b, 1 / l_b).  Warp 16 lane 0: TMA
+// producer of the Q block and K chunk of each tile.  Warp 17: tensor memory (two S
+// buffers of 128 columns) and lane 0 issues the MMAs.
 //
 // Every wait is bounded: on expiry the kernel records SSA_ERR_TIMEOUT, stops every role,
 // drains its copies and MMAs, frees tensor memory and returns.
@@ -36,30 +37,41 @@ namespace ssa {
 namespace {
 
 constexpr int kMapsMaxB = SSA_MAPS_MAX_B;
-constexpr int kMThreads = 320;
-constexpr int kMSoftmaxThreads = 256;
-constexpr int kMWarpTma = 8, kMWarpMma = 9;
-constexpr uint32_t kMTmemCols = 256;
+// The softmax splits every 128-column tile into kMParts column parts, one warpgroup
+// each, so that kMParts warps per SM sub-partition keep the MUFU fed.
+constexpr int kMParts = 4;
+constexpr int kMCols = 128 / kMParts;  // columns per thread and tile
+constexpr int kMSoftmaxThreads = 128 * kMParts;
+constexpr int kMThreads = kMSoftmaxThreads + 64;
+constexpr int kMWarpTma = kMParts * 4, kMWarpMma = kMParts * 4 + 1;
+constexpr int kMSBuf = 4;  // S buffers in tensor memory: the MMA runs up to three tiles ahead
+constexpr uint32_t kMTmemCols = 128 * kMSBuf;
 constexpr int kMBoxBytes = 128 * 128;  // 128 rows x 64 bf16, one 128-byte swizzle span
 constexpr int64_t kMDrainNs = 1000000000LL;
 
 template <int D>
 struct MCfg {
-    static constexpr int NS = (D == 64) ? 4 : 2;        // smem stages (Q block + K chunk)
+    static constexpr int NS = (D == 64) ? 3 : 2;        // smem stages (Q block + K chunk)
+    // d = 64 writes the map through shared memory with TMA stores (one 32-column x
+    // 128-row box per part); d = 128 has no room for the staging and stores directly
+    static constexpr bool STAGED = D == 64;
     static constexpr int BOXES = D / 64;
     static constexpr int TILE = BOXES * kMBoxBytes;     // one 128-row bf16 operand
     static constexpr int STAGE = 2 * TILE;
-    static constexpr int OFF_STAT = NS * STAGE;         // float2 [2 halves][MAXB][128]
-    static constexpr int OFF_XCH = OFF_STAT + 2 * kMapsMaxB * 128 * 8;  // float2 [2][2][128]
-    static constexpr int OFF_BAR = OFF_XCH + 2 * 2 * 128 * 8;
+    static constexpr int OFF_STAT = NS * STAGE;         // float2 [MAXB][128]: (m_b, 1 / l_b)
+    static constexpr int OFF_XCH = OFF_STAT + kMapsMaxB * 128 * 8;  // float2 [2][kMParts][128]
+    static constexpr int OFF_STG = OFF_XCH + 2 * kMParts * 128 * 8;  // [kMParts][128 rows][128 B]
+    static constexpr int OFF_BAR = OFF_STG + (STAGED ? kMParts * 128 * 128 : 0);
     static constexpr int SMEM = OFF_BAR + 1024 + 1024;  // barrier block + alignment slack
     static_assert(SMEM <= 232448, "shared memory budget exceeded");
 };
 
 struct MShared {
     uint64_t full[4], empty[4];
-    uint64_t s_full[2], s_empty[2];
+    uint64_t s_full[kMSBuf], s_empty[kMSBuf];
+    uint64_t stg_full[kMParts], stg_free[kMParts];  // staging buffer of each part
     uint64_t xch[2];
+    uint64_t stat_ready;  // part 0 has written every (m_b, 1 / l_b)
     uint64_t mma_drain, sm_done;
     uint32_t tmem_base;
     int abort;
@@ -88,6 +100,23 @@ __host__ __device__ constexpr uint32_t m_idesc(int M, int N) {
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Shared-memory store of four words; async-proxy fence; TMA tile store and bulk groups.
+__device__ __forceinline__ void m_st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ void m_fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void m_tma_store_2d(const void *tmap, const void *src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void m_bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void m_bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void m_bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Tile t of the CTA's sequence: pass 1 for t < nc B (b = t / nc, c = t % nc), then
 // pass 2 (c = t' / B, b = t' % B).
 __device__ __forceinline__ void m_tile(int t, int nc, int B, bool &pass2, int &b, int &c) {
@@ -106,7 +135,7 @@ __device__ __forceinline__ void m_tile(int t, int nc, int B, bool &pass2, int &b
 template <int D>
 __global__ void __launch_bounds__(kMThreads, 1)
     attn_maps_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const MapsParams p) {
+                     const __grid_constant__ CUtensorMap tmO, const MapsParams p) {
     using C = MCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -114,9 +143,10 @@ __global__ void __launch_bounds__(kMThreads, 1)
     MShared *sh = reinterpret_cast<MShared *>(smem + C::OFF_BAR);
     volatile int *abort = &sh->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // larger row blocks (more chunks) first
-    const int rb = p.nrb - 1 - static_cast<int>(blockIdx.x) / p.n_maps;
-    const int map = static_cast<int>(blockIdx.x) % p.n_maps;
+    // the row blocks of one map are adjacent CTAs (largest first), so the CTAs resident at
+    // a time share their maps' K rows in L2 and hold a working set of a few dozen maps
+    const int rb = p.nrb - 1 - static_cast<int>(blockIdx.x) % p.nrb;
+    const int map = static_cast<int>(blockIdx.x) / p.nrb;
     const int nc = rb + 1;
     const int T = 2 * nc * p.B;
     const int64_t lim = p.wait_ns;
@@ -126,11 +156,16 @@ __global__ void __launch_bounds__(kMThreads, 1)
             mbar_init(&sh->full[s], 1);
             mbar_init(&sh->empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kMSBuf; ++s) {
             mbar_init(&sh->s_full[s], 1);
             mbar_init(&sh->s_empty[s], kMSoftmaxThreads);
-            mbar_init(&sh->xch[s], kMSoftmaxThreads);
         }
+        for (int s = 0; s < 2; ++s) mbar_init(&sh->xch[s], kMSoftmaxThreads);
+        for (int h = 0; h < kMParts; ++h) {
+            mbar_init(&sh->stg_full[h], 4);  // one arrival per warp of the part
+            mbar_init(&sh->stg_free[h], 1);  // the part's leader, once the store has read it
+        }
+        mbar_init(&sh->stat_ready, 128);
         mbar_init(&sh->mma_drain, 1);
         mbar_init(&sh->sm_done, kMSoftmaxThreads);
         sh->abort = 0;
@@ -180,12 +215,15 @@ __global__ void __launch_bounds__(kMThreads, 1)
     } else if (warp == kMWarpMma) {
         if (lane == 0) {
             // ------------------------------- MMA issuer -------------------------------
+            // waits test the barrier first: try_wait in a thread with MMAs in flight costs
+            // about their drain time even on a completed phase
             constexpr uint32_t IDESC = m_idesc(128, 128);
             bool ok = true;
             for (int t = 0; t < T && ok; ++t) {
-                const int st = t % C::NS, sb = t & 1;
-                if (!mbar_wait(&sh->full[st], (t / C::NS) & 1, lim, abort)) ok = false;
-                if (ok && t >= 2 && !mbar_wait(&sh->s_empty[sb], ((t >> 1) - 1) & 1, lim, abort)) ok = false;
+                const int st = t % C::NS, sb = t % kMSBuf;
+                if (!mbar_wait_poll(&sh->full[st], (t / C::NS) & 1, lim, abort)) ok = false;
+                if (ok && t >= kMSBuf && !mbar_wait_poll(&sh->s_empty[sb], ((t / kMSBuf) - 1) & 1, lim, abort))
+                    ok = false;
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t sQ = smem_u32(smem + st * C::STAGE);
@@ -216,116 +254,208 @@ __global__ void __launch_bounds__(kMThreads, 1)
         tmem_dealloc(tmem, kMTmemCols);
     } else {
         // --------------------------------- softmax ---------------------------------
-        const int h = warp >> 2;  // column half of every tile
+        const int h = warp >> 2;  // column part of every tile
         const int il = 32 * (warp & 3) + lane;
         const int i = 128 * rb + il;
         const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-        float2 *stat = reinterpret_cast<float2 *>(smem + C::OFF_STAT) + h * kMapsMaxB * 128;
-        float2 *xch = reinterpret_cast<float2 *>(smem + C::OFF_XCH);  // [parity][half][row]
+        float2 *stat = reinterpret_cast<float2 *>(smem + C::OFF_STAT);
+        float2 *xch = reinterpret_cast<float2 *>(smem + C::OFF_XCH);  // [parity][part][row]
         const float sl2 = p.scale_log2;
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), zero2 = f2_pack(0.0f, 0.0f);
         float *row = p.maps + (static_cast<size_t>(map) * p.L + i) * p.L;
+        // A chunk of this part's columns of the row block (kMCols columns from col0), from
+        // w of every thread.  Staged: each thread writes its row into the part's staging
+        // buffer in the 128-byte swizzle the tensor map uses (16-byte unit j of row r at
+        // j ^ (r % 8)), the warps report on stg_full, and the part's leader stores the box
+        // with TMA and frees the buffer once the store has read it.
+        const bool leader = (warp & 3) == 0 && lane == 0;
+        uint8_t *stg = smem + C::OFF_STG + h * (128 * 128);
+        int ne = 0;  // chunks written by this part
+        auto put_chunk = [&](const uint32_t(&w)[kMCols], int col0) -> bool {
+            if constexpr (C::STAGED) {
+                if (ne >= 1 && !__all_sync(0xffffffffu, mbar_wait(&sh->stg_free[h], (ne - 1) & 1, lim, abort)))
+                    return false;
+                const uint32_t base = smem_u32(stg) + il * 128;
+#pragma unroll
+                for (int j = 0; j < kMCols / 4; ++j)
+                    m_st_shared_v4(base + ((j ^ (il & 7)) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                m_fence_proxy_async();  // the generic-proxy writes, before the TMA reads them
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh->stg_full[h]);
+                bool good = true;
+                if (leader) {
+                    if (mbar_wait(&sh->stg_full[h], ne & 1, lim, abort)) {
+                        m_tma_store_2d(&tmO, stg, col0, map * p.L + 128 * rb);
+                        m_bulk_commit();
+                        m_bulk_wait_read();
+                        mbar_arrive(&sh->stg_free[h]);
+                    } else {
+                        good = false;
+                    }
+                }
+                ++ne;
+                return __all_sync(0xffffffffu, good);
+            } else {
+                float *dst = row + col0;
+                if (p.align32) {
+#pragma unroll
+                    for (int k = 0; k < kMCols / 8; ++k) st_global_v8(dst + 8 * k, w + 8 * k);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < kMCols / 4; ++k)
+                        reinterpret_cast<uint4 *>(dst)[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                }
+                return true;
+            }
+        };
         bool ok = true;
         float m = -INFINITY, l = 0.0f;
-        float acc[64];
+        uint64_t acc[kMCols / 2];  // the row's running sum over samples, packed pairs
 #pragma unroll
-        for (int k = 0; k < 64; ++k) acc[k] = 0.0f;
+        for (int k = 0; k < kMCols / 2; ++k) acc[k] = zero2;
         for (int t = 0; t < T; ++t) {
             bool pass2;
             int b, c;
             m_tile(t, nc, p.B, pass2, b, c);
-            const int sb = t & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[sb], (t >> 1) & 1, lim, abort))) {
+            const int sb = t % kMSBuf;
+            if (pass2 && t == nc * p.B) {  // first tile of pass 2: every (m_b, 1 / l_b) is written
+                if (!__all_sync(0xffffffffu, mbar_wait(&sh->stat_ready, 0, lim, abort))) {
+                    ok = false;
+                    break;
+                }
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[sb], (t / kMSBuf) & 1, lim, abort))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            uint32_t r[64];
-            const uint32_t tS = tmem + lane_off + 128 * sb + 64 * h;
-            tmem_ld32(tS, r);
-            tmem_ld32(tS + 32, r + 32);
+            uint32_t r[kMCols];
+            tmem_ld32(tmem + lane_off + 128 * sb + kMCols * h, r);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&sh->s_empty[sb]);  // the S buffer may take tile t + 2
-            // causal keys of this row in the chunk: local column 64 h + k < nv
-            const int nv = (c < rb) ? 128 : il + 1;
-            const int kv = nv - 64 * h;  // k < kv active
+            mbar_arrive(&sh->s_empty[sb]);  // the S buffer may take tile t + kMSBuf
+            // causal keys of this row in the chunk: local column kMCols h + k < kv.  Only the
+            // diagonal chunk (c == rb) masks; the warp-uniform test keeps the other chunks
+            // free of selects.
+            const bool diag = c == rb;
+            const int kv = (diag ? il + 1 : 128) - kMCols * h;
             if (!pass2) {
-                float x[64];
-                float mx = -INFINITY;
+                uint64_t x[kMCols / 2];  // scaled logits as packed pairs (log2 domain)
 #pragma unroll
-                for (int k = 0; k < 64; ++k) {
-                    x[k] = (k < kv) ? __uint_as_float(r[k]) * sl2 : -INFINITY;
-                    mx = fmaxf(mx, x[k]);
-                }
-                const float m_new = fmaxf(m, mx);
-                if (m_new != -INFINITY) {  // else no causal key in this half yet
-                    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+                for (int k = 0; k < kMCols / 2; ++k)
+                    x[k] = f2_fma(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), sl2x2, zero2);
+                if (diag) {
 #pragma unroll
-                    for (int k = 0; k < 64; k += 4) {
-                        s0 += ex2_approx(x[k] - m_new);
-                        s1 += ex2_approx(x[k + 1] - m_new);
-                        s2 += ex2_approx(x[k + 2] - m_new);
-                        s3 += ex2_approx(x[k + 3] - m_new);
+                    for (int k = 0; k < kMCols / 2; ++k) {
+                        float a, b2;
+                        f2_unpack(x[k], a, b2);
+                        x[k] = f2_pack(2 * k < kv ? a : -INFINITY, 2 * k + 1 < kv ? b2 : -INFINITY);
                     }
-                    l = l * ex2_approx(m - m_new) + ((s0 + s1) + (s2 + s3));
+                }
+                float mx[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float a, b2;
+                    f2_unpack(x[q], a, b2);
+                    mx[q] = fmaxf(a, b2);
+                }
+#pragma unroll
+                for (int k = 4; k < kMCols / 2; ++k) {
+                    float a, b2;
+                    f2_unpack(x[k], a, b2);
+                    mx[k & 3] = fmax3(mx[k & 3], a, b2);
+                }
+                const float m_new = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
+                if (m_new != -INFINITY) {  // else no causal key in this part yet
+                    const uint64_t nm2 = f2_pack(-m_new, -m_new);
+                    uint64_t sum[4] = {zero2, zero2, zero2, zero2};
+#pragma unroll
+                    for (int k = 0; k < kMCols / 2; ++k) {
+                        float a, b2;
+                        f2_unpack(f2_add(x[k], nm2), a, b2);
+                        sum[k & 3] = f2_add(sum[k & 3], f2_pack(ex2_approx(a), ex2_approx(b2)));
+                    }
+                    float s0, s1, s2, s3, s4, s5, s6, s7;
+                    f2_unpack(sum[0], s0, s1);
+                    f2_unpack(sum[1], s2, s3);
+                    f2_unpack(sum[2], s4, s5);
+                    f2_unpack(sum[3], s6, s7);
+                    l = l * ex2_approx(m - m_new) + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
                     m = m_new;
                 }
                 if (c == nc - 1) {
-                    // combine the two halves of the row: both warpgroups compute the same
-                    // (m_b, 1 / l_b) from the same two pairs
+                    // combine the parts of the row: every part computes the same
+                    // (m_b, 1 / l_b) from the same pairs; part 0 keeps it for pass 2
                     const int par = b & 1;
-                    xch[(par * 2 + h) * 128 + il] = make_float2(m, l);
+                    xch[(par * kMParts + h) * 128 + il] = make_float2(m, l);
                     mbar_arrive(&sh->xch[par]);
                     if (!__all_sync(0xffffffffu, mbar_wait(&sh->xch[par], (b >> 1) & 1, lim, abort))) {
                         ok = false;
                         break;
                     }
-                    const float2 o0 = xch[(par * 2 + 0) * 128 + il];
-                    const float2 o1 = xch[(par * 2 + 1) * 128 + il];
-                    const float mb = fmaxf(o0.x, o1.x);  // finite: key 0 is causal for every row
-                    const float lb = o0.y * ex2_approx(o0.x - mb) + o1.y * ex2_approx(o1.x - mb);
-                    stat[b * 128 + il] = make_float2(mb, 1.0f / lb);
+                    if (h == 0) {
+                        float2 o[kMParts];
+                        float mb = -INFINITY;
+#pragma unroll
+                        for (int q = 0; q < kMParts; ++q) {
+                            o[q] = xch[(par * kMParts + q) * 128 + il];
+                            mb = fmaxf(mb, o[q].x);  // finite: key 0 is causal for every row
+                        }
+                        float lb = 0.0f;
+#pragma unroll
+                        for (int q = 0; q < kMParts; ++q) lb += o[q].y * ex2_approx(o[q].x - mb);
+                        stat[b * 128 + il] = make_float2(mb, 1.0f / lb);
+                        if (b == p.B - 1) mbar_arrive(&sh->stat_ready);  // release: every stat written
+                    }
                     m = -INFINITY;
                     l = 0.0f;
                 }
             } else {
                 const float2 st = stat[b * 128 + il];
+                const uint64_t nm2 = f2_pack(-st.x, -st.x), inv2 = f2_pack(st.y, st.y);
 #pragma unroll
-                for (int k = 0; k < 64; ++k) {
-                    const float e = ex2_approx(fmaf(__uint_as_float(r[k]), sl2, -st.x));
-                    acc[k] = fmaf((k < kv) ? e : 0.0f, st.y, acc[k]);
+                for (int k = 0; k < kMCols / 2; ++k) {
+                    float a, b2;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), sl2x2, nm2), a,
+                              b2);
+                    float e0 = ex2_approx(a), e1 = ex2_approx(b2);
+                    if (diag) {
+                        e0 = 2 * k < kv ? e0 : 0.0f;
+                        e1 = 2 * k + 1 < kv ? e1 : 0.0f;
+                    }
+                    acc[k] = f2_fma(f2_pack(e0, e1), inv2, acc[k]);
                 }
                 if (b == p.B - 1) {
-                    // the chunk of the map row, this half's 64 columns (256 bytes)
-                    uint32_t w[64];
+                    // the chunk of the map row, this part's columns
+                    const uint64_t ib2 = f2_pack(p.inv_B, p.inv_B);
+                    uint32_t w[kMCols];
 #pragma unroll
-                    for (int k = 0; k < 64; ++k) {
-                        w[k] = __float_as_uint(acc[k] * p.inv_B);
-                        acc[k] = 0.0f;
+                    for (int k = 0; k < kMCols / 2; ++k) {
+                        float a, b2;
+                        f2_unpack(f2_fma(acc[k], ib2, zero2), a, b2);
+                        w[2 * k] = __float_as_uint(a);
+                        w[2 * k + 1] = __float_as_uint(b2);
+                        acc[k] = zero2;
                     }
-                    float *dst = row + 128 * c + 64 * h;
-                    if (p.align32) {
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) st_global_v8(dst + 8 * k, w + 8 * k);
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 16; ++k)
-                            reinterpret_cast<uint4 *>(dst)[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                    if (!put_chunk(w, 128 * c + kMCols * h)) {
+                        ok = false;
+                        break;
                     }
                 }
             }
         }
         if (ok) {
             // the chunks above the diagonal block: zeros
-            for (int cc = nc; cc < p.nrb; ++cc) {
-                uint4 *dst = reinterpret_cast<uint4 *>(row + 128 * cc + 64 * h);
+            uint32_t z[kMCols];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) dst[k] = make_uint4(0, 0, 0, 0);
-            }
-        } else {
+            for (int k = 0; k < kMCols; ++k) z[k] = 0u;
+            for (int cc = nc; cc < p.nrb && ok; ++cc) ok = put_chunk(z, 128 * cc + kMCols * h);
+        }
+        if (!ok) {
             report(p.status, SSA_ERR_TIMEOUT);
             *abort = 1;
         }
+        if (C::STAGED && leader) m_bulk_wait_all();  // every map store of the part complete
         tc_fence_before();
         mbar_arrive(&sh->sm_done);
     }
@@ -366,16 +496,40 @@ int m_make_map(CUtensorMap *m, const void *base, int d, int rows, int depth) {
     return SSA_OK;
 }
 
+// 2-D map over the fp32 maps [n_maps * L rows][L columns]; box = 32 columns x 128 rows,
+// 128-byte swizzle (the staging layout of the kernel).
+int m_make_out_map(CUtensorMap *m, float *maps, int n_maps, int L) {
+    auto enc = m_encode_fn();
+    if (!enc) {
+        set_error("cuTensorMapEncodeTiled is unavailable");
+        return SSA_ERR_CUDA;
+    }
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(n_maps) * L};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(L) * 4};
+    cuuint32_t box[2] = {kMCols, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, maps, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (%d) for the maps output (n_maps=%d L=%d)", static_cast<int>(r),
+                  n_maps, L);
+        return SSA_ERR_CUDA;
+    }
+    return SSA_OK;
+}
+
 template <int D>
 int launch_maps(const void *Q, const void *K, const MapsParams &p, cudaStream_t s) {
     using C = MCfg<D>;
-    CUtensorMap mQ, mK;
+    CUtensorMap mQ, mK, mO;
     int rc;
     if ((rc = m_make_map(&mQ, Q, D, p.L, p.n_maps * p.B)) != SSA_OK) return rc;
     if ((rc = m_make_map(&mK, K, D, p.L, p.n_maps * p.B)) != SSA_OK) return rc;
+    if ((rc = m_make_out_map(&mO, p.maps, p.n_maps, p.L)) != SSA_OK) return rc;
     SSA_CUDA_TRY(cudaFuncSetAttribute(attn_maps_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
     const unsigned grid = static_cast<unsigned>(p.n_maps) * static_cast<unsigned>(p.nrb);
-    attn_maps_kernel<D><<<grid, kMThreads, C::SMEM, s>>>(mQ, mK, p);
+    attn_maps_kernel<D><<<grid, kMThreads, C::SMEM, s>>>(mQ, mK, mO, p);
     SSA_LAUNCH_CHECK();
     return SSA_OK;
 }
