@@ -7,7 +7,8 @@
 //   maps[m][i][j] = 0                                                        (j > i)
 // in the layout sparse_pattern_capture reads.
 //
-// One CTA per (map, 128-row block rb); the row block's keys are the chunks c = 0..rb of
+// Work items are (map, 128-row block rb), run by persistent CTAs (one per SM) whose
+// pipelines carry on from item to item; the row block's keys are the chunks c = 0..rb of
 // 128 keys, and a tile is one 128 x 128 block S = Q_b K_(b,c)^T (tcgen05, fp32 in TMEM):
 //   pass 1 (samples outer, chunks inner): per row the running max and sum of 2^(x - max)
 //          over the causal keys of sample b  ->  (m_b, 1 / l_b) kept in shared memory
@@ -117,6 +118,15 @@ __device__ __forceinline__ void m_bulk_commit() { asm volatile("cp.async.bulk.co
 __device__ __forceinline__ void m_bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void m_bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Work item q: row block nrb - 1 - q / n_maps of map q % n_maps.  The largest row blocks
+// come first and a CTA's items (q = x, x + gridDim.x, ...) cover every row-block size,
+// so the persistent CTAs get about the same number of tiles and the small items end the
+// run.
+__device__ __forceinline__ void m_item(int q, int n_maps, int nrb, int &map, int &rb) {
+    map = q % n_maps;
+    rb = nrb - 1 - q / n_maps;
+}
+
 // Tile t of the CTA's sequence: pass 1 for t < nc B (b = t / nc, c = t % nc), then
 // pass 2 (c = t' / B, b = t' % B).
 __device__ __forceinline__ void m_tile(int t, int nc, int B, bool &pass2, int &b, int &c) {
@@ -143,12 +153,9 @@ __global__ void __launch_bounds__(kMThreads, 1)
     MShared *sh = reinterpret_cast<MShared *>(smem + C::OFF_BAR);
     volatile int *abort = &sh->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // the row blocks of one map are adjacent CTAs (largest first), so the CTAs resident at
-    // a time share their maps' K rows in L2 and hold a working set of a few dozen maps
-    const int rb = p.nrb - 1 - static_cast<int>(blockIdx.x) % p.nrb;
-    const int map = static_cast<int>(blockIdx.x) / p.nrb;
-    const int nc = rb + 1;
-    const int T = 2 * nc * p.B;
+    // persistent: CTA x takes the items x, x + gridDim.x, ...; every role walks the same
+    // items and counts tiles (g), so the pipelines run on across items
+    const int n_items = p.n_maps * p.nrb;
     const int64_t lim = p.wait_ns;
 
     if (threadIdx.x == 0) {
@@ -186,22 +193,27 @@ __global__ void __launch_bounds__(kMThreads, 1)
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             bool ok = true;
-            int t = 0;
-            for (; t < T; ++t) {
-                const int st = t % C::NS;
-                if (t >= C::NS && !mbar_wait(&sh->empty[st], ((t / C::NS) - 1) & 1, lim, abort)) {
-                    ok = false;
-                    break;
-                }
-                bool pass2;
-                int b, c;
-                m_tile(t, nc, p.B, pass2, b, c);
-                const int z = map * p.B + b;
-                uint8_t *dq = smem + st * C::STAGE;
-                mbar_arrive_expect_tx(&sh->full[st], C::STAGE);
-                for (int x = 0; x < C::BOXES; ++x) {
-                    tma_load_3d(dq + x * kMBoxBytes, &tmQ, &sh->full[st], 64 * x, 128 * rb, z);
-                    tma_load_3d(dq + C::TILE + x * kMBoxBytes, &tmK, &sh->full[st], 64 * x, 128 * c, z);
+            int g = 0;
+            for (int q = blockIdx.x; q < n_items && ok; q += gridDim.x) {
+                int map, rb;
+                m_item(q, p.n_maps, p.nrb, map, rb);
+                const int nc = rb + 1, T = 2 * nc * p.B;
+                for (int t = 0; t < T; ++t, ++g) {
+                    const int st = g % C::NS;
+                    if (g >= C::NS && !mbar_wait(&sh->empty[st], ((g / C::NS) - 1) & 1, lim, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    bool pass2;
+                    int b, c;
+                    m_tile(t, nc, p.B, pass2, b, c);
+                    const int z = map * p.B + b;
+                    uint8_t *dq = smem + st * C::STAGE;
+                    mbar_arrive_expect_tx(&sh->full[st], C::STAGE);
+                    for (int x = 0; x < C::BOXES; ++x) {
+                        tma_load_3d(dq + x * kMBoxBytes, &tmQ, &sh->full[st], 64 * x, 128 * rb, z);
+                        tma_load_3d(dq + C::TILE + x * kMBoxBytes, &tmK, &sh->full[st], 64 * x, 128 * c, z);
+                    }
                 }
             }
             if (!ok) {
@@ -209,7 +221,7 @@ __global__ void __launch_bounds__(kMThreads, 1)
                 *abort = 1;
             }
             // never leave the CTA with a copy still writing shared memory
-            for (int u = (t > C::NS ? t - C::NS : 0); u < t; ++u)
+            for (int u = (g > C::NS ? g - C::NS : 0); u < g; ++u)
                 mbar_wait(&sh->full[u % C::NS], (u / C::NS) & 1, kMDrainNs, nullptr);
         }
     } else if (warp == kMWarpMma) {
@@ -219,10 +231,16 @@ __global__ void __launch_bounds__(kMThreads, 1)
             // about their drain time even on a completed phase
             constexpr uint32_t IDESC = m_idesc(128, 128);
             bool ok = true;
-            for (int t = 0; t < T && ok; ++t) {
-                const int st = t % C::NS, sb = t % kMSBuf;
-                if (!mbar_wait_poll(&sh->full[st], (t / C::NS) & 1, lim, abort)) ok = false;
-                if (ok && t >= kMSBuf && !mbar_wait_poll(&sh->s_empty[sb], ((t / kMSBuf) - 1) & 1, lim, abort))
+            int n_tiles = 0;
+            for (int q = blockIdx.x; q < n_items; q += gridDim.x) {
+                int map, rb;
+                m_item(q, p.n_maps, p.nrb, map, rb);
+                n_tiles += 2 * (rb + 1) * p.B;
+            }
+            for (int g = 0; g < n_tiles && ok; ++g) {
+                const int st = g % C::NS, sb = g % kMSBuf;
+                if (!mbar_wait_poll(&sh->full[st], (g / C::NS) & 1, lim, abort)) ok = false;
+                if (ok && g >= kMSBuf && !mbar_wait_poll(&sh->s_empty[sb], ((g / kMSBuf) - 1) & 1, lim, abort))
                     ok = false;
                 if (!ok) break;
                 tc_fence_after();
@@ -256,13 +274,13 @@ __global__ void __launch_bounds__(kMThreads, 1)
         // --------------------------------- softmax ---------------------------------
         const int h = warp >> 2;  // column part of every tile
         const int il = 32 * (warp & 3) + lane;
-        const int i = 128 * rb + il;
+        int map = 0, rb = 0;  // the current item
         const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
         float2 *stat = reinterpret_cast<float2 *>(smem + C::OFF_STAT);
         float2 *xch = reinterpret_cast<float2 *>(smem + C::OFF_XCH);  // [parity][part][row]
         const float sl2 = p.scale_log2;
         const uint64_t sl2x2 = f2_pack(sl2, sl2), zero2 = f2_pack(0.0f, 0.0f);
-        float *row = p.maps + (static_cast<size_t>(map) * p.L + i) * p.L;
+        float *row = p.maps;  // row 128 rb + il of the current item's map
         // A chunk of this part's columns of the row block (kMCols columns from col0), from
         // w of every thread.  Staged: each thread writes its row into the part's staging
         // buffer in the 128-byte swizzle the tensor map uses (16-byte unit j of row r at
@@ -313,143 +331,152 @@ __global__ void __launch_bounds__(kMThreads, 1)
         uint64_t acc[kMCols / 2];  // the row's running sum over samples, packed pairs
 #pragma unroll
         for (int k = 0; k < kMCols / 2; ++k) acc[k] = zero2;
-        for (int t = 0; t < T; ++t) {
-            bool pass2;
-            int b, c;
-            m_tile(t, nc, p.B, pass2, b, c);
-            const int sb = t % kMSBuf;
-            if (pass2 && t == nc * p.B) {  // first tile of pass 2: every (m_b, 1 / l_b) is written
-                if (!__all_sync(0xffffffffu, mbar_wait(&sh->stat_ready, 0, lim, abort))) {
+        int g = 0, gb = 0, gi = 0;  // tiles, samples (pass-1 exchanges) and items so far
+        for (int q = blockIdx.x; q < n_items && ok; q += gridDim.x, ++gi) {
+            m_item(q, p.n_maps, p.nrb, map, rb);
+            const int nc = rb + 1, T = 2 * nc * p.B;
+            row = p.maps + (static_cast<size_t>(map) * p.L + 128 * rb + il) * p.L;
+            for (int t = 0; t < T; ++t, ++g) {
+                bool pass2;
+                int b, c;
+                m_tile(t, nc, p.B, pass2, b, c);
+                const int sb = g % kMSBuf;
+                if (pass2 && t == nc * p.B) {  // first tile of pass 2: every (m_b, 1 / l_b) is written
+                    if (!__all_sync(0xffffffffu, mbar_wait(&sh->stat_ready, gi & 1, lim, abort))) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[sb], (g / kMSBuf) & 1, lim, abort))) {
                     ok = false;
                     break;
                 }
-            }
-            if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[sb], (t / kMSBuf) & 1, lim, abort))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            uint32_t r[kMCols];
-            tmem_ld32(tmem + lane_off + 128 * sb + kMCols * h, r);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&sh->s_empty[sb]);  // the S buffer may take tile t + kMSBuf
-            // causal keys of this row in the chunk: local column kMCols h + k < kv.  Only the
-            // diagonal chunk (c == rb) masks; the warp-uniform test keeps the other chunks
-            // free of selects.
-            const bool diag = c == rb;
-            const int kv = (diag ? il + 1 : 128) - kMCols * h;
-            if (!pass2) {
-                uint64_t x[kMCols / 2];  // scaled logits as packed pairs (log2 domain)
+                tc_fence_after();
+                uint32_t r[kMCols];
+                tmem_ld32(tmem + lane_off + 128 * sb + kMCols * h, r);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&sh->s_empty[sb]);  // the S buffer may take tile t + kMSBuf
+                // causal keys of this row in the chunk: local column kMCols h + k < kv.  Only the
+                // diagonal chunk (c == rb) masks; the warp-uniform test keeps the other chunks
+                // free of selects.
+                const bool diag = c == rb;
+                const int kv = (diag ? il + 1 : 128) - kMCols * h;
+                if (!pass2) {
+                    uint64_t x[kMCols / 2];  // scaled logits as packed pairs (log2 domain)
 #pragma unroll
-                for (int k = 0; k < kMCols / 2; ++k)
-                    x[k] = f2_fma(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), sl2x2, zero2);
-                if (diag) {
+                    for (int k = 0; k < kMCols / 2; ++k)
+                        x[k] = f2_fma(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), sl2x2, zero2);
+                    if (diag) {
 #pragma unroll
-                    for (int k = 0; k < kMCols / 2; ++k) {
+                        for (int k = 0; k < kMCols / 2; ++k) {
+                            float a, b2;
+                            f2_unpack(x[k], a, b2);
+                            x[k] = f2_pack(2 * k < kv ? a : -INFINITY, 2 * k + 1 < kv ? b2 : -INFINITY);
+                        }
+                    }
+                    float mx[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float a, b2;
+                        f2_unpack(x[q], a, b2);
+                        mx[q] = fmaxf(a, b2);
+                    }
+#pragma unroll
+                    for (int k = 4; k < kMCols / 2; ++k) {
                         float a, b2;
                         f2_unpack(x[k], a, b2);
-                        x[k] = f2_pack(2 * k < kv ? a : -INFINITY, 2 * k + 1 < kv ? b2 : -INFINITY);
+                        mx[k & 3] = fmax3(mx[k & 3], a, b2);
                     }
-                }
-                float mx[4];
+                    const float m_new = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
+                    if (m_new != -INFINITY) {  // else no causal key in this part yet
+                        const uint64_t nm2 = f2_pack(-m_new, -m_new);
+                        uint64_t sum[4] = {zero2, zero2, zero2, zero2};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float a, b2;
-                    f2_unpack(x[q], a, b2);
-                    mx[q] = fmaxf(a, b2);
-                }
-#pragma unroll
-                for (int k = 4; k < kMCols / 2; ++k) {
-                    float a, b2;
-                    f2_unpack(x[k], a, b2);
-                    mx[k & 3] = fmax3(mx[k & 3], a, b2);
-                }
-                const float m_new = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
-                if (m_new != -INFINITY) {  // else no causal key in this part yet
-                    const uint64_t nm2 = f2_pack(-m_new, -m_new);
-                    uint64_t sum[4] = {zero2, zero2, zero2, zero2};
-#pragma unroll
-                    for (int k = 0; k < kMCols / 2; ++k) {
-                        float a, b2;
-                        f2_unpack(f2_add(x[k], nm2), a, b2);
-                        sum[k & 3] = f2_add(sum[k & 3], f2_pack(ex2_approx(a), ex2_approx(b2)));
-                    }
-                    float s0, s1, s2, s3, s4, s5, s6, s7;
-                    f2_unpack(sum[0], s0, s1);
-                    f2_unpack(sum[1], s2, s3);
-                    f2_unpack(sum[2], s4, s5);
-                    f2_unpack(sum[3], s6, s7);
-                    l = l * ex2_approx(m - m_new) + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
-                    m = m_new;
-                }
-                if (c == nc - 1) {
-                    // combine the parts of the row: every part computes the same
-                    // (m_b, 1 / l_b) from the same pairs; part 0 keeps it for pass 2
-                    const int par = b & 1;
-                    xch[(par * kMParts + h) * 128 + il] = make_float2(m, l);
-                    mbar_arrive(&sh->xch[par]);
-                    if (!__all_sync(0xffffffffu, mbar_wait(&sh->xch[par], (b >> 1) & 1, lim, abort))) {
-                        ok = false;
-                        break;
-                    }
-                    if (h == 0) {
-                        float2 o[kMParts];
-                        float mb = -INFINITY;
-#pragma unroll
-                        for (int q = 0; q < kMParts; ++q) {
-                            o[q] = xch[(par * kMParts + q) * 128 + il];
-                            mb = fmaxf(mb, o[q].x);  // finite: key 0 is causal for every row
+                        for (int k = 0; k < kMCols / 2; ++k) {
+                            float a, b2;
+                            f2_unpack(f2_add(x[k], nm2), a, b2);
+                            sum[k & 3] = f2_add(sum[k & 3], f2_pack(ex2_approx(a), ex2_approx(b2)));
                         }
-                        float lb = 0.0f;
-#pragma unroll
-                        for (int q = 0; q < kMParts; ++q) lb += o[q].y * ex2_approx(o[q].x - mb);
-                        stat[b * 128 + il] = make_float2(mb, 1.0f / lb);
-                        if (b == p.B - 1) mbar_arrive(&sh->stat_ready);  // release: every stat written
+                        float s0, s1, s2, s3, s4, s5, s6, s7;
+                        f2_unpack(sum[0], s0, s1);
+                        f2_unpack(sum[1], s2, s3);
+                        f2_unpack(sum[2], s4, s5);
+                        f2_unpack(sum[3], s6, s7);
+                        l = l * ex2_approx(m - m_new) + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
+                        m = m_new;
                     }
-                    m = -INFINITY;
-                    l = 0.0f;
-                }
-            } else {
-                const float2 st = stat[b * 128 + il];
-                const uint64_t nm2 = f2_pack(-st.x, -st.x), inv2 = f2_pack(st.y, st.y);
+                    if (c == nc - 1) {
+                        // combine the parts of the row: every part computes the same
+                        // (m_b, 1 / l_b) from the same pairs; part 0 keeps it for pass 2
+                        // parts' slots double-buffered by sample parity: a part reaches the next
+                        // exchange of the same parity only after everyone passed the one between
+                        const int par = gb & 1;
+                        xch[(par * kMParts + h) * 128 + il] = make_float2(m, l);
+                        mbar_arrive(&sh->xch[par]);
+                        if (!__all_sync(0xffffffffu, mbar_wait(&sh->xch[par], (gb >> 1) & 1, lim, abort))) {
+                            ok = false;
+                            break;
+                        }
+                        if (h == 0) {
+                            float2 o[kMParts];
+                            float mb = -INFINITY;
 #pragma unroll
-                for (int k = 0; k < kMCols / 2; ++k) {
-                    float a, b2;
-                    f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), sl2x2, nm2), a,
-                              b2);
-                    float e0 = ex2_approx(a), e1 = ex2_approx(b2);
-                    if (diag) {
-                        e0 = 2 * k < kv ? e0 : 0.0f;
-                        e1 = 2 * k + 1 < kv ? e1 : 0.0f;
+                            for (int q = 0; q < kMParts; ++q) {
+                                o[q] = xch[(par * kMParts + q) * 128 + il];
+                                mb = fmaxf(mb, o[q].x);  // finite: key 0 is causal for every row
+                            }
+                            float lb = 0.0f;
+#pragma unroll
+                            for (int q = 0; q < kMParts; ++q) lb += o[q].y * ex2_approx(o[q].x - mb);
+                            stat[b * 128 + il] = make_float2(mb, 1.0f / lb);
+                            if (b == p.B - 1) mbar_arrive(&sh->stat_ready);  // release: every stat written
+                        }
+                        m = -INFINITY;
+                        l = 0.0f;
+                        ++gb;
                     }
-                    acc[k] = f2_fma(f2_pack(e0, e1), inv2, acc[k]);
-                }
-                if (b == p.B - 1) {
-                    // the chunk of the map row, this part's columns
-                    const uint64_t ib2 = f2_pack(p.inv_B, p.inv_B);
-                    uint32_t w[kMCols];
+                } else {
+                    const float2 st = stat[b * 128 + il];
+                    const uint64_t nm2 = f2_pack(-st.x, -st.x), inv2 = f2_pack(st.y, st.y);
 #pragma unroll
                     for (int k = 0; k < kMCols / 2; ++k) {
                         float a, b2;
-                        f2_unpack(f2_fma(acc[k], ib2, zero2), a, b2);
-                        w[2 * k] = __float_as_uint(a);
-                        w[2 * k + 1] = __float_as_uint(b2);
-                        acc[k] = zero2;
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), sl2x2, nm2), a,
+                                  b2);
+                        float e0 = ex2_approx(a), e1 = ex2_approx(b2);
+                        if (diag) {
+                            e0 = 2 * k < kv ? e0 : 0.0f;
+                            e1 = 2 * k + 1 < kv ? e1 : 0.0f;
+                        }
+                        acc[k] = f2_fma(f2_pack(e0, e1), inv2, acc[k]);
                     }
-                    if (!put_chunk(w, 128 * c + kMCols * h)) {
-                        ok = false;
-                        break;
+                    if (b == p.B - 1) {
+                        // the chunk of the map row, this part's columns
+                        const uint64_t ib2 = f2_pack(p.inv_B, p.inv_B);
+                        uint32_t w[kMCols];
+#pragma unroll
+                        for (int k = 0; k < kMCols / 2; ++k) {
+                            float a, b2;
+                            f2_unpack(f2_fma(acc[k], ib2, zero2), a, b2);
+                            w[2 * k] = __float_as_uint(a);
+                            w[2 * k + 1] = __float_as_uint(b2);
+                            acc[k] = zero2;
+                        }
+                        if (!put_chunk(w, 128 * c + kMCols * h)) {
+                            ok = false;
+                            break;
+                        }
                     }
                 }
             }
-        }
-        if (ok) {
-            // the chunks above the diagonal block: zeros
-            uint32_t z[kMCols];
+            if (ok) {
+                // the chunks above the diagonal block: zeros
+                uint32_t z[kMCols];
 #pragma unroll
-            for (int k = 0; k < kMCols; ++k) z[k] = 0u;
-            for (int cc = nc; cc < p.nrb && ok; ++cc) ok = put_chunk(z, 128 * cc + kMCols * h);
+                for (int k = 0; k < kMCols; ++k) z[k] = 0u;
+                for (int cc = nc; cc < p.nrb && ok; ++cc) ok = put_chunk(z, 128 * cc + kMCols * h);
+            }
         }
         if (!ok) {
             report(p.status, SSA_ERR_TIMEOUT);
@@ -528,7 +555,11 @@ int launch_maps(const void *Q, const void *K, const MapsParams &p, cudaStream_t 
     if ((rc = m_make_map(&mK, K, D, p.L, p.n_maps * p.B)) != SSA_OK) return rc;
     if ((rc = m_make_out_map(&mO, p.maps, p.n_maps, p.L)) != SSA_OK) return rc;
     SSA_CUDA_TRY(cudaFuncSetAttribute(attn_maps_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
-    const unsigned grid = static_cast<unsigned>(p.n_maps) * static_cast<unsigned>(p.nrb);
+    int dev = 0, sms = 0;
+    SSA_CUDA_TRY(cudaGetDevice(&dev));
+    SSA_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    const long long items = static_cast<long long>(p.n_maps) * p.nrb;
+    const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);  // one persistent CTA per SM
     attn_maps_kernel<D><<<grid, kMThreads, C::SMEM, s>>>(mQ, mK, mO, p);
     SSA_LAUNCH_CHECK();
     return SSA_OK;
