@@ -581,8 +581,8 @@ extern "C" int sparse_attn_maps(const void *Q, const void *K, int n_maps, int B,
                   kMapsMaxB);
     SSA_CHECK_ARG(L >= 128 && L <= SSA_MAPS_MAX_L && L % 128 == 0,
                   "sparse_attn_maps: L must be a multiple of 128 in [128, %d] (got %d)", SSA_MAPS_MAX_L, L);
-    SSA_CHECK_ARG(static_cast<int64_t>(n_maps) * B < (1LL << 30) &&
-                      static_cast<int64_t>(n_maps) * (L / 128) < (1LL << 31),
+    // tile coordinates (sample index, map row) are 32-bit in the kernel and the TMA maps
+    SSA_CHECK_ARG(static_cast<int64_t>(n_maps) * B < (1LL << 30) && static_cast<int64_t>(n_maps) * L < (1LL << 31),
                   "sparse_attn_maps: too many maps");
     SSA_CHECK_ARG(aligned16(Q) && aligned16(K) && aligned16(maps),
                   "sparse_attn_maps: Q, K and maps must be 16-byte aligned");

@@ -68,6 +68,15 @@ def test_host_argument_checks(lib):
     rc = lib.sparse_attn_fwd(dummy, dummy, dummy, 1, 1, 300, 64, C.byref(plan), None, 0.1, dummy, dummy,
                              None, 0, None, None)
     assert rc == -1 and b"plan" in lib.ssa_last_error()
+    # averaged maps: sizes and head dimension are checked before any device work
+    for n, B, L, d, want in [(1, 2, 200, 64, -1), (1, 0, 128, 64, -1), (1, 33, 128, 64, -1),
+                             (1, 2, 128, 96, -2), (1, 2, 8192, 64, -1), (1 << 20, 1, 4096, 64, -1)]:
+        rc = lib.sparse_attn_maps(dummy, dummy, n, B, L, d, 0.125, dummy, None, None)
+        assert rc == want, (n, B, L, d, rc)
+    rc = lib.sparse_attn_maps(dummy, dummy, 1, 2, 128, 64, 0.0, dummy, None, None)
+    assert rc == -1 and b"scale" in lib.ssa_last_error()
+    rc = lib.sparse_attn_maps(P(8), dummy, 1, 2, 128, 64, 0.125, dummy, None, None)
+    assert rc == -1 and b"aligned" in lib.ssa_last_error()
     # extend: bad sizes
     sizes = binding.PlanSizes()
     rc = lib.sparse_pattern_extend(0, dummy, dummy, dummy, dummy, 10, C.byref(sizes), None, dummy, 1 << 20,
