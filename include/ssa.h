@@ -73,7 +73,8 @@ extern "C" {
  *
  *   Q, K     device, bf16 [n_maps][B][L][d] contiguous (sample b of map m at
  *            (m * B + b) * L * d), 16-byte aligned
- *   n_maps   >= 1;  B in [1, SSA_MAPS_MAX_B];  L a multiple of 128 in [128, SSA_MAPS_MAX_L]
+ *   n_maps   >= 1 with n_maps * L < 2^31 and n_maps * B < 2^30;  B in [1, SSA_MAPS_MAX_B];
+ *            L a multiple of 128 in [128, SSA_MAPS_MAX_L]
  *   d        64 or 128 (else SSA_ERR_UNSUPPORTED)
  *   scale    > 0, usually 1 / sqrt(d)
  *   maps     device, float32 [n_maps][L][L] row-major, 16-byte aligned; every entry
