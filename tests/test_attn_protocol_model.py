@@ -23,46 +23,21 @@ The model also shows that releasing a V stage without first observing its fill (
 rule the issuers follow) breaks the phase invariant for runs of tile-less items.
 """
 
-import heapq
 import random
 
 import pytest
 
+from protocol_sim import Engine, ProtocolError
+
 NK, NV, RING = 2, 3, 4
 
 
-class ProtocolError(AssertionError):
-    pass
-
-
-class Barrier:
-    def __init__(self, sim, name, count):
-        self.sim, self.name, self.count = sim, name, count
-        self.pending = count
-        self.completions = 0
-        self.waiters = []  # (agent, phase)
-
-    def arrive(self, n=1):
-        self.pending -= n
-        if self.pending < 0:
-            raise ProtocolError(f"{self.name}: more arrivals than the count in one phase")
-        if self.pending == 0:
-            self.completions += 1
-            self.pending = self.count
-            woken, self.waiters = self.waiters, []
-            for agent, phase in woken:
-                self.sim.wait_on(agent, self, phase)
-
-
-class Sim:
+class Sim(Engine):
     def __init__(self, seed, items, release_without_fill=False):
-        self.rng = random.Random(seed)
-        self.t = 0
-        self.q = []
-        self.seq = 0
+        super().__init__(seed)
         self.items = items
         self.release_without_fill = release_without_fill
-        B = lambda n, c: Barrier(self, n, c)
+        B = self.barrier
         self.item_full = [B(f"item_full{r}", 1) for r in range(RING)]
         self.item_empty = [B(f"item_empty{r}", 1 + 2) for r in range(RING)]  # Q/V producer + 2 softmax
         self.q_full = [B(f"q_full{s}", 1) for s in range(2)]
@@ -77,103 +52,15 @@ class Sim:
         self.o_empty = [B(f"o_empty{s}", 1) for s in range(2)]
         self.ring = [None] * RING
         self.kflags = [None] * NK
-        self.turn = 0
-        self.turn_waiters = []
-        self.pipe_free_at = 0
-        self.readers = {}  # buffer -> completion time of the last MMA reading it
         self.epi_done = [0, 0]   # epilogues that have read O, per slot
         self.first_pv = [0, 0]   # first PVs of items issued, per slot
-        self.waiting = {}        # agent -> (barrier, phase) of its last wait
         self.k_content, self.v_content = [None] * NK, [None] * NV
         self.consumed = []
-        self.done = set()
-        self.agents = {}
-
-    # -- scheduling -------------------------------------------------------------------
-    def at(self, t, agent, value=None):
-        self.seq += 1
-        heapq.heappush(self.q, (t, self.seq, agent, value))
-
-    def wait_on(self, agent, bar, phase):
-        # parity wait for completion of `phase` (an explicit phase index)
-        self.waiting[agent] = (bar, phase)
-        if bar.completions >= phase + 2:
-            raise ProtocolError(f"{bar.name}: waiter {agent} targets phase {phase}, "
-                                f"but {bar.completions} phases have completed")
-        if bar.completions >= phase + 1:
-            self.at(self.t + self.rng.randint(1, 20), agent)
-        else:
-            bar.waiters.append((agent, phase))
-
-    def later(self, dt, fn):
-        self.seq += 1
-        heapq.heappush(self.q, (self.t + dt, self.seq, None, fn))
-
-    # -- tensor pipe ------------------------------------------------------------------
-    def mma(self, duration, reads):
-        start = max(self.t, self.pipe_free_at)
-        self.pipe_free_at = start + duration
-        for buf in reads:
-            self.readers[buf] = max(self.readers.get(buf, 0), self.pipe_free_at)
-        return self.pipe_free_at
-
-    def commit(self, bar):
-        done = max(self.t, self.pipe_free_at)
-        self.later(done - self.t + 1, lambda: bar.arrive())
-
-    def tma(self, bar, buf):
-        if self.readers.get(buf, 0) > self.t:
-            raise ProtocolError(f"{buf} refilled at {self.t} while an MMA reads it until {self.readers[buf]}")
-        self.later(self.rng.randint(200, 3000), lambda: bar.arrive())
 
     def run(self, limit=10 ** 9):
-        self.agents = {"kprod": k_producer(self), "qvprod": qv_producer(self),
-                       "mma0": mma_issuer(self, 0), "mma1": mma_issuer(self, 1),
-                       "sm0": softmax(self, 0), "sm1": softmax(self, 1)}
-        for name in self.agents:
-            self.at(0, name)
-        while self.q:
-            t, _, agent, value = heapq.heappop(self.q)
-            self.t = t
-            if t > limit:
-                break
-            if agent is None:
-                value()
-                continue
-            gen = self.agents[agent]
-            if agent in self.waiting:
-                bar, phase = self.waiting.pop(agent)
-                if bar.completions != phase + 1:  # a poll here would see the wrong parity
-                    raise ProtocolError(f"{bar.name}: {agent} resumes for phase {phase} after "
-                                        f"{bar.completions} completions")
-            try:
-                cmd = next(gen)
-            except StopIteration:
-                self.done.add(agent)
-                continue
-            kind = cmd[0]
-            if kind == "wait":
-                self.wait_on(agent, cmd[1], cmd[2])
-            elif kind == "delay":
-                self.at(self.t + cmd[1], agent)
-            elif kind == "turn":
-                if self.turn == cmd[1]:
-                    self.at(self.t + 1, agent)
-                else:
-                    self.turn_waiters.append((agent, cmd[1]))
-        if len(self.done) != len(self.agents):
-            stuck = sorted(set(self.agents) - self.done)
-            raise ProtocolError(f"deadlock: {stuck} never finished")
-
-    def pass_turn(self, value):
-        self.turn = value
-        keep = []
-        for agent, want in self.turn_waiters:
-            if want == value:
-                self.at(self.t + 1, agent)
-            else:
-                keep.append((agent, want))
-        self.turn_waiters = keep
+        super().run({"kprod": k_producer(self), "qvprod": qv_producer(self),
+                     "mma0": mma_issuer(self, 0), "mma1": mma_issuer(self, 1),
+                     "sm0": softmax(self, 0), "sm1": softmax(self, 1)}, limit)
 
 
 # ---------------------------------------------------------------------------------------
