@@ -122,6 +122,94 @@ def nnz_per_head(diags, verts, S):
     return np.array(out, np.int64)
 
 
+# Sensitivity of stage one to its free parameters (lambda, tau, mu): the referee's
+# missing analysis, run with the library's capture and the extension to S.
+SWEEP_WORKLOADS = {
+    "capture-sweep-128maps-l512": (128, 512, 65536),  # maps, L, S of the extended mask
+}
+SWEEP_GRID = {"lam": (0.5, 1.0), "tau": (0.1, 0.2, 0.3, 0.4, 0.5), "mu": (0.6, 0.7, 0.8, 0.9)}
+
+
+def capture_sweep(capture, planted, S, grid=SWEEP_GRID):
+    """For every (lambda, tau, mu) of `grid`: the kept diagonals and columns per map, the
+    recall and precision of the planted patterns, and the density of the extended mask at
+    S (retained pairs / causal pairs, mean over maps).  `capture(lam, tau, mu)` returns the
+    host CSR lists (diag_ptr, diag_offsets, vert_ptr, vert_cols) of the maps whose planted
+    (diagonals, columns) are `planted`."""
+    n = len(planted)
+    causal = S * (S + 1) / 2
+    rows = []
+    for lam in grid["lam"]:
+        for tau in grid["tau"]:
+            for mu in grid["mu"]:
+                dp, do, vp, vc = (np.asarray(a) for a in capture(lam, tau, mu))
+                diags = [do[dp[m]:dp[m + 1]] for m in range(n)]
+                verts = [vc[vp[m]:vp[m + 1]] for m in range(n)]
+                tp = fp = fn = 0
+                for m in range(n):
+                    pd, pc = set(np.asarray(planted[m][0]).tolist()), set(np.asarray(planted[m][1]).tolist())
+                    kd, kc = set(diags[m].tolist()), set(verts[m].tolist())
+                    tp += len(pd & kd) + len(pc & kc)
+                    fp += len(kd - pd) + len(kc - pc)
+                    fn += len(pd - kd) + len(pc - kc)
+                dens = nnz_per_head(diags, verts, S) / causal
+                rows.append({"lam": lam, "tau": tau, "mu": mu,
+                             "diags_per_map": float(np.mean([len(x) for x in diags])),
+                             "cols_per_map": float(np.mean([len(x) for x in verts])),
+                             "recall": tp / max(tp + fn, 1), "precision": tp / max(tp + fp, 1),
+                             "density_at_S": float(dens.mean())})
+    return rows
+
+
+def run_capture_sweep(args):
+    """Time the library's capture over the (lambda, tau, mu) grid on synthetic averaged maps
+    and report what each setting keeps (one JSON line; the capture kernels are HBM-bound)."""
+    import torch
+
+    import structured_sparse_attention_b200 as ssa
+    n, L, S = SWEEP_WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    seed = inputs.SEED_BASE + 2
+    maps_h = inputs.averaged_maps(seed, n, L=L, n_samples=16)
+    planted = inputs.planted_map_patterns(seed, n, L)
+    maps = torch.from_numpy(maps_h).to(dev)
+    ws = torch.empty(max(ssa.load().sparse_pattern_capture_ws_bytes(n, L), 16), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = ssa.capture(maps, ws=ws, status=status)
+    times = []
+
+    def capture(lam, tau, mu):
+        for _ in range(args.warmup):
+            ssa.capture(maps, lam=lam, tau=tau, mu=mu, out=out, ws=ws, status=status)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            ssa.capture(maps, lam=lam, tau=tau, mu=mu, out=out, ws=ws, status=status, check=False)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / args.steps)
+        if int(status.item()) != 0:
+            raise RuntimeError(f"device status {int(status.item())}")
+        return [out[k].cpu().numpy() for k in ("diag_ptr", "diag_offsets", "vert_ptr", "vert_cols")]
+
+    rows = capture_sweep(capture, planted, S)
+    ms = float(np.mean(times))
+    hbm_gbs, _, _, peak_kind = load_peaks()
+    algo_bytes = n * 4 * L * (L + 1) // 2  # the causal half of every map, read once
+    line = {"metric": "stage-one sensitivity sweep: kept patterns, planted recall/precision, extended density",
+            "value": n / (ms / 1e3), "unit": "maps/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "n_maps": n, "L": L, "S": S, "grid": SWEEP_GRID},
+            "roofline": {"bound": "hbm", "achieved": algo_bytes / (ms / 1e3) / 1e9, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": algo_bytes / (ms / 1e3) / 1e9 / hbm_gbs, "traffic": None,
+                         "kernel": "capture (hits + select + pack)", "peak_source": peak_kind},
+            "sweep": rows, "e2e": None, "gpu_launches": 3 * args.steps * len(rows), "cpu_baseline": None}
+    print(json.dumps(line), flush=True)
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason sampling during the timed region."""
 
@@ -641,7 +729,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ssa", choices=["ssa", "reference"])
-    ap.add_argument("--workload", default="llama3-8b-layer-64k", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(MAPS_WORKLOADS))
+    ap.add_argument("--workload", default="llama3-8b-layer-64k", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(MAPS_WORKLOADS) + sorted(SWEEP_WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle attention work")
@@ -653,6 +741,11 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if args.workload in SWEEP_WORKLOADS:
+        if args.impl != "ssa" or args.gpus != 1:
+            ap.error("sweep workloads run the library on one GPU")
+        run_capture_sweep(args)
+        return
     if args.workload in MAPS_WORKLOADS:
         if args.impl != "ssa" or args.gpus != 1:
             ap.error("map workloads run the library on one GPU")
