@@ -67,7 +67,9 @@ def _setup(L):
                                  C.c_double, P, P]
     L.ora_nnz.argtypes = [C.c_int, P, P, P, P, C.c_int, P]
     L.ora_attn_maps.argtypes = [P, P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_double, P]
-    for name in ("ora_attn_maps", "ora_true_mask", "ora_gamma", "ora_select", "ora_capture", "ora_extend",
+    L.ora_attn_dense_case2.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int, P, P, P, P, P,
+                                       C.c_double, P, C.c_int, P, P]
+    for name in ("ora_attn_dense_case2", "ora_attn_maps", "ora_true_mask", "ora_gamma", "ora_select", "ora_capture", "ora_extend",
                  "ora_attn_rows", "ora_attn_dense", "ora_nnz"):
         getattr(L, name).restype = C.c_int
 
@@ -227,6 +229,24 @@ def attn_rows(q, k, v, ext, scale, rows, kv_map=None):
     LSE = np.zeros((Hq, len(rows)), np.float64)
     _check(lib().ora_attn_rows(_p(q), _p(k), _p(v), Hq, Hkv, S, d, _p(dp), _p(do), _p(vp), _p(vo),
                                _p(km), scale, len(rows), _p(rows), _p(O), _p(LSE)), "attn_rows")
+    return O, LSE
+
+
+def attn_dense_case2(q, k, v, ext, scale, true_masks, kv_map=None):
+    """Case-2 reading: the captured true mask of each head (uint8 [Hq, L, L]) verbatim in
+    the first L x L block, the kept patterns elsewhere; dense fp64 attention (S <= 8192)."""
+    q, k, v = (_c(a, np.uint16) for a in (q, k, v))
+    Hq, S, d = q.shape
+    Hkv = k.shape[0]
+    dp, do, vp, vo = (_c(a, np.int32) for a in ext)
+    tm = _c(true_masks, np.uint8)
+    if tm.ndim != 3 or tm.shape[0] != Hq or tm.shape[1] != tm.shape[2]:
+        raise ValueError("true_masks must be [Hq, L, L]")
+    km = None if kv_map is None else _c(kv_map, np.int32)
+    O = np.zeros((Hq, S, d), np.float64)
+    LSE = np.zeros((Hq, S), np.float64)
+    _check(lib().ora_attn_dense_case2(_p(q), _p(k), _p(v), Hq, Hkv, S, d, _p(dp), _p(do), _p(vp), _p(vo),
+                                      _p(km), scale, _p(tm), tm.shape[1], _p(O), _p(LSE)), "attn_dense_case2")
     return O, LSE
 
 

@@ -602,14 +602,18 @@ int ora_attn_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int H
 
 /* Dense-mask attention (small S): materialises the S x S boolean extended mask as the
  * union of every kept pattern's cells, then soft-maxes each row over its set cells in
- * ascending key order.  O [Hq][S][d], LSE [Hq][S]. */
-int ora_attn_dense(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int Hq, int Hkv, int S,
-                   int d, const int32_t *ext_diag_ptr, const int32_t *ext_diag_offsets,
-                   const int32_t *ext_vert_ptr, const int32_t *ext_vert_cols,
-                   const int32_t *kv_map, double scale, double *O, double *LSE) {
+ * ascending key order.  With `block` (uint8 [Hq][Lb][Lb], may be NULL) the first
+ * Lb x Lb cells of head h are replaced by block[h] (j <= i only): the Case-2 reading
+ * of the extended mask.  O [Hq][S][d], LSE [Hq][S]. */
+static int attn_dense_impl(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int Hq, int Hkv, int S,
+                           int d, const int32_t *ext_diag_ptr, const int32_t *ext_diag_offsets,
+                           const int32_t *ext_vert_ptr, const int32_t *ext_vert_cols,
+                           const int32_t *kv_map, double scale, const uint8_t *block, int Lb, double *O,
+                           double *LSE) {
     if (!Q || !K || !V || Hq <= 0 || Hkv <= 0 || S <= 0 || S > 8192 || d <= 0)
         return ORA_ERR_INVALID;
     if (!kv_map && Hq % Hkv != 0) return ORA_ERR_INVALID;
+    if (block && Lb <= 0) return ORA_ERR_INVALID;
     uint8_t *Mt = (uint8_t *)malloc((size_t)S * S);
     if (!Mt) return ORA_ERR_NOMEM;
     int err = ORA_OK;
@@ -623,6 +627,12 @@ int ora_attn_dense(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int 
             for (long i = D[k]; i < S; ++i) Mt[(size_t)i * S + (i - D[k])] = 1;
         for (int k = 0; k < nc; ++k)
             for (long i = C[k]; i < S; ++i) Mt[(size_t)i * S + C[k]] = 1;
+        if (block) {
+            const uint8_t *Bh = block + (size_t)h * Lb * Lb;
+            int lim = Lb < S ? Lb : S;
+            for (int i = 0; i < lim; ++i)
+                for (int j = 0; j <= i; ++j) Mt[(size_t)i * S + j] = Bh[(size_t)i * Lb + j] ? 1 : 0;
+        }
         int g = kv_head(h, Hq, Hkv, kv_map);
 #pragma omp parallel
         {
@@ -644,6 +654,28 @@ int ora_attn_dense(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int 
     }
     free(Mt);
     return err;
+}
+
+int ora_attn_dense(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int Hq, int Hkv, int S,
+                   int d, const int32_t *ext_diag_ptr, const int32_t *ext_diag_offsets,
+                   const int32_t *ext_vert_ptr, const int32_t *ext_vert_cols,
+                   const int32_t *kv_map, double scale, double *O, double *LSE) {
+    return attn_dense_impl(Q, K, V, Hq, Hkv, S, d, ext_diag_ptr, ext_diag_offsets, ext_vert_ptr,
+                           ext_vert_cols, kv_map, scale, NULL, 0, O, LSE);
+}
+
+/* Case-2 reading of the extended mask (DAM review page, Referee Report major comment 2:
+ * the patterns are pasted beyond the first L tokens): the captured L x L true mask of
+ * each head kept verbatim in the first L x L block, the union of the kept patterns
+ * everywhere else.  true_masks uint8 [Hq][L][L] (entries j > i ignored). */
+int ora_attn_dense_case2(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int Hq, int Hkv, int S,
+                         int d, const int32_t *ext_diag_ptr, const int32_t *ext_diag_offsets,
+                         const int32_t *ext_vert_ptr, const int32_t *ext_vert_cols,
+                         const int32_t *kv_map, double scale, const uint8_t *true_masks, int L, double *O,
+                         double *LSE) {
+    if (!true_masks) return ORA_ERR_INVALID;
+    return attn_dense_impl(Q, K, V, Hq, Hkv, S, d, ext_diag_ptr, ext_diag_offsets, ext_vert_ptr,
+                           ext_vert_cols, kv_map, scale, true_masks, L, O, LSE);
 }
 
 /* Number of retained (i, j) pairs of each head over the S x S extended mask, counted

@@ -1,0 +1,123 @@
+"""Pins of the oracle's Case-2 extended mask (CPU only).
+
+Case 2 reads the extension to S > L (DAM review page, Referee Report major comment 2:
+the patterns are pasted beyond the first L tokens) with the captured L x L true mask
+kept verbatim in the first block and the union of the kept patterns everywhere else.
+The routine is pinned by reductions to the already pinned dense routine and by the
+cases whose output is known outright.
+"""
+
+import numpy as np
+import pytest
+
+from structured_sparse_attention_b200 import inputs
+
+
+def _ext(ora, diags, verts, S):
+    dp, do = inputs.to_csr(diags)
+    vp, vo = inputs.to_csr(verts)
+    return ora.extend(dp, do, vp, vo, S)
+
+
+def _pattern_block(diags, verts, L):
+    """The patterns' own cells in the first L x L block, as a mask."""
+    out = []
+    i, j = np.meshgrid(np.arange(L), np.arange(L), indexing="ij")
+    for D, C in zip(diags, verts):
+        m = np.isin(i - j, D) | np.isin(j, C)
+        out.append((m & (j <= i)).astype(np.uint8))
+    return np.stack(out)
+
+
+def test_pattern_block_reduces_to_case_one(ora):
+    # a true mask equal to the patterns' cells gives the plain extended mask exactly
+    S, L, d, H = 300, 128, 16, 2
+    diags = [np.array([0, 3, 40]), np.array([1, 2])]
+    verts = [np.array([5, 130]), np.array([0, 200])]
+    ext = _ext(ora, diags, verts, S)
+    q, k, v = inputs.qkv(5, H, H, S, d)
+    o1, l1 = ora.attn_dense(q, k, v, ext, 0.25)
+    o2, l2 = ora.attn_dense_case2(q, k, v, ext, 0.25, _pattern_block(diags, verts, L))
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_rows_past_the_block_use_the_patterns_only(ora):
+    S, L, d = 260, 128, 8
+    diags, verts = [np.array([0, 7])], [np.array([3])]
+    ext = _ext(ora, diags, verts, S)
+    q, k, v = inputs.qkv(6, 1, 1, S, d)
+    rng = np.random.default_rng(1)
+    tm = (rng.random((1, L, L)) < 0.3).astype(np.uint8)
+    o1, l1 = ora.attn_dense(q, k, v, ext, 0.3)
+    o2, l2 = ora.attn_dense_case2(q, k, v, ext, 0.3, tm)
+    assert np.array_equal(o1[:, L:], o2[:, L:]) and np.array_equal(l1[:, L:], l2[:, L:])
+    assert not np.array_equal(o1[:, :L], o2[:, :L])  # the block itself did change
+
+
+def test_single_key_rows_copy_that_value(ora):
+    # one marked key j0 in row i, no patterns: O[i] = V[j0], LSE[i] = scale * q_i . k_j0
+    S, L, d = 128, 128, 8
+    ext = _ext(ora, [np.array([], np.int64)], [np.array([], np.int64)], S)
+    q, k, v = inputs.qkv(7, 1, 1, S, d)
+    tm = np.zeros((1, L, L), np.uint8)
+    picks = {10: 3, 50: 50, 127: 0}
+    for i, j0 in picks.items():
+        tm[0, i, j0] = 1
+    O, LSE = ora.attn_dense_case2(q, k, v, ext, 0.5, tm)
+    f = lambda a: inputs.f32_from_bf16_bits(a).astype(np.float64)
+    for i, j0 in picks.items():
+        np.testing.assert_array_equal(O[0, i], f(v[0, j0]))
+        assert LSE[0, i] == pytest.approx(0.5 * float(f(q[0, i]) @ f(k[0, j0])), abs=1e-12)
+    # rows with no marked key and no pattern: O = 0, LSE = -inf
+    assert (O[0, 11] == 0).all() and LSE[0, 11] == -np.inf
+
+
+def test_full_block_is_causal_attention(ora):
+    # every causal cell of the block marked, S = L: the same as the all-diagonals mask
+    S = L = 96
+    d = 16
+    q, k, v = inputs.qkv(8, 1, 1, S, d)
+    empty = _ext(ora, [np.array([], np.int64)], [np.array([], np.int64)], S)
+    full = _ext(ora, [np.arange(S)], [np.array([], np.int64)], S)
+    o1, l1 = ora.attn_dense(q, k, v, full, 0.25)
+    o2, l2 = ora.attn_dense_case2(q, k, v, empty, 0.25, np.ones((1, L, L), np.uint8))
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_entries_above_the_diagonal_are_ignored(ora):
+    S, L, d = 200, 128, 8
+    ext = _ext(ora, [np.array([0, 2])], [np.array([9])], S)
+    q, k, v = inputs.qkv(9, 1, 1, S, d)
+    rng = np.random.default_rng(2)
+    tm = (rng.random((1, L, L)) < 0.2).astype(np.uint8)
+    up = tm.copy()
+    up[0][np.triu_indices(L, 1)] = 1
+    a = ora.attn_dense_case2(q, k, v, ext, 0.2, tm)
+    b = ora.attn_dense_case2(q, k, v, ext, 0.2, up)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_captured_true_mask_feeds_the_block(ora):
+    # the block comes from stage one: the true mask of an averaged map
+    L, S, d = 128, 256, 16
+    maps = inputs.averaged_maps(12, 1, L=L, n_samples=3)
+    tm = ora.true_mask(maps[0]).astype(np.uint8)[None]
+    dp, do, vp, vc = ora.capture(maps)
+    ext = ora.extend(dp, do, vp, vc, S)
+    q, k, v = inputs.qkv(10, 1, 1, S, d)
+    O, LSE = ora.attn_dense_case2(q, k, v, ext, 0.25, tm)
+    assert np.isfinite(O).all()
+    # row 0 always marks its only key (a constant row counts as t = 1)
+    f = lambda a: inputs.f32_from_bf16_bits(a).astype(np.float64)
+    np.testing.assert_array_equal(O[0, 0], f(v[0, 0]))
+
+
+def test_block_replaces_the_patterns_there(ora):
+    # inside the block the true mask decides alone: a pattern cell it leaves out is dropped
+    S, L, d = 160, 128, 8
+    ext = _ext(ora, [np.array([0])], [np.array([], np.int64)], S)
+    q, k, v = inputs.qkv(11, 1, 1, S, d)
+    O, LSE = ora.attn_dense_case2(q, k, v, ext, 0.3, np.zeros((1, L, L), np.uint8))
+    assert (O[0, :L] == 0).all() and (LSE[0, :L] == -np.inf).all()
+    f = lambda a: inputs.f32_from_bf16_bits(a).astype(np.float64)
+    np.testing.assert_array_equal(O[0, L:], f(v[0, L:]))  # past the block: the diagonal r = 0
