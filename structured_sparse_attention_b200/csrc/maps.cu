@@ -22,9 +22,11 @@
 // (part h takes columns 32h..32h+31; thread il of a warpgroup owns row 128 rb + il,
 // TMEM lane il), so four warps per SM sub-partition share the MUFU and hide each
 // other's latencies; the parts' running max and sum are combined through shared memory
-// at the end of each sample, and part 0 keeps (m_b, 1 / l_b).  Warp 16 lane 0: TMA
-// producer of the Q block and K chunk of each tile.  Warp 17: tensor memory (two S
-// buffers of 128 columns) and lane 0 issues the MMAs.
+// at the end of each sample, and part 0 keeps (m_b, 1 / l_b); at d = 64 each part sends
+// its 32 columns of a finished chunk to the map with a TMA store from a swizzled staging
+// buffer.  Warp 16 lane 0: TMA producer of the Q block and K chunk of each tile.
+// Warp 17: tensor memory (four S buffers of 128 columns, so the MMAs run up to three
+// tiles ahead of the softmax) and lane 0 issues the MMAs.
 //
 // Every wait is bounded: on expiry the kernel records SSA_ERR_TIMEOUT, stops every role,
 // drains its copies and MMAs, frees tensor memory and returns.
