@@ -96,3 +96,18 @@ def test_product_path_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"(from|import)\s+oracle|libssa_oracle|ssa_oracle|\bora_\w+\(", txt), f
+
+
+def test_binding_rejects_host_tensors_before_any_call(lib):
+    # the binding marshals CUDA tensors only: host tensors fail loudly, nothing falls back
+    import torch
+
+    from structured_sparse_attention_b200 import binding
+    q = torch.zeros((1, 1, 128, 64), dtype=torch.bfloat16)
+    with pytest.raises(binding.SSAError) as e:
+        binding.attn_maps(q, q)
+    assert e.value.code == -1 and "CUDA" in str(e.value)
+    with pytest.raises(binding.SSAError):
+        binding.capture(torch.zeros((1, 16, 16), dtype=torch.float32))
+    with pytest.raises(binding.SSAError):
+        binding.extend(*(torch.zeros(2, dtype=torch.int32) for _ in range(4)), 64)
