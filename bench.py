@@ -1,9 +1,9 @@
 """Benchmark of the DAM structured-sparse-attention hot path on B200.
 
-One step = one pass of the whole path over one synthetic layer:
-  sparse_pattern_capture  (one layer's 32 averaged maps at L = 512)
-  sparse_pattern_extend   (fill pass: validate, extend to S, compile the tile plan)
-  sparse_attn_fwd         (stripe gather + tcgen05 attention forward)
+The timed step is the prefill call itself, sparse_attn_fwd (stripe gather + tcgen05
+attention forward) over one synthetic layer; `value` is its tokens/s.  The whole path
+(sparse_pattern_capture of the layer's 32 averaged maps at L = 512, the fill pass of
+sparse_pattern_extend, sparse_attn_fwd) is timed as well and reported under "path".
 The default workload is the LLaMA-3-8B-shaped layer at S = 65536 (32 Q / 8 KV heads,
 d = 128, per head 1024 contiguous diagonals at a random offset + 128 random columns).
 The sizing pass of sparse_pattern_extend (an allocation-size query) runs once at set-up.
@@ -82,27 +82,34 @@ def load_peaks():
 
 
 def profiled_traffic(workload):
-    """DRAM bytes per attention launch from the committed ncu summary of this workload,
-    if the attention sources are still the ones it was taken on (else None)."""
+    """DRAM bytes per attention launch from the ncu record of this workload
+    (profiles/sparse_attn_fwd_<workload>_dram.json), if the attention sources are still
+    the ones it was taken on (else None)."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"sparse_attn_fwd_{workload}_dram.md")
+    path = os.path.join(ROOT, "profiles", f"sparse_attn_fwd_{workload}_dram.json")
     if not os.path.exists(path):
         return None
-    fields = {}
-    for line in open(path):
-        if ":" in line and not line.startswith(("|", "#", " ")):
-            k, _, v = line.partition(":")
-            fields[k.strip()] = v.strip()
+    rec = json.load(open(path))
     csrc = os.path.join(ROOT, "structured_sparse_attention_b200", "csrc")
     h = hashlib.sha256()
     for f in ("attn_fwd.cu", "common.cuh"):
         h.update(open(os.path.join(csrc, f), "rb").read())
-    if fields.get("source_sha256_16") != h.hexdigest()[:16]:
+    if rec.get("source_sha256_16") != h.hexdigest()[:16]:
         return None
     try:
-        return float(fields["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
+        return float(rec["traffic_bytes_per_launch"])
+    except (KeyError, TypeError, ValueError):
         return None
+
+
+def attn_source_hash():
+    """First 16 hex digits of the sha256 of the attention sources (attn_fwd.cu, common.cuh)."""
+    import hashlib
+    csrc = os.path.join(ROOT, "structured_sparse_attention_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("attn_fwd.cu", "common.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def nnz_per_head(diags, verts, S):
@@ -120,6 +127,98 @@ def nnz_per_head(diags, verts, S):
             total -= int(shared)
         out.append(total)
     return np.array(out, np.int64)
+
+
+# Stage one at full size: the averaged maps of 16 layers x 32 heads at L = 512 (B = 16
+# samples averaged), captured with lambda = 0.5, tau = 0.3, mu = 0.8.
+CAPTURE_WORKLOADS = {
+    "capture-512maps-l512": (512, 512),  # maps, L
+}
+
+
+def run_capture(args):
+    """Time sparse_pattern_capture alone on one GPU: maps/s and the achieved HBM bandwidth
+    of the causal half of every map (the bytes the capture must read) against the measured
+    copy peak.  The maps (537 MB) exceed L2, and L2 is flushed between timed calls."""
+    import torch
+
+    import structured_sparse_attention_b200 as ssa
+    n, L = CAPTURE_WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    seed = inputs.SEED_BASE + 2
+    maps_h = inputs.averaged_maps(seed, n, L=L, n_samples=16)
+    h_maps = torch.from_numpy(maps_h).pin_memory()
+    maps = h_maps.to(dev)
+    ws = torch.empty(max(ssa.load().sparse_pattern_capture_ws_bytes(n, L), 16), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = ssa.capture(maps, ws=ws, status=status)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def call():
+        ssa.capture(maps, out=out, ws=ws, status=status, check=False)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0")
+    sampler.start()
+    time.sleep(0.3)
+    for e0, e1 in ev:
+        flush.fill_(1)  # evict the maps from L2 (not timed)
+        e0.record()
+        call()
+        e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())}")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    kept = int(out["diag_ptr"][-1].item()) + int(out["vert_ptr"][-1].item())
+    # end to end: the maps in from pinned host memory, the four lists back
+    outs_h = {k_: torch.empty(out[k_].shape, dtype=out[k_].dtype).pin_memory()
+              for k_ in ("diag_ptr", "diag_offsets", "vert_ptr", "vert_cols")}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(3, min(args.steps, 10))
+    e0.record()
+    for _ in range(e_steps):
+        maps.copy_(h_maps, non_blocking=True)
+        call()
+        for k_, t_ in outs_h.items():
+            t_.copy_(out[k_], non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1) / e_steps
+    algo_bytes = n * 4 * L * (L + 1) // 2  # the causal half of every map, read once
+    hbm_gbs, _, _, peak_kind = load_peaks()
+    achieved = algo_bytes / (ms / 1e3) / 1e9
+    line = {"metric": "stage-one pattern capture maps/s & achieved HBM GB/s vs roofline", "value": n / (ms / 1e3),
+            "unit": "maps/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "n_maps": n, "L": L, "lambda": 0.5, "tau": 0.3, "mu": 0.8,
+                       "eps": 1e-8, "kept_patterns": kept,
+                       "l2": "maps (%.0f MB) larger than L2, and L2 flushed between timed calls" % (n * L * L * 4 / 1e6)},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": achieved / hbm_gbs, "traffic": None, "peak_source": f"{peak_kind} (copy)",
+                         "kernel": "sparse_pattern_capture (hits + select + pack)",
+                         "algorithmic": {"bytes": algo_bytes, "what": "the causal half of every map, fp32"}},
+            "clocks": clocks,
+            "e2e": {"value": n / (e_ms / 1e3), "unit": "maps/s", "h2d_bytes_per_step": int(h_maps.numel() * 4),
+                    "d2h_bytes_per_step": int(sum(t_.numel() * 4 for t_ in outs_h.values())), "ms_per_step": e_ms},
+            "gpu_launches": LAUNCHES["capture"] * args.steps, "cpu_baseline": None}
+    if not args.no_cpu_baseline:
+        from oracle import oracle as ora
+        ora.build()
+        cores = len(os.sched_getaffinity(0))
+        n_cpu = min(n, max(16, cores))
+        t0 = time.perf_counter()
+        ora.capture(maps_h[:n_cpu])
+        cpu_s = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": n_cpu / cpu_s, "unit": "maps/s", "cores": cores, "kind": "oracle",
+                                "sample": f"the first {n_cpu} of the {n} maps, fp64 scalar oracle"}
+    print(json.dumps(line), flush=True)
 
 
 # Sensitivity of stage one to its free parameters (lambda, tau, mu): the referee's
@@ -287,8 +386,11 @@ def max_over_ranks(x: float, dist, device):
 # ------------------------------------------------------------------------------------
 
 def oracle_leg(workload, budget_s=15.0, maps=None):
-    """Time the oracle as it stands on a bounded sample of the workload.  Returns
-    (tokens/s extrapolated to the whole step, description dict)."""
+    """Time the oracle as it stands on a bounded sample of the workload: the attention
+    rows of randomly drawn query rows (all heads), grown until `budget_s` seconds of
+    work; tokens/s is extrapolated to all S rows.  The capture of the layer's maps and
+    the extension are timed in full and reported beside it.  Returns (tokens/s,
+    description dict)."""
     from oracle import oracle as ora
     Hq, Hkv, S, d, builder = WORKLOADS[workload]
     diags, verts = builder()
@@ -316,12 +418,14 @@ def oracle_leg(workload, budget_s=15.0, maps=None):
         t_rows += time.perf_counter() - t0
         done += len(rows)
         n_rows *= 2
-    t_step = t_cap + t_ext + t_rows * (S / done)
+    t_attn = t_rows * (S / done)  # extrapolated to all S rows
     desc = {"kind": "oracle", "cores": int(os.environ.get("OMP_NUM_THREADS", cores)),
-            "sample": f"capture of {CAPTURE_MAPS} maps at L={CAPTURE_L} in full ({t_cap:.2f} s), "
-                      f"extension in full, attention on {done} random query rows x {Hq} heads "
-                      f"({t_rows:.1f} s), extrapolated to S={S} rows"}
-    return S / t_step, desc
+            "extrapolated": True, "rows_timed": int(done), "seconds_timed": round(t_rows, 3),
+            "sample": f"attention on {done} random query rows x {Hq} heads ({t_rows:.1f} s of oracle work), "
+                      f"extrapolated to S={S} rows; capture of {CAPTURE_MAPS} maps at L={CAPTURE_L} "
+                      f"({t_cap:.2f} s) and the extension ({t_ext:.2f} s) timed in full, not in the value",
+            "path_tokens_per_s_extrapolated": S / (t_cap + t_ext + t_attn)}
+    return S / t_attn, desc
 
 
 # ------------------------------------------------------------------------------------
@@ -369,7 +473,12 @@ def run_gpu(args, rank, world, local, dist):
 
     ev = {n: [torch.cuda.Event(enable_timing=True) for _ in range(2)] for n in ("cap", "ext", "attn")}
 
-    def step(timed_stage=None):
+    def attn_step():
+        """The timed step: the prefill call (stripe gather + attention kernel)."""
+        ssa.attn_fwd(q, k, v, plan, out=O, lse=LSE, ws=attn_ws, status=status, check=False)
+
+    def path_step(timed_stage=None):
+        """The whole path: capture of the layer's maps, extension fill pass, attention."""
         if timed_stage:
             ev["cap"][0].record(stream)
         ssa.capture(maps, out=cap_out, ws=cap_ws, status=status, check=False)
@@ -380,17 +489,17 @@ def run_gpu(args, rank, world, local, dist):
         if timed_stage:
             ev["ext"][1].record(stream)
             ev["attn"][0].record(stream)
-        ssa.attn_fwd(q, k, v, plan, out=O, lse=LSE, ws=attn_ws, status=status, check=False)
+        attn_step()
         if timed_stage:
             ev["attn"][1].record(stream)
 
     for _ in range(args.warmup):
-        step()
+        path_step()
     torch.cuda.synchronize()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during warm-up")
 
-    # ---------------- device-timed region ----------------
+    # ---------------- device-timed region: K prefill calls ----------------
     stage_ms = {"cap": 0.0, "ext": 0.0, "attn": 0.0}
     props = torch.cuda.get_device_properties(dev)
     sampler = ClockSampler(f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0")
@@ -403,7 +512,7 @@ def run_gpu(args, rank, world, local, dist):
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for _ in range(args.steps):
-        step()
+        attn_step()
     t_end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -412,10 +521,20 @@ def run_gpu(args, rank, world, local, dist):
     ms_total = t_start.elapsed_time(t_end)
     ms_step = max_over_ranks(ms_total / args.steps, dist, dev)
 
-    # per-stage device times, averaged over a second pass of timed steps
+    # the whole path, K steps, then its per-stage device times over a second pass
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for _ in range(args.steps):
+        path_step()
+    p1.record(stream)
+    torch.cuda.synchronize()
+    path_ms = max_over_ranks(p0.elapsed_time(p1) / args.steps, dist, dev)
     reps = max(5, min(args.steps, 50))
     for _ in range(reps):
-        step(timed_stage=True)
+        path_step(timed_stage=True)
         torch.cuda.synchronize()
         for n in stage_ms:
             stage_ms[n] += ev[n][0].elapsed_time(ev[n][1]) / reps
@@ -436,7 +555,7 @@ def run_gpu(args, rank, world, local, dist):
             v.copy_(h_v, non_blocking=True)
             for dst, src in zip(lists, h_lists):
                 dst.copy_(src, non_blocking=True)
-            step()
+            path_step()
             h_O.copy_(O, non_blocking=True)
             h_L.copy_(LSE, non_blocking=True)
 
@@ -456,7 +575,9 @@ def run_gpu(args, rank, world, local, dist):
                sum(t.numel() * 4 for t in h_lists))
         d2h = h_O.numel() * 2 + h_L.numel() * 4
         e2e = {"value": world * S / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms}
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms,
+               "what": "the whole path through the public API per step: maps, pattern lists and Q/K/V in "
+                       "from pinned host memory, capture + extend + attention, O and LSE back"}
 
     # ---------------- dense reference point (context, not the target) ----------------
     dense = None
@@ -490,7 +611,7 @@ def run_gpu(args, rank, world, local, dist):
     causal_pairs = S * (S + 1) / 2
     density = float(nnz.mean() / causal_pairs)
     hbm_gbs, tf_burst, tf_sust, peak_kind = load_peaks()
-    attn_ms = max_over_ranks(stage_ms["attn"], dist, dev)
+    attn_ms = ms_step  # the timed step is the prefill call
     algo_bytes = (2 * Hq * S * d * 2) + (2 * Hkv * S * d * 2) + Hq * S * 4
     t_tensor = flops / (tf_burst * 1e12)
     t_hbm = algo_bytes / (hbm_gbs * 1e9)
@@ -528,16 +649,20 @@ def run_gpu(args, rank, world, local, dist):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": args.workload, "H_q": Hq, "H_kv": Hkv, "S": S, "d": d,
                    "density_of_causal": density, "nnz_per_head_mean": float(nnz.mean()),
-                   "capture": f"{CAPTURE_MAPS} maps x L={CAPTURE_L} per step", "batch": 1,
+                   "step": "one sparse_attn_fwd call (stripe gather + attention) over the layer",
+                   "path_capture": f"{CAPTURE_MAPS} maps x L={CAPTURE_L} per path step", "batch": 1,
                    "parallelism": f"replicas x{world}" if world > 1 else "single-gpu",
                    "l2": "inputs larger than L2 (Q+K+V+O %.2f GB)" % ((2 * Hq + 2 * Hkv) * S * d * 2 / 1e9)},
-        "stages_ms": {"capture": stage_ms["cap"], "extend_fill": stage_ms["ext"], "attn_fwd": attn_ms},
-        "attn_tokens_per_s": S / (attn_ms / 1e3),
+        "path": {"what": "capture of the layer's 32 maps + extend fill pass + attention, per step",
+                 "ms_per_step": path_ms, "tokens_per_s": world * S / (path_ms / 1e3),
+                 "stages_ms": {"capture": stage_ms["cap"], "extend_fill": stage_ms["ext"],
+                               "attn_fwd": stage_ms["attn"]},
+                 "gpu_launches_per_step": sum(LAUNCHES.values())},
         "effective_tflops": flops / (attn_ms / 1e3) / 1e12,
         "roofline": roof,
         "clocks": clocks,
         "e2e": e2e,
-        "gpu_launches": args.steps * sum(LAUNCHES.values()),
+        "gpu_launches": args.steps * LAUNCHES["attn"],
         "dense_reference": dense,
     }
     return line
@@ -729,7 +854,9 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ssa", choices=["ssa", "reference"])
-    ap.add_argument("--workload", default="llama3-8b-layer-64k", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(MAPS_WORKLOADS) + sorted(SWEEP_WORKLOADS))
+    ap.add_argument("--workload", default="llama3-8b-layer-64k",
+                    choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(MAPS_WORKLOADS)
+                    + sorted(SWEEP_WORKLOADS) + sorted(CAPTURE_WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle attention work")
@@ -741,6 +868,11 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if args.workload in CAPTURE_WORKLOADS:
+        if args.impl != "ssa" or args.gpus != 1:
+            ap.error("capture workloads run the library on one GPU")
+        run_capture(args)
+        return
     if args.workload in SWEEP_WORKLOADS:
         if args.impl != "ssa" or args.gpus != 1:
             ap.error("sweep workloads run the library on one GPU")
@@ -761,7 +893,7 @@ def main():
         if rank == 0:
             Hq, Hkv, S, d, _ = WORKLOADS[args.workload]
             t0 = time.perf_counter()
-            vals = []
+            vals, rows, secs = [], 0, 0.0
             desc = None
             maps = inputs.averaged_maps(inputs.SEED_BASE + 2, CAPTURE_MAPS, L=CAPTURE_L, n_samples=16)
             for i in range(args.warmup + args.steps):
@@ -769,13 +901,18 @@ def main():
                 v, desc = oracle_leg(args.workload, budget_s=budget, maps=maps)
                 if i >= args.warmup:
                     vals.append(v)
+                    rows += desc["rows_timed"]
+                    secs += desc["seconds_timed"]
             value = float(np.median(vals))
+            # Each step is a bounded sample of the layer (a few thousand query rows, not all
+            # S): ms_per_step is the extrapolated time of a whole layer, not a measured one.
             line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                     "steps": args.steps, "warmup": args.warmup, "ms_per_step": S / value * 1e3,
+                    "extrapolated": True, "rows_timed": rows, "seconds_timed": round(secs, 3),
                     "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                     "data": "synthetic", "config": {"workload": args.workload, "H_q": Hq, "H_kv": Hkv, "S": S,
-                                                    "d": d},
-                    "cpu_baseline": dict(desc, value=value, unit=UNIT),
+                                                    "d": d, "step": "one sparse-attention prefill of the layer"},
+                    "cpu_baseline": dict(desc, value=value, unit=UNIT, rows_timed=rows, seconds_timed=round(secs, 3)),
                     "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
                     "wall_s": time.perf_counter() - t0}
             print(json.dumps(line), flush=True)

@@ -25,25 +25,29 @@
 //                    each slot's Q tile at the slot's first step of the item
 //                    (each blocking role has a warp of its own: single-lane loops of one
 //                    warp would serialise on each other's waits)
-//     warps 9, 11    MMA issuers, one per slot (warp 9 allocates tensor memory).  For
-//                    merged step u, slot s issues PV_s of its tile at u-1, then QK_s(u).
-//                    S_s = Q_s K^T goes to TMEM, O_s += P_s V with P_s read from TMEM.
-//                    P_s is written over the first half of S_s, so a slot's QK^T always
-//                    follows the PV of its previous tile (tcgen05.mma operations of one
-//                    thread execute in issue order).  Two issuers keep the tensor pipe
-//                    fed while either one waits or commits; while one slot's softmax
-//                    works, the tensor core runs the other's MMAs.
+//     warps 9, 11    MMA issuers, one per slot (warp 9 allocates tensor memory).  Each
+//                    128-key tile is processed as two key regions, a (keys 0-63) and b
+//                    (keys 64-127), each with its own S-ready and P-ready barrier.  For
+//                    merged step u and region h, slot s issues PV of region h of its tile
+//                    at u-1 (P_h written over the first 32 columns of region h of S_s),
+//                    then QK^T of region h of the tile at u into the same 64 columns
+//                    (N = 64).  So while the softmax works on region b, the tensor core
+//                    runs region a's PV and the next tile's region-a QK^T: the softmax no
+//                    longer waits for the MMAs of its own tile.  The two issuers run
+//                    independently (an issue order between the slots made each wait for
+//                    the other slot's softmax).
 //     warps 0-3      softmax of slot 0 (query block 2p), one thread per query row
 //     warps 4-7      softmax of slot 1 (query block 2p+1)
-//                    tcgen05.ld S (128 columns), element mask from the plan (FULL
-//                    tiles skip it), online max/sum in fp32 (log2 domain, packed f32x2
-//                    arithmetic), P as bf16 into TMEM, lazy O rescale (only when the
-//                    max grows by > 2^8); epilogue O / l -> bf16 and LSE.  A slot's
-//                    epilogue runs after it has handed over the P of its first tile of
-//                    the next item: the tensor pipe gets that P without waiting for the
+//                    per region: tcgen05.ld S (64 columns), element mask from the plan
+//                    (FULL tiles skip it), online max/sum in fp32 (log2 domain, packed
+//                    f32x2 arithmetic), P as bf16 into TMEM, lazy O rescale (only when
+//                    the max grows by > 2^8); epilogue O / l -> bf16 and LSE.  A slot's
+//                    epilogue runs after it has handed over the P of region a of its
+//                    first tile of the next item: the tensor pipe gets that P without waiting for the
 //                    epilogue, and the first PV of the next item (which overwrites O_s)
 //                    waits on o_empty until the epilogue has read O_s.
-// Tensor memory (512 columns): S0 0..127, S1 128..255, O0 256.., O1 256+d...
+// Tensor memory (512 columns): S0 0..127, S1 128..255 (region a, then b), O0 256..,
+// O1 256+d...
 //
 // Every barrier is waited on with a counter of its own completions, and every wait
 // happens only after the previous completion of the same barrier was observed by the
@@ -84,10 +88,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if the ma
 // logits is computed by exp2_fma2 instead of the MUFU ex2, which alone would take as
 // long as the tile's MMAs.  Coefficients: degree-4 minimax fit of 2^f on [-1/2, 1/2]
 // (Remez exchange; printed by exp2_poly.py), relative error <= 2.7e-6 in fp32.
-#ifndef SSA_EMU_EVERY
-#define SSA_EMU_EVERY 0
-#endif
-constexpr int kEmuEvery = SSA_EMU_EVERY;  // 0: every exponential on the MUFU
+constexpr int kEmuEvery = 0;  // 0: every exponential on the MUFU
 __host__ __device__ constexpr bool emulated_pair(int k) {
     return kEmuEvery > 0 && (k % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1;
 }
@@ -139,13 +140,14 @@ struct Shared {
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[kMaxStages], k_empty[kMaxStages];
     uint64_t v_full[kMaxStages], v_empty[kMaxStages];
-    uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+    uint64_t s_full[2][2], p_full[2][2];  // per slot and key region (keys 0-63, 64-127 of a tile)
+    uint64_t pv_a[2];                      // PV of a tile's region a complete
+    uint64_t o_full[2], o_empty[2];
     uint64_t mma_drain, softmax_done;
     ItemDesc items[kRing];
     uint32_t kflags[kMaxStages];
     uint32_t tmem_base;
     int abort;
-    int turn;  // MMA issue order: bracket 2u + s (step u, slot s) may issue when turn == 2u + s
 };
 static_assert(sizeof(Shared) <= 1024, "barrier block too large");
 
@@ -247,14 +249,21 @@ __global__ void __launch_bounds__(256) stripe_gather_kernel(const uint16_t *__re
 // ---------------------------------------------------------------------------------
 
 // Work item idx -> descriptor of the pair of query blocks (2 pq, 2 pq + 1) of head h.
-// Items run from the last pair down (later blocks hold more tiles under causal
-// patterns) with the heads of one pair side by side, so heads of a KV group read the
-// same key tiles close together in time.
+// Items come in groups of G = H / H_kv consecutive heads (the heads that share one KV
+// head under the default map); within a group the pairs run from the last down (later
+// blocks hold more tiles under causal patterns) with the group's heads side by side.
+// The CTAs then work on one KV head at a time, so the band windows that consecutive
+// pairs of a head share are still in L2 when the later pair reads them.
 __device__ ItemDesc make_pair(const AttnParams &p, int idx) {
     ItemDesc d;
     const int npair = (p.nqb + 1) >> 1;
-    const int pq = npair - 1 - idx / p.H;
-    d.h = idx % p.H;
+    const int G = max(1, p.H / p.Hkv);
+    const int grp = idx / (npair * G);
+    const int h0 = grp * G;
+    const int gsz = min(G, p.H - h0);  // the last group may be short
+    const int rem = idx - grp * npair * G;
+    const int pq = npair - 1 - rem / gsz;
+    d.h = h0 + rem % gsz;
     d.g = kv_head(p, d.h);
     d.end = 0;
     const bool bad = d.g < 0 || d.g >= p.Hkv;
@@ -381,8 +390,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sh->q_full[s], 1);
             mbar_init(&sh->q_empty[s], 1);
-            mbar_init(&sh->s_full[s], 1);
-            mbar_init(&sh->p_full[s], kSlotThreads);
+            for (int h = 0; h < 2; ++h) {
+                mbar_init(&sh->s_full[s][h], 1);
+                mbar_init(&sh->p_full[s][h], kSlotThreads);
+            }
+            mbar_init(&sh->pv_a[s], 1);
             mbar_init(&sh->o_full[s], 1);
             mbar_init(&sh->o_empty[s], kSlotThreads);
         }
@@ -397,7 +409,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sh->mma_drain, 2);
         mbar_init(&sh->softmax_done, 2 * kSlotThreads);
         sh->abort = 0;
-        sh->turn = 0;
         fence_barrier_init();
     }
     if (warp == kWarpMma0) {
@@ -555,10 +566,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // issuing only its own slot's tcgen05.mma.  A tcgen05.mma blocks its thread while
         // the tensor pipe's short queue is full, so a single issuer leaves the pipe idle
         // whenever it does its waits and commits; with two, one slot's MMAs run while
-        // the other's issuer does its bookkeeping.  Per merged step u, slot s:
-        //   PV_s of its tile at u-1 (if any) | wait K_u | QK_s(u) (if s uses K_u)
-        // A slot's QK^T always follows the PV of its previous tile (P_s shares the S_s
-        // columns; tcgen05.mma of one thread execute in issue order).  Every PV is issued
+        // the other's issuer does its bookkeeping.  Per merged step u, slot s, region h:
+        //   PV_h of its tile at u-1 (if any) | (region a: wait K_u) | QK_h(u) (if s uses K_u)
+        // A region's QK^T always follows the PV of the same region of the previous tile
+        // (P_h shares the region's columns; tcgen05.mma of one thread execute in issue
+        // order).  After the PV of region a the issuer commits pv_a, which the softmax
+        // waits for only when it has to rescale O at region b.  Every PV is issued
         // at the step after its QK^T, so no V tile is held longer than one step.  Each
         // issuer releases every K and V stage once (a commit after its own MMAs on it,
         // else a plain arrival), so each stage's empty barrier takes two arrivals; the
@@ -569,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // producer never waits more than one phase behind.
         if (lane == 0) {
             const int s = (warp == kWarpMma1) ? 1 : 0;
-            constexpr uint32_t IDESC_QK = idesc_bf16(kBM, kBN, false);
+            constexpr uint32_t IDESC_QK = idesc_bf16(kBM, kBN / 2, false);  // one key region: N = 64
             constexpr uint32_t IDESC_PV = idesc_bf16(kBM, D, true);
             const uint32_t sQ = smem_u32(smem + C::OFF_Q + s * C::TILE_BYTES);
             const uint32_t tS = tmem + 128 * s, tO = tmem + C::COL_O + D * s;
@@ -583,82 +596,84 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ok && !mbar_wait_poll(bar, parity, lim, abort)) ok = false;
                 return ok;
             };
-            volatile int *turn = &sh->turn;
-            // the issue order of the single-issuer schedule: brackets (u, 0), (u, 1), (u+1, 0) ...
-            auto wait_turn = [&](int t) {
-                if (!ok) return false;
-                if (*turn == t) return true;
-                const uint64_t t0 = global_timer_ns();
-                while (*turn != t) {
-                    if (*abort || static_cast<int64_t>(global_timer_ns() - t0) >= lim) {
-                        ok = false;
-                        return false;
-                    }
-                }
-                return true;
-            };
             while (ok) {
-                // 1. every wait of this step's bracket, while the other slot's MMAs run
                 const int v = u - 1;
-                if (u >= 1 && !wait(&sh->v_full[v % C::NV], (v / C::NV) & 1)) break;
-                if (pend && !wait(&sh->p_full[s], pcnt & 1)) break;
-                // the first PV of an item overwrites O_s: the previous item's epilogue
-                // must have read it
-                if (pend && pfirst && ocnt >= 1 && !wait(&sh->o_empty[s], (ocnt - 1) & 1)) break;
-                if (!wait(&sh->k_full[u % C::NK], (u / C::NK) & 1)) break;
-                const uint32_t f = sh->kflags[u % C::NK];
-                const bool end = (f & kStepEnd) != 0;
-                const bool in = !end && (f & f_in(s));
-                if (in && (f & f_first(s)) && !wait(&sh->q_full[s], qcnt & 1)) break;
-                // 2. this slot's turn: PV_s of its tile at u-1, then QK_s(u)
-                if (!wait_turn(2 * u + s)) break;
-                tc_fence_after();
-                if (pend) {
-                    const uint32_t sV = smem_u32(smem + C::OFF_V + (v % C::NV) * C::TILE_BYTES);
+                uint32_t f = 0;
+                bool end = false, in = false;
+                // Two brackets per merged step, one per key region h (keys 64 h .. 64 h + 63):
+                // PV of region h of the slot's tile at u-1 (reads P_h, written over the first
+                // 32 columns of region h of S_s), then QK^T of region h of the tile at u into
+                // the same region.  Region a's MMAs run while the softmax works on region b.
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    // 1. every wait of this bracket, while the other slot's MMAs run
+                    if (h == 0 && u >= 1 && !wait(&sh->v_full[v % C::NV], (v / C::NV) & 1)) break;
+                    if (pend && !wait(&sh->p_full[s][h], pcnt & 1)) break;
+                    // the first PV of an item overwrites O_s: the previous item's epilogue
+                    // must have read it
+                    if (h == 0 && pend && pfirst && ocnt >= 1 && !wait(&sh->o_empty[s], (ocnt - 1) & 1)) break;
+                    if (h == 0) {
+                        if (!wait(&sh->k_full[u % C::NK], (u / C::NK) & 1)) break;
+                        f = sh->kflags[u % C::NK];
+                        end = (f & kStepEnd) != 0;
+                        in = !end && (f & f_in(s));
+                        if (in && (f & f_first(s)) && !wait(&sh->q_full[s], qcnt & 1)) break;
+                    }
+                    // 2. PV of region h of the slot's tile at u-1, then QK^T of region h of the
+                    // tile at u
+                    tc_fence_after();
+                    if (pend) {
+                        const uint32_t sV = smem_u32(smem + C::OFF_V + (v % C::NV) * C::TILE_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk) {
-                        // B = V tile, MN-major: 16 keys per step (2 x 8-row groups of 128 B)
-                        umma_ts(tO, tS + 8 * kk, sdesc(sV + kk * 2048, kBoxBytes, 1024), IDESC_PV,
-                                (!pfirst || kk > 0) ? 1u : 0u);
+                        for (int q = 0; q < 4; ++q) {
+                            // B = V tile, MN-major: 16 keys per step (2 x 8-row groups of 128 B)
+                            const int kk = 4 * h + q;
+                            umma_ts(tO, tS + 64 * h + 8 * q, sdesc(sV + kk * 2048, kBoxBytes, 1024), IDESC_PV,
+                                    (!pfirst || kk > 0) ? 1u : 0u);
+                        }
+                        if (h == 0) umma_commit(&sh->pv_a[s]);
+                    }
+                    if (in) {
+                        // key rows 64 h .. 64 h + 63 of the K tile start 8 KB into each box
+                        const uint32_t sK = smem_u32(smem + C::OFF_K + (u % C::NK) * C::TILE_BYTES) + 8192 * h;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            // A = Q, B = K rows, both K-major: 16 elements = 32 B per step
+                            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                            umma_ss(tS + 64 * h, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), IDESC_QK,
+                                    kk > 0 ? 1u : 0u);
+                        }
+                    }
+                    // 3. completions.  A release of V_(u-1) by a slot that did not read it comes
+                    // after its fill was observed above: the fill of step u-1 follows the
+                    // completion of the stage's previous phase, so the release lands in the
+                    // phase of step u-1 (never in the previous one, where it would stand in
+                    // for the other slot's PV still reading the stage, and never a phase
+                    // ahead of the producer, as for a no-op step that no slot reads).
+                    if (in) umma_commit(&sh->s_full[s][h]);
+                    if (h == 1) {
+                        if (pend) {
+                            if (plast) umma_commit(&sh->o_full[s]);  // O_s of the item complete
+                            umma_commit(&sh->v_empty[v % C::NV]);    // completes once the PVs have read V
+                            if (pfirst) ++ocnt;
+                            ++pcnt;
+                        } else if (u >= 1) {
+                            mbar_arrive(&sh->v_empty[v % C::NV]);
+                        }
+                        if (in) {
+                            if (f & f_last(s)) umma_commit(&sh->q_empty[s]);  // Q_s no longer read
+                            umma_commit(&sh->k_empty[u % C::NK]);
+                            if (f & f_first(s)) ++qcnt;
+                        } else if (!end) {
+                            mbar_arrive(&sh->k_empty[u % C::NK]);
+                        }
                     }
                 }
+                if (!ok || end) break;
+                pend = in;
                 if (in) {
-                    const uint32_t sK = smem_u32(smem + C::OFF_K + (u % C::NK) * C::TILE_BYTES);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        // A = Q, B = K tile, both K-major: 16 elements = 32 B per step
-                        const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                        umma_ss(tS, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), IDESC_QK,
-                                kk > 0 ? 1u : 0u);
-                    }
-                }
-                *turn = 2 * u + s + 1;
-                // 3. completions.  A release of V_(u-1) by a slot that did not read it comes
-                // after its fill was observed above: the fill of step u-1 follows the
-                // completion of the stage's previous phase, so the release lands in the
-                // phase of step u-1 (never in the previous one, where it would stand in
-                // for the other slot's PV still reading the stage, and never a phase
-                // ahead of the producer, as for a no-op step that no slot reads).
-                if (pend) {
-                    if (plast) umma_commit(&sh->o_full[s]);  // O_s of the item complete
-                    umma_commit(&sh->v_empty[v % C::NV]);    // completes once the PV has read V
-                    if (pfirst) ++ocnt;
-                    pend = false;
-                    ++pcnt;
-                } else if (u >= 1) {
-                    mbar_arrive(&sh->v_empty[v % C::NV]);
-                }
-                if (end) break;
-                if (in) {
-                    umma_commit(&sh->s_full[s]);
-                    if (f & f_last(s)) umma_commit(&sh->q_empty[s]);  // Q_s no longer read
-                    umma_commit(&sh->k_empty[u % C::NK]);
-                    if (f & f_first(s)) ++qcnt;
-                    pend = true;
                     pfirst = (f & f_first(s)) != 0;
                     plast = (f & f_last(s)) != 0;
-                } else {
-                    mbar_arrive(&sh->k_empty[u % C::NK]);
                 }
                 ++u;
             }
@@ -828,111 +843,117 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mhi = lk >= 128 ? ~0ull : (lk <= 64 ? 0ull : (1ull << (lk - 64)) - 1ull);
                 }
                 prefetch_l1(j + 1);
-                if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[s], tcnt & 1, lim, abort))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const bool do_mask = !__all_sync(0xffffffffu, full || (mlo & mhi) == ~0ull);
-                const uint32_t w[4] = {static_cast<uint32_t>(mlo), static_cast<uint32_t>(mlo >> 32),
-                                       static_cast<uint32_t>(mhi), static_cast<uint32_t>(mhi >> 32)};
-                uint32_t pk[64];
-                float psum = 0.0f;
-                auto load_s = [&](uint32_t(&r)[128]) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r + 32 * c);
-                    tmem_wait_ld();
-                };
-                // P = 2^(s * scale_log2 - mref) over this thread's row as packed bf16 pairs for
-                // the first 64 S columns; psum is the row's sum of P
-                auto exps = [&](const uint32_t(&r)[128], float mref) {
-                    const uint64_t nm2 = f2_pack(-mref, -mref);
-                    uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-                    for (int k = 0; k < 64; ++k) {
-                        float x0, x1;
-                        f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), sl2x2,
-                                         nm2),
-                                  x0, x1);
-                        float p0, p1;
-                        if (emulated_pair(k)) {
-                            exp2_fma2(x0, x1, p0, p1);
-                        } else {
-                            p0 = ex2_approx(x0);
-                            p1 = ex2_approx(x1);
-                        }
-                        acc[k & 3] = f2_add(acc[k & 3], f2_pack(p0, p1));
-                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                        pk[k] = *reinterpret_cast<const uint32_t *>(&pb);
+                // the tile's two key regions in order; each is a step of the online softmax
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[s][h], tcnt & 1, lim, abort))) {
+                        ok = false;
+                        break;
                     }
-                    float a0, a1, a2, a3, a4, a5, a6, a7;
-                    f2_unpack(acc[0], a0, a1);
-                    f2_unpack(acc[1], a2, a3);
-                    f2_unpack(acc[2], a4, a5);
-                    f2_unpack(acc[3], a6, a7);
-                    psum = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
-                };
-                // Mask the logits, take the tile's row max, then the lazy rescale rule: a new
-                // reference only when the row max grows by more than 2^8.
-                bool need_o = false;
-                float factor = 1.0f;
-                {
-                    uint32_t r[128];
-                    load_s(r);
+                    tc_fence_after();
+                    const uint64_t mk = h ? mhi : mlo;
+                    const bool do_mask = !__all_sync(0xffffffffu, full || mk == ~0ull);
+                    uint32_t r[64];
+                    tmem_ld32(tS + 64 * h, r);
+                    tmem_ld32(tS + 64 * h + 32, r + 32);
+                    tmem_wait_ld();
                     if (do_mask) {
+                        const uint32_t w0 = static_cast<uint32_t>(mk), w1 = static_cast<uint32_t>(mk >> 32);
 #pragma unroll
-                        for (int k = 0; k < 128; ++k)
-                            r[k] = (w[k >> 5] & (1u << (k & 31))) ? r[k] : kNegInf;
+                        for (int k = 0; k < 64; ++k)
+                            r[k] = (((k < 32 ? w0 : w1) >> (k & 31)) & 1u) ? r[k] : kNegInf;
                     }
                     float a[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q) a[q] = fmaxf(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
 #pragma unroll
-                    for (int k = 16; k < 128; k += 16) {
+                    for (int k = 16; k < 64; k += 16) {
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
                             a[q] = fmax3(a[q], __uint_as_float(r[k + 2 * q]), __uint_as_float(r[k + 2 * q + 1]));
                     }
                     const float tmax = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+                    // lazy rescale rule: a new reference only when the row max grows by more
+                    // than 2^8
                     const float m_new = fmaxf(m_run, tmax * sl2);  // -inf stays -inf
                     const bool grow = (m_new != -INFINITY) && (m_run == -INFINITY || m_new > m_run + kRescaleThreshold);
-                    need_o = grow && (m_run != -INFINITY);
+                    const bool need_o = grow && (m_run != -INFINITY);
+                    float factor = 1.0f;
                     if (grow) {
                         factor = (m_run == -INFINITY) ? 0.0f : ex2_approx(m_run - m_new);
                         l_run *= factor;
                         m_run = m_new;
                     }
-                    exps(r, (m_run == -INFINITY) ? 0.0f : m_run);
-                    l_run += psum;
-                }
-                tmem_st32(tS, pk);
-                tmem_st32(tS + 32, pk + 32);
-                if (__any_sync(0xffffffffu, need_o)) {
-                    // O_s holds every earlier tile: S_s of this tile was committed after the
-                    // PV of the previous tile, so that PV has completed.
-                    const float f = need_o ? factor : 1.0f;
+                    // P = 2^(s * scale_log2 - mref) over the region as packed bf16 pairs, over
+                    // the region's first 32 columns
+                    {
+                        const float mref = (m_run == -INFINITY) ? 0.0f : m_run;
+                        const uint64_t nm2 = f2_pack(-mref, -mref);
+                        uint64_t acc[4] = {0, 0, 0, 0};
+                        uint32_t pk[32];
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + 32 * c, o);
-                        tmem_wait_ld();
+                        for (int k = 0; k < 32; ++k) {
+                            float x0, x1;
+                            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), sl2x2, nm2),
+                                      x0, x1);
+                            float p0, p1;
+                            if (emulated_pair(k)) {
+                                exp2_fma2(x0, x1, p0, p1);
+                            } else {
+                                p0 = ex2_approx(x0);
+                                p1 = ex2_approx(x1);
+                            }
+                            acc[k & 3] = f2_add(acc[k & 3], f2_pack(p0, p1));
+                            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                            pk[k] = *reinterpret_cast<const uint32_t *>(&pb);
+                        }
+                        tmem_st32(tS + 64 * h, pk);
+                        float a0, a1, a2, a3, a4, a5, a6, a7;
+                        f2_unpack(acc[0], a0, a1);
+                        f2_unpack(acc[1], a2, a3);
+                        f2_unpack(acc[2], a4, a5);
+                        f2_unpack(acc[3], a6, a7);
+                        l_run += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+                    }
+                    if (__any_sync(0xffffffffu, need_o)) {
+                        // O_s must hold every PV taken against the old reference, and none
+                        // against the new one.  Region a: the PV of region b of the previous
+                        // tile precedes this tile's region-b QK^T (s_full[s][1]).  Region b:
+                        // the PV of this tile's region a (pv_a), whose P the warps have handed
+                        // over.  This tile's P of region h is not handed over yet.
+                        const bool okw = h == 0 ? mbar_wait(&sh->s_full[s][1], tcnt & 1, lim, abort)
+                                                : mbar_wait(&sh->pv_a[s], tcnt & 1, lim, abort);
+                        if (!__all_sync(0xffffffffu, okw)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const float f = need_o ? factor : 1.0f;
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
-                        tmem_st32(tO + 32 * c, o);
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(tO + 32 * c, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+                            tmem_st32(tO + 32 * c, o);
+                        }
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&sh->p_full[s][h]);
+                    // the previous item's epilogue, now that the tensor pipe has the P of
+                    // this item's first region (its first PV waits for O_s to be read)
+                    if (j == 0 && h == 0 && owed) {
+                        if (!epilogue()) {
+                            ok = false;
+                            break;
+                        }
+                        owed = false;
                     }
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&sh->p_full[s]);
+                if (!ok) break;
                 ++tcnt;
-                // the previous item's epilogue, now that the tensor pipe has this P
-                if (j == 0 && owed) {
-                    if (!epilogue()) {
-                        ok = false;
-                        break;
-                    }
-                    owed = false;
-                }
             }
             if (!ok) break;
             owed = true;

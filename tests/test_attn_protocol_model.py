@@ -1,12 +1,15 @@
 """Discrete-event model of the barrier protocol of sparse_attn_fwd_kernel (CPU only).
 
 The attention kernel's roles (scheduler + K producer, Q/V producer, one MMA issuer per
-slot with the turn token, one softmax per slot) are re-enacted here with the same loop
+slot, one softmax per slot) are re-enacted here with the same loop
 structure, barrier counts and phase counters, over random work items (items without
 tiles, items where one slot has no tile, windows shared by both slots, stripe tiles)
 and random latencies for the copies, the MMAs, the softmax and the epilogue.  The
 tensor pipe executes MMA groups in issue order; a commit completes when every group
-issued before it has completed.
+issued before it has completed.  Each key tile is processed as two key regions (keys
+0-63 and 64-127): per region an S-ready and a P-ready barrier, and one MMA bracket per
+region (PV of that region of the previous tile, QK^T of that region of this tile), so
+region a's MMAs run while the softmax works on region b.
 
 Checked in every run:
   * no deadlock: every role finishes;
@@ -18,7 +21,11 @@ Checked in every run:
     the slot's previous item has read O.  That epilogue runs after the softmax of the
     slot's first tile of the next item (it is deferred so the tensor pipe gets the next
     item's first P sooner); the issuer waits for it on o_empty;
-  * every tile the producers stage is consumed by exactly the slots that list it.
+  * every tile the producers stage is consumed by exactly the slots that list it;
+  * when the softmax rescales O (a row max that grows past the lazy threshold), O holds
+    exactly the PVs of the regions before the current one: region a waits for this
+    tile's region-b QK^T (which follows the previous tile's region-b PV), region b for
+    the PV of this tile's region a (pv_a).
 The model also shows that releasing a V stage without first observing its fill (the
 rule the issuers follow) breaks the phase invariant for runs of tile-less items.
 """
@@ -46,8 +53,10 @@ class Sim(Engine):
         self.k_empty = [B(f"k_empty{i}", 2) for i in range(NK)]
         self.v_full = [B(f"v_full{i}", 1) for i in range(NV)]
         self.v_empty = [B(f"v_empty{i}", 2) for i in range(NV)]
-        self.s_full = [B(f"s_full{s}", 1) for s in range(2)]
-        self.p_full = [B(f"p_full{s}", 1) for s in range(2)]
+        self.s_full = [[B(f"s_full{s}{h}", 1) for h in range(2)] for s in range(2)]
+        self.p_full = [[B(f"p_full{s}{h}", 1) for h in range(2)] for s in range(2)]
+        self.pv_a = [B(f"pv_a{s}", 1) for s in range(2)]
+        self.pv_done = [[], []]  # per slot: completion time of the PV of each region, in order
         self.o_full = [B(f"o_full{s}", 1) for s in range(2)]
         self.o_empty = [B(f"o_empty{s}", 1) for s in range(2)]
         self.ring = [None] * RING
@@ -189,55 +198,62 @@ def mma_issuer(sim, s):
     ptile = None
     while True:
         v = u - 1
-        if u >= 1 and not (sim.release_without_fill and not pend):
-            yield ("wait", sim.v_full[v % NV], v // NV)
-        if pend:
-            yield ("wait", sim.p_full[s], pcnt)
-            if pfirst and ocnt >= 1:
-                yield ("wait", sim.o_empty[s], ocnt - 1)
-        yield ("wait", sim.k_full[u % NK], u // NK)
-        tile, fl, end = sim.kflags[u % NK]
-        inn = (not end) and s in fl
-        if inn and fl[s][0]:
-            yield ("wait", sim.q_full[s], qcnt)
-        yield ("turn", 2 * u + s)
-        if pend:
-            if pfirst:
-                if sim.first_pv[s] > sim.epi_done[s]:
-                    raise ProtocolError(f"slot {s}: first PV of an item before the epilogue read O")
-                sim.first_pv[s] += 1
-                ocnt += 1
-            if sim.v_content[v % NV] != ptile:
-                raise ProtocolError(f"slot {s}: PV reads {sim.v_content[v % NV]}, wants {ptile}")
-            sim.mma(512, [f"V{v % NV}"])
-        if inn:
-            if sim.k_content[u % NK] != tile:
-                raise ProtocolError(f"slot {s}: QK reads {sim.k_content[u % NK]}, wants {tile}")
-            sim.consumed.append((s, tile))
-            sim.mma(512, [f"K{u % NK}", f"Q{s}"])
-        sim.pass_turn(2 * u + s + 1)
-        if pend:
-            if plast:
-                sim.commit(sim.o_full[s])
-            sim.commit(sim.v_empty[v % NV])
-            pend = False
-            pcnt += 1
-        elif u >= 1:
-            sim.v_empty[v % NV].arrive()
+        tile, fl, end, inn = None, {}, False, False
+        for h in range(2):
+            if h == 0 and u >= 1 and not (sim.release_without_fill and not pend):
+                yield ("wait", sim.v_full[v % NV], v // NV)
+            if pend:
+                yield ("wait", sim.p_full[s][h], pcnt)
+                if h == 0 and pfirst and ocnt >= 1:
+                    yield ("wait", sim.o_empty[s], ocnt - 1)
+            if h == 0:
+                yield ("wait", sim.k_full[u % NK], u // NK)
+                tile, fl, end = sim.kflags[u % NK]
+                inn = (not end) and s in fl
+                if inn and fl[s][0]:
+                    yield ("wait", sim.q_full[s], qcnt)
+            if pend:
+                if h == 0 and pfirst:
+                    if sim.first_pv[s] > sim.epi_done[s]:
+                        raise ProtocolError(f"slot {s}: first PV of an item before the epilogue read O")
+                    sim.first_pv[s] += 1
+                    ocnt += 1
+                if sim.v_content[v % NV] != ptile:
+                    raise ProtocolError(f"slot {s}: PV reads {sim.v_content[v % NV]}, wants {ptile}")
+                sim.pv_done[s].append(sim.mma(256, [f"V{v % NV}"]))
+                if h == 0:
+                    sim.commit(sim.pv_a[s])
+            if inn:
+                if sim.k_content[u % NK] != tile:
+                    raise ProtocolError(f"slot {s}: QK reads {sim.k_content[u % NK]}, wants {tile}")
+                if h == 0:
+                    sim.consumed.append((s, tile))
+                sim.mma(400, [f"K{u % NK}", f"Q{s}"])
+            if inn:
+                sim.commit(sim.s_full[s][h])
+            if h == 1:
+                if pend:
+                    if plast:
+                        sim.commit(sim.o_full[s])
+                    sim.commit(sim.v_empty[v % NV])
+                    pcnt += 1
+                elif u >= 1:
+                    sim.v_empty[v % NV].arrive()
+                if inn:
+                    if fl[s][1]:
+                        sim.commit(sim.q_empty[s])
+                    sim.commit(sim.k_empty[u % NK])
+                    if fl[s][0]:
+                        qcnt += 1
+                elif not end:
+                    sim.k_empty[u % NK].arrive()
+            yield ("delay", sim.rng.randint(1, 50))
         if end:
             return
+        pend = inn
         if inn:
-            sim.commit(sim.s_full[s])
-            if fl[s][1]:
-                sim.commit(sim.q_empty[s])
-            sim.commit(sim.k_empty[u % NK])
-            if fl[s][0]:
-                qcnt += 1
-            pend, pfirst, plast, ptile = True, fl[s][0], fl[s][1], tile
-        else:
-            sim.k_empty[u % NK].arrive()
+            pfirst, plast, ptile = fl[s][0], fl[s][1], tile
         u += 1
-        yield ("delay", sim.rng.randint(1, 50))
 
 
 def softmax(sim, s):
@@ -265,13 +281,26 @@ def softmax(sim, s):
         if n == 0:
             continue
         for j in range(n):
-            yield ("wait", sim.s_full[s], tcnt)
-            yield ("delay", sim.rng.randint(800, 3000))
-            sim.p_full[s].arrive()
+            for h in range(2):
+                yield ("wait", sim.s_full[s][h], tcnt)
+                yield ("delay", sim.rng.randint(400, 1500))
+                if j > 0 and sim.rng.random() < 0.2:
+                    # O rescale: O must hold exactly the PVs of the regions before this one
+                    if h == 0:
+                        yield ("wait", sim.s_full[s][1], tcnt)
+                    else:
+                        yield ("wait", sim.pv_a[s], tcnt)
+                    region = 2 * tcnt + h
+                    done = sim.pv_done[s]
+                    if len(done) != region or (done and done[-1] > sim.t):
+                        raise ProtocolError(f"slot {s}: O rescaled at region {region} with "
+                                            f"{len(done)} PVs issued")
+                    yield ("delay", sim.rng.randint(100, 400))
+                sim.p_full[s][h].arrive()
+                if j == 0 and h == 0 and owed:
+                    yield from epilogue()
+                    owed = False
             tcnt += 1
-            if j == 0 and owed:
-                yield from epilogue()
-                owed = False
         owed = True
     if owed:
         yield from epilogue()
