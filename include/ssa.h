@@ -146,7 +146,10 @@ SSA_API int sparse_pattern_capture(const float *maps, int n_maps, int L, double 
  *     fixed size are rejected with SSA_ERR_CAPACITY before any device work
  *     (L = 512 allows up to 1023 maps).
  *   - The first call on each device looks up the array's device address with that
- *     device current; make that first call before any stream capture begins.
+ *     device current and keeps it for the life of the process; make that first call
+ *     before any stream capture begins.  A device reset (cudaDeviceReset, or anything
+ *     else that tears down the primary context) invalidates the kept address: do not
+ *     call this entry point again in a process that has reset the device.
  *   - Every call shares the one array per device and clears what must start at zero
  *     itself; calls that overlap on the GPU (different streams or host threads) race
  *     on it and must be serialised by the caller.

@@ -50,6 +50,9 @@ P = C.c_void_p
 
 def _setup(L):
     L.ora_true_mask.argtypes = [P, C.c_int, C.c_double, C.c_double, C.c_double, P]
+    L.ora_true_mask_ex.argtypes = [P, C.c_int, C.c_double, C.c_double, C.c_double, C.c_int, P]
+    L.ora_capture_ex.argtypes = [P, C.c_int, C.c_int, C.c_double, C.c_double, C.c_double, C.c_double,
+                                 C.c_int, P, P, P, P]
     L.ora_gamma.argtypes = [P, C.c_int, P, P]
     L.ora_select.argtypes = [P, P, C.c_int, C.c_double, P, P, P, P]
     L.ora_capture.argtypes = [P, C.c_int, C.c_int, C.c_double, C.c_double, C.c_double, C.c_double,
@@ -69,7 +72,7 @@ def _setup(L):
     L.ora_attn_maps.argtypes = [P, P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_double, P]
     L.ora_attn_dense_case2.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int, P, P, P, P, P,
                                        C.c_double, P, C.c_int, P, P]
-    for name in ("ora_attn_dense_case2", "ora_attn_maps", "ora_true_mask", "ora_gamma", "ora_select", "ora_capture", "ora_extend",
+    for name in ("ora_true_mask_ex", "ora_capture_ex", "ora_attn_dense_case2", "ora_attn_maps", "ora_true_mask", "ora_gamma", "ora_select", "ora_capture", "ora_extend",
                  "ora_attn_rows", "ora_attn_dense", "ora_nnz"):
         getattr(L, name).restype = C.c_int
 
@@ -104,12 +107,20 @@ def attn_maps(q, k, scale):
     return out
 
 
-def true_mask(amap, lam=0.5, eps=1e-8, tau=0.3):
-    """Binary true mask uint8 [L, L] of one averaged map (row min-max of Box-Cox, t >= tau)."""
+SCALINGS = {"row": 0, "map": 1}
+
+
+def true_mask(amap, lam=0.5, eps=1e-8, tau=0.3, scaling="row"):
+    """Binary true mask uint8 [L, L] of one averaged map: min-max of the Box-Cox output
+    over each row's causal entries (scaling="row") or over the whole map's causal
+    entries (scaling="map"), then t >= tau."""
     amap = _c(amap, np.float32)
     Ln = amap.shape[0]
     M = np.zeros((Ln, Ln), np.uint8)
-    _check(lib().ora_true_mask(_p(amap), Ln, lam, eps, tau, _p(M)), "true_mask")
+    if scaling == "row":
+        _check(lib().ora_true_mask(_p(amap), Ln, lam, eps, tau, _p(M)), "true_mask")
+    else:
+        _check(lib().ora_true_mask_ex(_p(amap), Ln, lam, eps, tau, SCALINGS[scaling], _p(M)), "true_mask")
     return M
 
 
@@ -135,16 +146,21 @@ def select(gd, gv, mu=0.8):
     return do[:nd[0]].copy(), vo[:nv[0]].copy()
 
 
-def capture(maps, lam=0.5, tau=0.3, mu=0.8, eps=1e-8):
-    """Whole stage one over maps [n, L, L]; returns CSR (diag_ptr, diag_offsets, vert_ptr, vert_cols)."""
+def capture(maps, lam=0.5, tau=0.3, mu=0.8, eps=1e-8, scaling="row"):
+    """Whole stage one over maps [n, L, L]; returns CSR (diag_ptr, diag_offsets, vert_ptr, vert_cols).
+    `scaling` is the reading of the Box-Cox output's scaling before tau ("row" or "map")."""
     maps = _c(maps, np.float32)
     n, Ln, _ = maps.shape
     dp = np.zeros(n + 1, np.int32)
     do = np.zeros(n * Ln + 1, np.int32)
     vp = np.zeros(n + 1, np.int32)
     vo = np.zeros(n * Ln + 1, np.int32)
-    _check(lib().ora_capture(_p(maps), n, Ln, lam, tau, mu, eps, _p(dp), _p(do), _p(vp), _p(vo)),
-           "capture")
+    if scaling == "row":
+        _check(lib().ora_capture(_p(maps), n, Ln, lam, tau, mu, eps, _p(dp), _p(do), _p(vp), _p(vo)),
+               "capture")
+    else:
+        _check(lib().ora_capture_ex(_p(maps), n, Ln, lam, tau, mu, eps, SCALINGS[scaling], _p(dp), _p(do),
+                                    _p(vp), _p(vo)), "capture")
     return dp, do[:dp[-1]].copy(), vp, vo[:vp[-1]].copy()
 
 

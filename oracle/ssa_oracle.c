@@ -62,11 +62,23 @@ static double box_cox(double v, double lambda, double eps) {
     return (pow(z, lambda) - 1.0) / lambda;
 }
 
-/* True mask of one L x L averaged attention map (row-major float32).
- * Row i uses its causal entries j <= i: Box-Cox each, scale the row to [0,1] by its
- * own min and max, and set M[i][j] = (t >= tau).  Entries j > i are 0. */
-int ora_true_mask(const float *map, int L, double lambda, double eps, double tau, uint8_t *M) {
-    if (!map || !M || L <= 0) return ORA_ERR_INVALID;
+/* True mask of one L x L averaged attention map (row-major float32), with the Box-Cox
+ * output scaled to [0,1] before the threshold (the page does not say how; two readings):
+ *   scaling 0 (per row): row i uses the min and max of its own causal entries j <= i;
+ *   scaling 1 (per map): every row uses the min and max over all causal entries of the
+ *                        map.
+ * Then M[i][j] = (t >= tau) for j <= i, where t = (bc(x) - bc(min)) / (bc(max) - bc(min))
+ * and t = 1 when max == min.  Entries j > i are 0. */
+int ora_true_mask_ex(const float *map, int L, double lambda, double eps, double tau, int scaling,
+                     uint8_t *M) {
+    if (!map || !M || L <= 0 || (scaling != 0 && scaling != 1)) return ORA_ERR_INVALID;
+    double map_mn = INFINITY, map_mx = -INFINITY;
+    for (int i = 0; i < L; ++i)
+        for (int j = 0; j <= i; ++j) {
+            double x = (double)map[(size_t)i * L + j];
+            if (x < map_mn) map_mn = x;
+            if (x > map_mx) map_mx = x;
+        }
     for (int i = 0; i < L; ++i) {
         const float *row = map + (size_t)i * L;
         double mn = INFINITY, mx = -INFINITY;
@@ -74,6 +86,10 @@ int ora_true_mask(const float *map, int L, double lambda, double eps, double tau
             double x = (double)row[j];
             if (x < mn) mn = x;
             if (x > mx) mx = x;
+        }
+        if (scaling == 1) {
+            mn = map_mn;
+            mx = map_mx;
         }
         double ylo = box_cox(mn, lambda, eps);
         double yhi = box_cox(mx, lambda, eps);
@@ -92,6 +108,11 @@ int ora_true_mask(const float *map, int L, double lambda, double eps, double tau
         }
     }
     return ORA_OK;
+}
+
+/* The per-row reading (scaling 0). */
+int ora_true_mask(const float *map, int L, double lambda, double eps, double tau, uint8_t *M) {
+    return ora_true_mask_ex(map, L, lambda, eps, tau, 0, M);
 }
 
 /* gamma_k = sum_{i,j} M[i][j] P_k[i][j] / sum_{i,j} P_k[i][j], with the sums taken over
@@ -131,12 +152,13 @@ int ora_select(const double *gamma_diag, const double *gamma_vert, int L, double
     return ORA_OK;
 }
 
-/* Whole stage one over n_maps maps [n_maps][L][L]; outputs are CSR lists per map with
- * capacity n_maps*L each (diag_ptr / vert_ptr have n_maps+1 entries). */
-int ora_capture(const float *maps, int n_maps, int L, double lambda, double tau, double mu,
-                double eps, int32_t *diag_ptr, int32_t *diag_offsets, int32_t *vert_ptr,
-                int32_t *vert_cols) {
-    if (!maps || n_maps < 0 || L <= 0) return ORA_ERR_INVALID;
+/* Whole stage one over n_maps maps [n_maps][L][L] with the given scaling (see
+ * ora_true_mask_ex); outputs are CSR lists per map with capacity n_maps*L each
+ * (diag_ptr / vert_ptr have n_maps+1 entries). */
+int ora_capture_ex(const float *maps, int n_maps, int L, double lambda, double tau, double mu,
+                   double eps, int scaling, int32_t *diag_ptr, int32_t *diag_offsets,
+                   int32_t *vert_ptr, int32_t *vert_cols) {
+    if (!maps || n_maps < 0 || L <= 0 || (scaling != 0 && scaling != 1)) return ORA_ERR_INVALID;
     int32_t *tmp_d = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_maps * L + 4);
     int32_t *tmp_v = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_maps * L + 4);
     int32_t *cnt_d = (int32_t *)calloc((size_t)n_maps + 1, sizeof(int32_t));
@@ -152,7 +174,7 @@ int ora_capture(const float *maps, int n_maps, int L, double lambda, double tau,
 #pragma omp for schedule(dynamic, 1)
             for (int m = 0; m < n_maps; ++m) {
                 if (!M || !gd || !gv) continue;
-                ora_true_mask(maps + (size_t)m * L * L, L, lambda, eps, tau, M);
+                ora_true_mask_ex(maps + (size_t)m * L * L, L, lambda, eps, tau, scaling, M);
                 ora_gamma(M, L, gd, gv);
                 ora_select(gd, gv, L, mu, tmp_d + (size_t)m * L, &cnt_d[m], tmp_v + (size_t)m * L,
                            &cnt_v[m]);
@@ -178,6 +200,14 @@ int ora_capture(const float *maps, int n_maps, int L, double lambda, double tau,
     free(cnt_d);
     free(cnt_v);
     return err;
+}
+
+/* The per-row reading (scaling 0). */
+int ora_capture(const float *maps, int n_maps, int L, double lambda, double tau, double mu,
+                double eps, int32_t *diag_ptr, int32_t *diag_offsets, int32_t *vert_ptr,
+                int32_t *vert_cols) {
+    return ora_capture_ex(maps, n_maps, L, lambda, tau, mu, eps, 0, diag_ptr, diag_offsets, vert_ptr,
+                          vert_cols);
 }
 
 /* ----------------------------------------------------------------------------------

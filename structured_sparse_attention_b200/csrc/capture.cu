@@ -27,7 +27,6 @@ namespace {
 
 constexpr int kCaptureThreads = 256;
 constexpr int kCaptureWarps = kCaptureThreads / 32;
-constexpr int kRowChunks = 8;  // CTAs per map; rows interleaved across them
 
 struct CaptureParams {
     const float *maps;
@@ -45,6 +44,7 @@ struct CaptureParams {
     int32_t *vert_ptr;
     int32_t *vert_cols;
     int32_t *status;
+    int row_chunks;  // CTAs per map of the hits kernel; rows interleaved across them
 };
 
 __device__ __forceinline__ double box_cox_rn(double x, double eps, double lambda, bool half) {
@@ -120,12 +120,12 @@ __device__ uint32_t find_cut(uint32_t u0, uint32_t u1, float mn, float mx, doubl
 }
 
 template <int MAXK>
-__global__ void __launch_bounds__(kCaptureThreads)
+__global__ void __launch_bounds__(kCaptureThreads, MAXK <= 16 ? 3 : 1)
     capture_hits_kernel(CaptureParams p) {
     extern __shared__ int32_t s_hist[];  // [2][L]: diagonal hits, column hits
     const int L = p.L;
-    const int m = blockIdx.x / kRowChunks;
-    const int chunk = blockIdx.x % kRowChunks;
+    const int m = blockIdx.x / p.row_chunks;
+    const int chunk = blockIdx.x % p.row_chunks;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int k = threadIdx.x; k < 2 * L; k += kCaptureThreads) s_hist[k] = 0;
     __syncthreads();
@@ -133,25 +133,36 @@ __global__ void __launch_bounds__(kCaptureThreads)
     const bool half = (p.lambda == 0.5);
     const float *map = p.maps + static_cast<size_t>(m) * L * L;
     bool bad = false;
-    for (int i = chunk + kRowChunks * warp; i < L; i += kRowChunks * kCaptureWarps) {
+    // Rows are software-pipelined: the loads of the warp's next row are issued before the
+    // current row's cut point is searched, so each warp keeps a row in flight while it
+    // computes (the search is a chain of dependent fp64 steps).
+    auto load_row = [&](int i, float (&x)[MAXK]) {
         const float *row = map + static_cast<size_t>(i) * L;
+#pragma unroll
+        for (int k = 0; k < MAXK; ++k) {
+            const int j = lane + 32 * k;
+            x[k] = (i < L && j <= i) ? __ldg(row + j) : 0.0f;
+        }
+    };
+    const int stride = p.row_chunks * kCaptureWarps;
+    int i = chunk + p.row_chunks * warp;
+    float xc[MAXK], xn[MAXK];
+    load_row(i, xc);
+    for (; i < L; i += stride) {
+        load_row(i + stride, xn);
         const int n = i + 1;
-        uint32_t xb[MAXK];
         float mn = __int_as_float(0x7f800000), mx = 0.0f;
 #pragma unroll
         for (int k = 0; k < MAXK; ++k) {
             const int j = lane + 32 * k;
-            uint32_t b = 0;
             if (j < n) {
-                float x = __ldg(row + j);
+                float x = xc[k];
                 if (!(x >= 0.0f) || x == __int_as_float(0x7f800000)) bad = true;
-                b = __float_as_uint(x);
-                if (b == 0x80000000u) b = 0;  // -0 counts as +0
-                float xv = __uint_as_float(b);
-                mn = fminf(mn, xv);
-                mx = fmaxf(mx, xv);
+                if (__float_as_uint(x) == 0x80000000u) x = 0.0f;  // -0 counts as +0
+                xc[k] = x;
+                mn = fminf(mn, x);
+                mx = fmaxf(mx, x);
             }
-            xb[k] = b;
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -165,14 +176,18 @@ __global__ void __launch_bounds__(kCaptureThreads)
         } else {
             cut = find_cut(u0, u1, mn, mx, p.eps, p.lambda, half, p.tau);
         }
+        // for non-negative floats the order of the values is the order of their bits, so
+        // x >= x* is the comparison of the bit patterns (a cut of 0xffffffff keeps none)
 #pragma unroll
         for (int k = 0; k < MAXK; ++k) {
             const int j = lane + 32 * k;
-            if (j < n && xb[k] >= cut) {
+            if (j < n && __float_as_uint(xc[k]) >= cut) {
                 atomicAdd(&s_hist[i - j], 1);
                 atomicAdd(&s_hist[L + j], 1);
             }
         }
+#pragma unroll
+        for (int k = 0; k < MAXK; ++k) xc[k] = xn[k];
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) report(p.status, SSA_ERR_INVALID);
     __syncthreads();
@@ -181,6 +196,19 @@ __global__ void __launch_bounds__(kCaptureThreads)
         const int v = s_hist[k];
         if (v) atomicAdd(hits + k, v);
     }
+}
+
+// Multiprocessors of the current device (cached per device).
+int sm_count_capture() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
 }
 
 // Ordered compaction of {x in [0, L) : keep(x)} by the whole block.
@@ -332,7 +360,14 @@ extern "C" int sparse_pattern_capture(const float *maps, int n_maps, int L, doub
 
     SSA_CUDA_TRY(cudaMemsetAsync(p.hits, 0, static_cast<size_t>(n_maps) * 2 * L * sizeof(int32_t), s));
     const size_t smem = 2 * static_cast<size_t>(L) * sizeof(int32_t);
-    const unsigned grid = static_cast<unsigned>(n_maps) * kRowChunks;
+    // Enough CTAs to fill the GPU a few times over even for a few maps (each warp then
+    // takes fewer rows), at most one row per warp.
+    int chunks = 8;
+    while (chunks < 64 && static_cast<long long>(n_maps) * chunks < 4LL * sm_count_capture() &&
+           chunks * 2 * kCaptureWarps <= L)
+        chunks *= 2;
+    p.row_chunks = chunks;
+    const unsigned grid = static_cast<unsigned>(n_maps) * chunks;
     if (L <= 512) {
         capture_hits_kernel<16><<<grid, kCaptureThreads, smem, s>>>(p);
     } else {
@@ -359,12 +394,15 @@ extern "C" int sparse_pattern_capture(const float *maps, int n_maps, int L, doub
 #include <mutex>
 
 namespace ssa {
-namespace {
 
 constexpr size_t kNoAllocScratchBytes = SSA_CAPTURE_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
-__device__ __align__(256) int32_t g_capture_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
+// The scratch itself: a file-scope static device array (internal linkage).
+static __device__ __align__(256) int32_t g_capture_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
 
 std::mutex g_scratch_mutex;
 void *g_scratch_addr[kMaxDevices] = {};

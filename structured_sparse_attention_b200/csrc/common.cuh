@@ -162,40 +162,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-#ifndef SSA_POLL_MODE
-#define SSA_POLL_MODE 0
-#endif
-// Bounded wait that only polls with the non-blocking test (never suspends the thread).
-__device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, int64_t limit_ns,
-                                               volatile int *abort) {
-    if (mbar_test(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
-#pragma unroll 1
-        for (int k = 0; k < 16; ++k) {
-            if (mbar_test(bar, parity)) return true;
-#if SSA_POLL_MODE == 2
-            __nanosleep(20);
-#endif
-        }
-        if (abort && *abort) return false;
-        if (static_cast<int64_t>(global_timer_ns() - t0) >= limit_ns) return false;
-    }
-}
-
 // Bounded wait for a thread that issues tcgen05.mma.  mbarrier.try_wait in a thread with
 // MMAs in flight costs about the drain time of those operations (several hundred cycles)
 // even when the phase has already completed, which would leave the tensor pipe idle at
 // every wait; a test_wait costs a few cycles.  So test first; a phase that is not yet
-// complete is then waited for by sleeping in try_wait (or by polling).
+// complete is then waited for by sleeping in try_wait.
 __device__ __forceinline__ bool mbar_wait_poll(uint64_t *bar, uint32_t parity, int64_t limit_ns,
                                                volatile int *abort) {
     if (mbar_test(bar, parity)) return true;
-#if SSA_POLL_MODE == 0
     return mbar_wait(bar, parity, limit_ns, abort);
-#else
-    return mbar_wait_spin(bar, parity, limit_ns, abort);
-#endif
 }
 
 // Named-barrier AND reduction over `count` threads (whole warps) of barrier `id`;

@@ -163,3 +163,55 @@ def test_boxcox_eps_row(ora):
     for c in fx["eps_cases"]:
         M = ora.true_mask(amap, lam=0.5, eps=c["eps"], tau=0.3)
         assert M[L - 1].tolist() == c["M"], c
+
+
+@pytest.mark.parametrize("case", json.load(open(os.path.join(GOLDEN, "scaling_cases.json")))["cases"],
+                         ids=lambda c: f"l{c['lambda']}-t{c['tau']}-{c['scaling']}")
+def test_scaling_readings_and_general_lambda_fixture(ora, case):
+    # hand-derived masks (exact binary fractions) for the per-row and per-map readings
+    # of the scaling before tau, at lambda 1/2, 1 and a general lambda (2, through pow)
+    fx = json.load(open(os.path.join(GOLDEN, "scaling_cases.json")))
+    amap = np.array(fx["map"], np.float32)
+    M = ora.true_mask(amap, lam=case["lambda"], eps=0.0, tau=case["tau"], scaling=case["scaling"])
+    assert [M[i, :i + 1].tolist() for i in range(len(amap))] == case["M"]
+    assert not np.triu(M, 1).any()
+
+
+def test_per_map_equals_per_row_when_every_row_spans_the_map(ora):
+    # every row holds the map's minimum and maximum, so the two readings coincide
+    g = np.random.default_rng(3)
+    L = 48
+    amap = np.tril(g.uniform(0.1, 0.9, size=(L, L))).astype(np.float32)
+    amap[0, 0] = 1.0
+    for i in range(1, L):
+        amap[i, 0] = 0.0
+        amap[i, i] = 1.0
+    for lam in (0.5, 1.0, 1.7):
+        for tau in (0.2, 0.5):
+            np.testing.assert_array_equal(ora.true_mask(amap, lam=lam, tau=tau),
+                                          ora.true_mask(amap, lam=lam, tau=tau, scaling="map"))
+
+
+def test_per_map_scaling_invariants(ora):
+    maps = inputs.averaged_maps(12, 3, L=96, n_samples=4)
+    L = 96
+    # tau = 0 keeps every candidate; raising tau never adds a pattern
+    dp, do, vp, vo = ora.capture(maps, tau=0.0, scaling="map")
+    assert np.all(np.diff(dp) == L) and np.all(np.diff(vp) == L)
+    prev = None
+    for tau in (0.001, 0.01, 0.05, 0.2):
+        cur = ora.capture(maps, tau=tau, mu=0.5, scaling="map")
+        if prev is not None:
+            for a, b in ((0, 1), (2, 3)):
+                for m in range(len(maps)):
+                    assert set(cur[b][cur[a][m]:cur[a][m + 1]].tolist()) <= \
+                        set(prev[b][prev[a][m]:prev[a][m + 1]].tolist())
+        prev = cur
+    # one global threshold per map: a cell is set iff its value's transform clears it,
+    # so within a map the set cells are exactly the entries at or above one cut value
+    for m in maps:
+        M = ora.true_mask(m, tau=0.05, scaling="map")
+        cells = np.tril(np.ones((L, L), bool))
+        on, off = m[cells & (M == 1)], m[cells & (M == 0)]
+        if on.size and off.size:
+            assert on.min() > off.max()

@@ -6,9 +6,10 @@ must not call cudaMalloc/cudaFree after start-up (they can synchronise the devic
 stall other streams) cannot let the library allocate either.  This entry point keeps
 its scratch in a fixed device array inside the library instead of a caller workspace.
 
-The test calls it through the C ABI and checks that two calls in a row give exactly
-the kept lists of the regular entry point (lists are integers: bit-exact), and that a
-size beyond the fixed scratch is rejected.  It must pass alone in a fresh process and
+The test calls it through the C ABI and checks that calls in a row (the second keeping
+fewer patterns than the first from the same number of maps) give exactly the kept lists
+of the oracle and of the regular entry point (lists are integers: bit-exact), and that
+a size beyond the fixed scratch is rejected.  It must pass alone in a fresh process and
 after the rest of the suite, so it creates everything it needs itself.
 """
 
@@ -60,20 +61,30 @@ def _regular(ssa, maps_dev, **kw):
     return dp, out["diag_offsets"].cpu().numpy()[:dp[-1]], vp, out["vert_cols"].cpu().numpy()[:vp[-1]]
 
 
-def test_noalloc_capture_matches_regular_on_two_calls():
+def test_noalloc_capture_matches_oracle_and_regular_on_calls_in_a_row():
+    from oracle import oracle as ora
+    ora.build()
     ssa, lib = _lib()
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
-    # call 1: a model's worth of maps at L = 512; call 2: a different size and inputs,
-    # so the second call must not see anything the first left in the scratch
-    a = torch.from_numpy(inputs.averaged_maps(inputs.SEED_BASE + 2, 64, L=512, n_samples=4)).to(dev)
-    b = torch.from_numpy(inputs.averaged_maps(991, 40, L=300, n_samples=3)).to(dev)
-    for maps, kw in ((a, {}), (b, dict(tau=0.25, mu=0.7))):
+    # call 1: a model's worth of maps at L = 512; call 2: the same maps with stricter
+    # thresholds, so it keeps fewer patterns per map with the same map count (staging
+    # or counts left by call 1 must not leak into its lists); call 3: another size
+    a_h = inputs.averaged_maps(inputs.SEED_BASE + 2, 64, L=512, n_samples=4)
+    b_h = inputs.averaged_maps(991, 40, L=300, n_samples=3)
+    a, b = torch.from_numpy(a_h).to(dev), torch.from_numpy(b_h).to(dev)
+    calls = ((a, a_h, {}), (a, a_h, dict(tau=0.5, mu=0.97)), (b, b_h, dict(tau=0.25, mu=0.7)))
+    kept = []
+    for maps, maps_h, kw in calls:
         got = _noalloc(lib, maps, **kw)
-        want = _regular(ssa, maps, **kw)
-        for x, y, name in zip(got, want, ("diag_ptr", "diag_offsets", "vert_ptr", "vert_cols")):
+        want = ora.capture(maps_h, **kw)
+        regular = _regular(ssa, maps, **kw)
+        for x, y, z, name in zip(got, want, regular, ("diag_ptr", "diag_offsets", "vert_ptr", "vert_cols")):
             np.testing.assert_array_equal(x, y, err_msg=name)
+            np.testing.assert_array_equal(x, z, err_msg=name)
         assert got[0][-1] > 0 and got[2][-1] > 0
+        kept.append(int(got[0][-1]) + int(got[2][-1]))
+    assert kept[1] < kept[0], kept  # the second call keeps fewer patterns than the first
 
 
 def test_noalloc_rejects_sizes_beyond_the_scratch():
