@@ -105,14 +105,17 @@ SSA_API size_t sparse_pattern_capture_ws_bytes(int n_maps, int L);
  *   M[i][j] = t_j >= tau
  * then gamma_diag[r] = #{i >= r : M[i][i-r]} / (L - r), gamma_vert[c] =
  * #{i >= c : M[i][c]} / (L - c), both in fp64, and r (resp. c) is kept iff
- * gamma >= mu.  Every threshold decision is made with correctly rounded fp64
- * arithmetic in the stated order, so the kept lists are exactly reproducible.
+ * gamma >= mu.  At lambda 0.5 and 1 every threshold decision is made with correctly
+ * rounded fp64 arithmetic in the stated order, so the kept lists are exactly
+ * reproducible.  Other lambdas (0 = log) go through fp64 pow / log, which are not
+ * correctly rounded: an entry whose t lies within a few units in the last place of
+ * tau may be decided differently by another implementation.
  *
  *   maps         device, float32 [n_maps][L][L] row-major, already averaged over the
  *                calibration batches; causal entries must be finite and >= 0
  *                (entries j > i are ignored)
  *   n_maps       >= 1;  L in [1, 1024]
- *   lambda       0.5 or 1.0 (else SSA_ERR_UNSUPPORTED); tau, mu in fp64; eps >= 0
+ *   lambda       in [0, 64] (else SSA_ERR_INVALID); tau, mu in fp64; eps >= 0
  *   diag_ptr     device int32 [n_maps + 1]   CSR row pointers of the kept diagonals
  *   diag_offsets device int32 [n_maps * L]   kept r, ascending within each map
  *   vert_ptr     device int32 [n_maps + 1]
@@ -125,6 +128,29 @@ SSA_API int sparse_pattern_capture(const float *maps, int n_maps, int L, double 
                            double mu, double eps, int32_t *diag_ptr, int32_t *diag_offsets,
                            int32_t *vert_ptr, int32_t *vert_cols, void *ws, size_t ws_bytes,
                            int32_t *dev_status, void *stream);
+
+/* Scalings of the Box-Cox output to [0, 1] before tau (the page leaves it unstated). */
+#define SSA_SCALE_ROW 0 /* min and max over each row's causal entries (the default reading) */
+#define SSA_SCALE_MAP 1 /* min and max over all causal entries of the map */
+
+/*
+ * sparse_pattern_capture_ex -- sparse_pattern_capture with the two optional readings
+ * and outputs of stage one:
+ *   scaling    SSA_SCALE_ROW (as sparse_pattern_capture) or SSA_SCALE_MAP: every row
+ *              of a map uses the map's min and max (a constant map has t = 1); this
+ *              reading reads the maps twice (a min/max pass, then the decisions)
+ *   true_mask  null, or device uint32 [n_maps][L][ceil(L/32)], 4-byte aligned: the
+ *              binary true mask M itself, bit (j % 32) of word j / 32 of row i set iff
+ *              j <= i and M[i][j] (the input of the Case-2 extension,
+ *              sparse_pattern_extend_case2)
+ * All other arguments, the workspace and the errors are those of
+ * sparse_pattern_capture; a scaling other than the two is SSA_ERR_INVALID.
+ */
+SSA_API int sparse_pattern_capture_ex(const float *maps, int n_maps, int L, double lambda, double tau,
+                                      double mu, double eps, int scaling, int32_t *diag_ptr,
+                                      int32_t *diag_offsets, int32_t *vert_ptr, int32_t *vert_cols,
+                                      uint32_t *true_mask, void *ws, size_t ws_bytes,
+                                      int32_t *dev_status, void *stream);
 
 /* Size of the fixed device scratch of sparse_pattern_capture_noalloc (8 MiB). */
 #define SSA_CAPTURE_NOALLOC_SCRATCH_BYTES (8u << 20)
@@ -172,6 +198,7 @@ typedef struct ssa_plan_sizes {
     int32_t n_vert;    /* total extended columns over all heads */
     int32_t max_vert;  /* max over heads of the extended column count */
     int64_t n_tiles;   /* total listed band tiles */
+    int32_t bitmap_slots; /* Case-2 plans: element-bitmap slots per head (0 otherwise) */
 } ssa_plan_sizes;
 
 /*
@@ -213,6 +240,9 @@ typedef struct ssa_plan {
     uint64_t *tile_cmask;
     uint32_t *tile_flags;
     int32_t *stripe_cnt;
+    /* Case-2 plans only (sparse_pattern_extend_case2; zero / NULL otherwise): */
+    int32_t bitmap_slots; /* from ssa_plan_sizes */
+    uint64_t *tile_bits;  /* [n_heads * bitmap_slots][128][2] (uint64), 16-byte aligned */
 } ssa_plan;
 
 /* Workspace bytes of either pass of sparse_pattern_extend (about 4 * n_heads * S for
@@ -243,6 +273,37 @@ SSA_API int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr, const in
                           const int32_t *vert_ptr, const int32_t *vert_cols, int S,
                           ssa_plan_sizes *sizes, const ssa_plan *plan, void *ws, size_t ws_bytes,
                           int32_t *dev_status, void *stream);
+
+/*
+ * sparse_pattern_extend_case2 -- the Case-2 reading of the extension (DAM review page,
+ * Referee Report major comment 2: the patterns are pasted beyond the first L tokens):
+ * the captured L x L true mask of each head is kept verbatim in the first block, the
+ * union of the kept patterns everywhere else.  Cell (i, j), j <= i < S, is retained iff
+ *   i < L:  bit j of row i of true_mask[h]     (the patterns play no part there)
+ *   i >= L: i - j is a kept diagonal or j a kept column (as sparse_pattern_extend).
+ * The paper has no tile plan; this is the library's layout: every query block holding
+ * a row below min(L, S) is covered by element-bitmap tiles, one per key block kb = 0..qb
+ * (key0 = 128 kb), listed when any of its cells is set, with tile_flags bit 1 (BITMAP),
+ * the bitmap's slot h * bitmap_slots + qb (qb + 1) / 2 + kb in tile_dmask word 0, and
+ * no stripe tiles (stripe_cnt 0); plan->tile_bits[slot][il][w] holds the cells of row il,
+ * key column jl at bit jl % 64 of word jl / 64.  The other query blocks have the plan of
+ * sparse_pattern_extend.
+ *
+ *   true_mask  device uint32 [n_heads][L][ceil(L/32)], 4-byte aligned, bit j % 32 of
+ *              word j / 32 of row i = M[i][j] (sparse_pattern_capture_ex writes it;
+ *              bits above the diagonal are ignored)
+ *   L          capture length, [1, 1024]
+ * Everything else as sparse_pattern_extend; the sizing pass also sets
+ * sizes->bitmap_slots, and the fill pass needs plan->bitmap_slots equal to it and
+ * plan->tile_bits (16-byte aligned) of n_heads * bitmap_slots * 128 * 2 uint64.
+ * sparse_attn_fwd takes the plan as it is; sparse_attn_decode rejects it
+ * (SSA_ERR_UNSUPPORTED: decoding follows the first reading only).
+ */
+SSA_API int sparse_pattern_extend_case2(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offsets,
+                                        const int32_t *vert_ptr, const int32_t *vert_cols,
+                                        const uint32_t *true_mask, int L, int S, ssa_plan_sizes *sizes,
+                                        const ssa_plan *plan, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                        void *stream);
 
 /* ------------------------------------------------------------------------------ */
 /* Attention forward                                                               */

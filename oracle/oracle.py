@@ -278,3 +278,82 @@ def attn_dense(q, k, v, ext, scale, kv_map=None):
     _check(lib().ora_attn_dense(_p(q), _p(k), _p(v), Hq, Hkv, S, d, _p(dp), _p(do), _p(vp), _p(vo),
                                 _p(km), scale, _p(O), _p(LSE)), "attn_dense")
     return O, LSE
+
+
+def case2_bitmap_slots(L, S):
+    """Bitmap slots per head of a Case-2 plan: one per (query block qb, key block kb <= qb)
+    over the query blocks that hold a row below min(L, S)."""
+    nL = (min(L, S) + TILE - 1) // TILE
+    return nL, nL * (nL + 1) // 2
+
+
+def plan_case2(ext, S, true_masks, routine="brute"):
+    """Tile plan of the Case-2 extended mask (the L x L true mask of each head verbatim in
+    the first block, the kept patterns elsewhere; DAM review page, Referee Report major
+    comment 2), brute force from the definition.
+
+    Query blocks holding a row below min(L, S) are covered by element-bitmap tiles: key
+    windows at 128 kb for kb = 0..qb, listed when any cell is set, flag 2, the bitmap's
+    slot (head h, block qb, key block kb -> h * slots + qb (qb + 1) / 2 + kb) in dmask word
+    0, and no stripe tiles (stripe_cnt 0).  A cell (i, j) of such a tile is set iff
+    i < S, j <= i and: i < L and true_masks[h][i][j]; or i >= L and i - j is a kept
+    diagonal or j a kept column.  The other blocks keep the plain plan.  Returns the plan
+    dict with "tile_bits" uint64 [H * slots, 128, 2] (bit jl of word jl / 64 of row il)."""
+    dp, do, vp, vo = (_c(a, np.int32) for a in ext)
+    H = len(dp) - 1
+    tm = np.ascontiguousarray(true_masks).astype(bool)
+    L = tm.shape[1]
+    base = plan(ext, S, routine)
+    nqb = base["nqb"]
+    nL, slots = case2_bitmap_slots(L, S)
+    bits = np.zeros((H * slots, TILE, 2), np.uint64)
+    ptr, key0, dmask, cmask, flags = [0], [], [], [], []
+    stripe = base["stripe_cnt"].copy()
+    jl = np.arange(TILE)
+    for h in range(H):
+        D = set(do[dp[h]:dp[h + 1]].tolist())
+        Cs = set(vo[vp[h]:vp[h + 1]].tolist())
+        for qb in range(nqb):
+            it = h * nqb + qb
+            if qb < nL:
+                stripe[it] = 0
+                for kb in range(qb + 1):
+                    cell = np.zeros((TILE, TILE), bool)
+                    for il in range(TILE):
+                        i = TILE * qb + il
+                        if i >= S:
+                            break
+                        for c in range(TILE):
+                            j = TILE * kb + c
+                            if j > i:
+                                break
+                            if i < L:
+                                cell[il, c] = tm[h, i, j]
+                            else:
+                                cell[il, c] = (i - j) in D or j in Cs
+                    if not cell.any():
+                        continue
+                    slot = h * slots + qb * (qb + 1) // 2 + kb
+                    for il in range(TILE):
+                        for w in range(2):
+                            v = 0
+                            for b in range(64):
+                                if cell[il, 64 * w + b]:
+                                    v |= 1 << b
+                            bits[slot, il, w] = np.uint64(v)
+                    key0.append(TILE * kb)
+                    dmask.append([slot, 0, 0, 0])
+                    cmask.append([0, 0])
+                    flags.append(2)
+            else:
+                a, b = base["tile_ptr"][it], base["tile_ptr"][it + 1]
+                key0.extend(base["tile_key0"][a:b].tolist())
+                dmask.extend(base["tile_dmask"][a:b].tolist())
+                cmask.extend(base["tile_cmask"][a:b].tolist())
+                flags.extend(base["tile_flags"][a:b].tolist())
+            ptr.append(len(key0))
+    n = len(key0)
+    return dict(tile_ptr=np.array(ptr, np.int32), tile_key0=np.array(key0, np.int32).reshape(n),
+                tile_dmask=np.array(dmask, np.uint64).reshape(n, 4), tile_cmask=np.array(cmask, np.uint64).reshape(n, 2),
+                tile_flags=np.array(flags, np.uint32).reshape(n), stripe_cnt=stripe, n_tiles=n, nqb=nqb,
+                tile_bits=bits, bitmap_slots=slots)

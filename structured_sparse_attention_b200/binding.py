@@ -25,7 +25,8 @@ ERRORS = {-1: "SSA_ERR_INVALID", -2: "SSA_ERR_UNSUPPORTED", -3: "SSA_ERR_CAPACIT
 BLOCK = 128
 
 #: Every symbol include/ssa.h declares.
-EXPORTS = ("sparse_attn_maps", "sparse_pattern_capture_ws_bytes", "sparse_pattern_capture", "sparse_pattern_capture_noalloc",
+EXPORTS = ("sparse_attn_maps", "sparse_pattern_capture_ws_bytes", "sparse_pattern_capture", "sparse_pattern_capture_ex",
+           "sparse_pattern_capture_noalloc", "sparse_pattern_extend_case2",
            "sparse_pattern_extend_ws_bytes", "sparse_pattern_extend",
            "sparse_attn_fwd_ws_bytes", "sparse_attn_fwd",
            "sparse_attn_decode_ws_bytes", "sparse_attn_decode",
@@ -41,7 +42,7 @@ class SSAError(RuntimeError):
 class PlanSizes(C.Structure):
     _fields_ = [("n_heads", C.c_int32), ("S", C.c_int32), ("nqb", C.c_int32),
                 ("n_diag", C.c_int32), ("n_vert", C.c_int32), ("max_vert", C.c_int32),
-                ("n_tiles", C.c_int64)]
+                ("n_tiles", C.c_int64), ("bitmap_slots", C.c_int32)]
 
 
 class PlanStruct(C.Structure):
@@ -50,7 +51,8 @@ class PlanStruct(C.Structure):
                 ("ext_diag_ptr", C.c_void_p), ("ext_diag_offsets", C.c_void_p),
                 ("ext_vert_ptr", C.c_void_p), ("ext_vert_cols", C.c_void_p),
                 ("tile_ptr", C.c_void_p), ("tile_key0", C.c_void_p), ("tile_dmask", C.c_void_p),
-                ("tile_cmask", C.c_void_p), ("tile_flags", C.c_void_p), ("stripe_cnt", C.c_void_p)]
+                ("tile_cmask", C.c_void_p), ("tile_flags", C.c_void_p), ("stripe_cnt", C.c_void_p),
+                ("bitmap_slots", C.c_int32), ("tile_bits", C.c_void_p)]
 
 
 _lib = None
@@ -70,6 +72,11 @@ def load():
         lib.sparse_pattern_capture_ws_bytes.restype = SZ
         lib.sparse_pattern_capture.argtypes = [V, I, I, D, D, D, D, V, V, V, V, V, SZ, V, V]
         lib.sparse_pattern_capture.restype = I
+        lib.sparse_pattern_capture_ex.argtypes = [V, I, I, D, D, D, D, I, V, V, V, V, V, V, SZ, V, V]
+        lib.sparse_pattern_capture_ex.restype = I
+        lib.sparse_pattern_extend_case2.argtypes = [I, V, V, V, V, V, I, I, C.POINTER(PlanSizes),
+                                                    C.POINTER(PlanStruct), V, SZ, V, V]
+        lib.sparse_pattern_extend_case2.restype = I
         lib.sparse_pattern_extend_ws_bytes.argtypes = [I, I]
         lib.sparse_pattern_extend_ws_bytes.restype = SZ
         lib.sparse_pattern_extend.argtypes = [I, V, V, V, V, I, C.POINTER(PlanSizes),
@@ -156,10 +163,15 @@ def attn_maps(q: torch.Tensor, k: torch.Tensor, scale: float = None, *, stream=N
     return out
 
 
+SCALINGS = {"row": 0, "map": 1}  # SSA_SCALE_ROW, SSA_SCALE_MAP
+
+
 def capture(maps: torch.Tensor, lam: float = 0.5, tau: float = 0.3, mu: float = 0.8,
-            eps: float = 1e-8, *, stream=None, check: bool = True, out=None, ws=None, status=None):
-    """sparse_pattern_capture on maps [n, L, L] float32 (CUDA).  Returns a dict of CUDA
-    int32 tensors: diag_ptr [n+1], diag_offsets [n*L], vert_ptr [n+1], vert_cols [n*L]."""
+            eps: float = 1e-8, *, scaling: str = "row", true_mask: bool = False, stream=None,
+            check: bool = True, out=None, ws=None, status=None):
+    """sparse_pattern_capture(_ex) on maps [n, L, L] float32 (CUDA).  Returns a dict of CUDA
+    int32 tensors: diag_ptr [n+1], diag_offsets [n*L], vert_ptr [n+1], vert_cols [n*L], and
+    with true_mask=True also "true_mask": the bitmap uint32 [n, L, ceil(L/32)] (as int32)."""
     lib = load()
     _need_cuda(maps, "maps", torch.float32)
     n, L, L2 = maps.shape
@@ -177,9 +189,20 @@ def capture(maps: torch.Tensor, lam: float = 0.5, tau: float = 0.3, mu: float = 
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=dev)
     cs, s = _stream(stream)
-    _check(lib.sparse_pattern_capture(_ptr(maps), n, L, lam, tau, mu, eps, _ptr(out["diag_ptr"]),
-                                      _ptr(out["diag_offsets"]), _ptr(out["vert_ptr"]),
-                                      _ptr(out["vert_cols"]), _ptr(ws), ws.numel(), _ptr(status), cs))
+    if scaling not in SCALINGS:
+        raise SSAError(-1, f"scaling must be one of {sorted(SCALINGS)}")
+    if true_mask and "true_mask" not in out:
+        out["true_mask"] = torch.empty((n, L, (L + 31) // 32), dtype=torch.int32, device=dev)
+    if scaling == "row" and not true_mask:
+        _check(lib.sparse_pattern_capture(_ptr(maps), n, L, lam, tau, mu, eps, _ptr(out["diag_ptr"]),
+                                          _ptr(out["diag_offsets"]), _ptr(out["vert_ptr"]),
+                                          _ptr(out["vert_cols"]), _ptr(ws), ws.numel(), _ptr(status), cs))
+    else:
+        tm = out.get("true_mask") if true_mask else None
+        _check(lib.sparse_pattern_capture_ex(_ptr(maps), n, L, lam, tau, mu, eps, SCALINGS[scaling],
+                                             _ptr(out["diag_ptr"]), _ptr(out["diag_offsets"]),
+                                             _ptr(out["vert_ptr"]), _ptr(out["vert_cols"]), _ptr(tm),
+                                             _ptr(ws), ws.numel(), _ptr(status), cs))
     if check:
         _check_status(status, s)
     return out
@@ -212,6 +235,11 @@ class Plan:
         for name in ("ext_diag_ptr", "ext_diag_offsets", "ext_vert_ptr", "ext_vert_cols", "tile_ptr",
                      "tile_key0", "tile_dmask", "tile_cmask", "tile_flags", "stripe_cnt"):
             setattr(st, name, getattr(self, name).data_ptr())
+        self.tile_bits = None
+        if sizes.bitmap_slots > 0:  # Case-2 plan: element bitmaps, 128 rows x 2 words per slot
+            self.tile_bits = torch.empty((H * sizes.bitmap_slots, 128, 2), dtype=torch.int64, device=device)
+            st.bitmap_slots = sizes.bitmap_slots
+            st.tile_bits = self.tile_bits.data_ptr()
         self.struct = st
 
     @property
@@ -234,6 +262,8 @@ class Plan:
                    tile_cmask=self.tile_cmask[:T].cpu().numpy().view("uint64"),
                    tile_flags=self.tile_flags[:T].cpu().numpy().view("uint32"),
                    stripe_cnt=self.stripe_cnt.cpu().numpy())
+        if self.tile_bits is not None:
+            out["tile_bits"] = self.tile_bits.cpu().numpy().view("uint64")
         edp = self.ext_diag_ptr.cpu().numpy()
         evp = self.ext_vert_ptr.cpu().numpy()
         out["ext"] = (edp, self.ext_diag_offsets.cpu().numpy()[:edp[-1]], evp,
@@ -242,8 +272,10 @@ class Plan:
 
 
 def extend(diag_ptr, diag_offsets, vert_ptr, vert_cols, S: int, *, stream=None, check: bool = True,
-           ws=None, status=None, sizes_only: bool = False):
-    """sparse_pattern_extend: sizing pass (synchronises) then fill pass.  Returns a Plan."""
+           ws=None, status=None, sizes_only: bool = False, true_mask=None):
+    """sparse_pattern_extend: sizing pass (synchronises) then fill pass.  Returns a Plan.
+    With true_mask (the capture's bitmap, int32 [H, L, ceil(L/32)] on the device) it is
+    sparse_pattern_extend_case2: the first L x L block keeps the true mask."""
     lib = load()
     for t, nm in ((diag_ptr, "diag_ptr"), (diag_offsets, "diag_offsets"), (vert_ptr, "vert_ptr"),
                   (vert_cols, "vert_cols")):
@@ -265,16 +297,25 @@ def extend(diag_ptr, diag_offsets, vert_ptr, vert_cols, S: int, *, stream=None, 
         status = torch.zeros(1, dtype=torch.int32, device=dev)
     cs, s = _stream(stream)
     sizes = PlanSizes()
-    _check(lib.sparse_pattern_extend(H, _ptr(diag_ptr), _ptr(diag_offsets), _ptr(vert_ptr),
-                                     _ptr(vert_cols), S, C.byref(sizes), None, _ptr(ws), ws.numel(),
-                                     _ptr(status), cs))
+    if true_mask is not None:
+        _need_cuda(true_mask, "true_mask", torch.int32)
+        if true_mask.dim() != 3 or true_mask.shape[0] != H or true_mask.shape[2] != (true_mask.shape[1] + 31) // 32:
+            raise SSAError(-1, "true_mask must be [H, L, ceil(L/32)] int32")
+        L = true_mask.shape[1]
+        run = lambda pl: lib.sparse_pattern_extend_case2(H, _ptr(diag_ptr), _ptr(diag_offsets), _ptr(vert_ptr),
+                                                         _ptr(vert_cols), _ptr(true_mask), L, S, C.byref(sizes),
+                                                         pl, _ptr(ws), ws.numel(), _ptr(status), cs)
+    else:
+        run = lambda pl: lib.sparse_pattern_extend(H, _ptr(diag_ptr), _ptr(diag_offsets), _ptr(vert_ptr),
+                                                   _ptr(vert_cols), S, C.byref(sizes), pl, _ptr(ws), ws.numel(),
+                                                   _ptr(status), cs)
+    _check(run(None))
     if sizes_only:
         return sizes
     plan = Plan(sizes, dev)
     plan._ws = ws
-    _check(lib.sparse_pattern_extend(H, _ptr(diag_ptr), _ptr(diag_offsets), _ptr(vert_ptr),
-                                     _ptr(vert_cols), S, C.byref(sizes), C.byref(plan.struct), _ptr(ws),
-                                     ws.numel(), _ptr(status), cs))
+    plan._true_mask = true_mask
+    _check(run(C.byref(plan.struct)))
     if check:
         _check_status(status, s)
     return plan

@@ -158,6 +158,7 @@ struct AttnParams {
     const uint64_t *tile_dmask;
     const uint64_t *tile_cmask;
     const uint32_t *tile_flags;
+    const uint64_t *tile_bits;  // Case-2 plans: element bitmaps (flag 2 tiles), else null
     const int32_t *stripe_cnt;
     const int32_t *vert_ptr;
     const int32_t *vert_cols;
@@ -832,9 +833,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fetch(j);
                 if (j < nb) {
                     full = (mf & 1u) != 0;
-                    row_diag_mask(md, il, mlo, mhi);
-                    mlo &= ~mc[0];
-                    mhi &= ~mc[1];
+                    if (mf & 2u) {
+                        // element-bitmap tile (Case 2): the row's 128 bits, slot in dmask word 0
+                        const ulonglong2 b =
+                            __ldg(reinterpret_cast<const ulonglong2 *>(p.tile_bits) + md[0] * kBM + il);
+                        mlo = b.x;
+                        mhi = b.y;
+                    } else {
+                        row_diag_mask(md, il, mlo, mhi);
+                        mlo &= ~mc[0];
+                        mhi &= ~mc[1];
+                    }
                     if (!row_ok) mlo = mhi = 0;
                 } else {
                     const int lk = n_i - (j - nb) * kBN;  // key column k active iff k < lk
@@ -1105,6 +1114,8 @@ extern "C" int sparse_attn_fwd(const void *Q, const void *K, const void *V, int 
                   "sparse_attn_fwd: Q, K, V and O must be 16-byte aligned");
     SSA_CHECK_ARG(aligned16(plan->tile_dmask) && aligned16(plan->tile_cmask),
                   "sparse_attn_fwd: plan tile_dmask and tile_cmask must be 16-byte aligned");
+    SSA_CHECK_ARG(plan->bitmap_slots == 0 || (plan->tile_bits && aligned16(plan->tile_bits)),
+                  "sparse_attn_fwd: a Case-2 plan needs tile_bits (16-byte aligned)");
     SSA_CHECK_ARG(scale > 0.0f && scale < 1e30f, "sparse_attn_fwd: scale must be positive and finite");
     SSA_CHECK_ARG(static_cast<int64_t>(H_q) * ((S + kBM - 1) / kBM) < (1LL << 30),
                   "sparse_attn_fwd: too many query blocks");
@@ -1125,6 +1136,7 @@ extern "C" int sparse_attn_fwd(const void *Q, const void *K, const void *V, int 
     p.tile_dmask = plan->tile_dmask;
     p.tile_cmask = plan->tile_cmask;
     p.tile_flags = plan->tile_flags;
+    p.tile_bits = plan->tile_bits;
     p.stripe_cnt = plan->stripe_cnt;
     p.vert_ptr = plan->ext_vert_ptr;
     p.vert_cols = plan->ext_vert_cols;

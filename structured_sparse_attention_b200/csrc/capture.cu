@@ -20,6 +20,8 @@
 // 33-way bracketing search), so each decision equals the one obtained by evaluating
 // the sequence at every entry.  Each row thus costs a few fp64 evaluations per lane
 // instead of one per entry.
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace ssa {
@@ -45,37 +47,59 @@ struct CaptureParams {
     int32_t *vert_cols;
     int32_t *status;
     int row_chunks;  // CTAs per map of the hits kernel; rows interleaved across them
+    int scaling;     // 0: min and max of each row's causal entries; 1: of the whole map's
+    uint32_t *map_mm;  // per map: min and max bits of its causal entries (scaling 1)
+    uint32_t *bits;    // optional true mask [n_maps][L][bits_words] (bit j of row i), or null
+    int bits_words;    // ceil(L / 32)
 };
 
-__device__ __forceinline__ double box_cox_rn(double x, double eps, double lambda, bool half) {
+// Box-Cox of x + eps: ((x + eps)^lambda - 1) / lambda, log(x + eps) at lambda = 0.  At
+// lambda 1/2 and 1 every step is correctly rounded (sqrt, +, -, /), as in the oracle;
+// other lambdas use pow / log, which are not correctly rounded on either side, so a
+// decision within a few units in the last place of tau may differ from the oracle's.
+// Transform kinds: TR_SQRT (lambda = 1/2), TR_LINEAR (lambda = 1), TR_POW (any other).
+constexpr int TR_SQRT = 0, TR_LINEAR = 1, TR_POW = 2;
+
+template <int TR>
+__device__ __forceinline__ double box_cox_rn(double x, double eps, double lambda) {
     double z = __dadd_rn(x, eps);
-    double s = half ? __dsqrt_rn(z) : z;
-    return __ddiv_rn(__dsub_rn(s, 1.0), lambda);
+    if constexpr (TR == TR_SQRT) return __ddiv_rn(__dsub_rn(__dsqrt_rn(z), 1.0), lambda);
+    if constexpr (TR == TR_LINEAR) return __ddiv_rn(__dsub_rn(z, 1.0), lambda);
+    if (lambda == 0.0) return log(z);
+    return __ddiv_rn(__dsub_rn(pow(z, lambda), 1.0), lambda);
 }
 
-__device__ __forceinline__ bool decide(uint32_t xbits, double eps, double lambda, bool half,
-                                       double ylo, double yrange, double tau) {
+template <int TR>
+__device__ __forceinline__ bool decide(uint32_t xbits, double eps, double lambda, double ylo, double yrange,
+                                       double tau) {
     double x = static_cast<double>(__uint_as_float(xbits));
-    double t = __ddiv_rn(__dsub_rn(box_cox_rn(x, eps, lambda, half), ylo), yrange);
+    double t = __ddiv_rn(__dsub_rn(box_cox_rn<TR>(x, eps, lambda), ylo), yrange);
     return t >= tau;
 }
 
 // Smallest float bit pattern u in [u0, u1] with decide(u) true, or u1 + 1 if none.
 // Collective over the warp; every lane returns the same value.
-__device__ uint32_t find_cut(uint32_t u0, uint32_t u1, float mn, float mx, double eps,
-                             double lambda, bool half, double tau) {
+template <int TR>
+__device__ uint32_t find_cut(uint32_t u0, uint32_t u1, float mn, float mx, double eps, double lambda,
+                             double tau) {
     const int lane = threadIdx.x & 31;
-    const double ylo = box_cox_rn(static_cast<double>(mn), eps, lambda, half);
-    const double yhi = box_cox_rn(static_cast<double>(mx), eps, lambda, half);
+    const double ylo = box_cox_rn<TR>(static_cast<double>(mn), eps, lambda);
+    const double yhi = box_cox_rn<TR>(static_cast<double>(mx), eps, lambda);
     const double yrange = __dsub_rn(yhi, ylo);
     // Closed-form estimate of the cut (only steers the first probe window).
     double est;
-    if (half) {
+    if constexpr (TR == TR_SQRT) {
         double a = sqrt(static_cast<double>(mn) + eps), b = sqrt(static_cast<double>(mx) + eps);
         double s = a + tau * (b - a);
         est = s * s - eps;
-    } else {
+    } else if constexpr (TR == TR_LINEAR) {
         est = static_cast<double>(mn) + tau * (static_cast<double>(mx) - static_cast<double>(mn));
+    } else if (lambda == 0.0) {
+        const double a = log(static_cast<double>(mn) + eps), b = log(static_cast<double>(mx) + eps);
+        est = exp(a + tau * (b - a)) - eps;
+    } else {
+        const double a = pow(static_cast<double>(mn) + eps, lambda), b = pow(static_cast<double>(mx) + eps, lambda);
+        est = pow(a + tau * (b - a), 1.0 / lambda) - eps;
     }
     float ef = static_cast<float>(est);
     if (!(ef >= mn)) ef = mn;
@@ -107,7 +131,7 @@ __device__ uint32_t find_cut(uint32_t u0, uint32_t u1, float mn, float mx, doubl
         }
         int64_t p = window ? first + lane : first + (step_num * (lane + 1)) / 33;
         bool val = true;
-        if (lane < np) val = decide(static_cast<uint32_t>(p), eps, lambda, half, ylo, yrange, tau);
+        if (lane < np) val = decide<TR>(static_cast<uint32_t>(p), eps, lambda, ylo, yrange, tau);
         const uint32_t ball = __ballot_sync(0xffffffffu, val);
         // first true (lanes >= np report true); 32 when all 32 probes are false
         const int f = ball ? (__ffs(ball) - 1) : 32;
@@ -119,8 +143,8 @@ __device__ uint32_t find_cut(uint32_t u0, uint32_t u1, float mn, float mx, doubl
     return static_cast<uint32_t>(hi);
 }
 
-template <int MAXK>
-__global__ void __launch_bounds__(kCaptureThreads, MAXK <= 16 ? 3 : 1)
+template <int MAXK, int TR>
+__global__ void __launch_bounds__(kCaptureThreads)
     capture_hits_kernel(CaptureParams p) {
     extern __shared__ int32_t s_hist[];  // [2][L]: diagonal hits, column hits
     const int L = p.L;
@@ -130,9 +154,20 @@ __global__ void __launch_bounds__(kCaptureThreads, MAXK <= 16 ? 3 : 1)
     for (int k = threadIdx.x; k < 2 * L; k += kCaptureThreads) s_hist[k] = 0;
     __syncthreads();
 
-    const bool half = (p.lambda == 0.5);
     const float *map = p.maps + static_cast<size_t>(m) * L * L;
     bool bad = false;
+    // per-map scaling: one cut for the whole map, from its min and max (found by warp 0)
+    __shared__ uint32_t s_map_cut;
+    if (p.scaling == 1) {
+        if (warp == 0) {
+            const float mn = __uint_as_float(p.map_mm[2 * m]), mx = __uint_as_float(p.map_mm[2 * m + 1]);
+            const uint32_t u0 = __float_as_uint(mn), u1 = __float_as_uint(mx);
+            const uint32_t c = (u0 == u1) ? ((1.0 >= p.tau) ? 0u : 0xffffffffu)
+                                          : find_cut<TR>(u0, u1, mn, mx, p.eps, p.lambda, p.tau);
+            if (lane == 0) s_map_cut = c;
+        }
+        __syncthreads();
+    }
     // Rows are software-pipelined: the loads of the warp's next row are issued before the
     // current row's cut point is searched, so each warp keeps a row in flight while it
     // computes (the search is a chain of dependent fp64 steps).
@@ -171,19 +206,28 @@ __global__ void __launch_bounds__(kCaptureThreads, MAXK <= 16 ? 3 : 1)
         }
         uint32_t cut;
         const uint32_t u0 = __float_as_uint(mn), u1 = __float_as_uint(mx);
-        if (u0 == u1) {
+        if (p.scaling == 1) {
+            cut = s_map_cut;
+        } else if (u0 == u1) {
             cut = (1.0 >= p.tau) ? 0u : 0xffffffffu;  // constant row: t = 1
         } else {
-            cut = find_cut(u0, u1, mn, mx, p.eps, p.lambda, half, p.tau);
+            cut = find_cut<TR>(u0, u1, mn, mx, p.eps, p.lambda, p.tau);
         }
         // for non-negative floats the order of the values is the order of their bits, so
         // x >= x* is the comparison of the bit patterns (a cut of 0xffffffff keeps none)
 #pragma unroll
         for (int k = 0; k < MAXK; ++k) {
             const int j = lane + 32 * k;
-            if (j < n && __float_as_uint(xc[k]) >= cut) {
+            const bool on = j < n && __float_as_uint(xc[k]) >= cut;
+            if (on) {
                 atomicAdd(&s_hist[i - j], 1);
                 atomicAdd(&s_hist[L + j], 1);
+            }
+            if (p.bits) {
+                // the row's true mask, 32 columns per word
+                const uint32_t word = __ballot_sync(0xffffffffu, on);
+                if (lane == 0 && k < p.bits_words)
+                    p.bits[(static_cast<size_t>(m) * L + i) * p.bits_words + k] = word;
             }
         }
 #pragma unroll
@@ -209,6 +253,45 @@ int sm_count_capture() {
         cached[dev] = n;
     }
     return cached[dev];
+}
+
+// Per-map min and max of the causal entries (scaling 1), as float bit patterns: for the
+// non-negative floats of a map the order of the bits is the order of the values (-0 is
+// taken as +0).  map_mm must hold {0xffffffff, 0} per map on entry.
+__global__ void __launch_bounds__(kCaptureThreads) capture_minmax_kernel(CaptureParams p) {
+    const int L = p.L;
+    const int m = blockIdx.x / p.row_chunks;
+    const int chunk = blockIdx.x % p.row_chunks;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float *map = p.maps + static_cast<size_t>(m) * L * L;
+    uint32_t mn = 0xffffffffu, mx = 0u;
+    for (int i = chunk + p.row_chunks * warp; i < L; i += p.row_chunks * kCaptureWarps) {
+        const float *row = map + static_cast<size_t>(i) * L;
+        for (int j = lane; j <= i; j += 32) {
+            uint32_t b = __float_as_uint(__ldg(row + j));
+            if (b == 0x80000000u) b = 0;
+            mn = min(mn, b);
+            mx = max(mx, b);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (lane == 0) {
+        atomicMin(p.map_mm + 2 * m, mn);
+        atomicMax(p.map_mm + 2 * m + 1, mx);
+    }
+}
+
+// {0xffffffff, 0} for every map: the identities of the min / max reductions.
+__global__ void capture_minmax_init_kernel(uint32_t *mm, int n_maps) {
+    const int m = blockIdx.x * blockDim.x + threadIdx.x;
+    if (m < n_maps) {
+        mm[2 * m] = 0xffffffffu;
+        mm[2 * m + 1] = 0u;
+    }
 }
 
 // Ordered compaction of {x in [0, L) : keep(x)} by the whole block.
@@ -313,11 +396,12 @@ extern "C" size_t sparse_pattern_capture_ws_bytes(int n_maps, int L) {
     return static_cast<size_t>(n_maps) * (4 * static_cast<size_t>(L) + 2) * sizeof(int32_t);
 }
 
-extern "C" int sparse_pattern_capture(const float *maps, int n_maps, int L, double lambda,
-                                      double tau, double mu, double eps, int32_t *diag_ptr,
-                                      int32_t *diag_offsets, int32_t *vert_ptr,
-                                      int32_t *vert_cols, void *ws, size_t ws_bytes,
-                                      int32_t *dev_status, void *stream) {
+extern "C" int sparse_pattern_capture_ex(const float *maps, int n_maps, int L, double lambda,
+                                         double tau, double mu, double eps, int scaling,
+                                         int32_t *diag_ptr, int32_t *diag_offsets,
+                                         int32_t *vert_ptr, int32_t *vert_cols,
+                                         uint32_t *true_mask, void *ws, size_t ws_bytes,
+                                         int32_t *dev_status, void *stream) {
     SSA_CHECK_ARG(maps && diag_ptr && diag_offsets && vert_ptr && vert_cols && ws,
                   "sparse_pattern_capture: null pointer argument");
     SSA_CHECK_ARG(n_maps >= 1, "sparse_pattern_capture: n_maps must be >= 1 (got %d)", n_maps);
@@ -325,10 +409,12 @@ extern "C" int sparse_pattern_capture(const float *maps, int n_maps, int L, doub
         set_error("sparse_pattern_capture: L must be in [1, 1024] (got %d)", L);
         return L < 1 ? SSA_ERR_INVALID : SSA_ERR_UNSUPPORTED;
     }
-    if (!(lambda == 0.5 || lambda == 1.0)) {
-        set_error("sparse_pattern_capture: lambda must be 0.5 or 1.0 (got %g)", lambda);
-        return SSA_ERR_UNSUPPORTED;
-    }
+    SSA_CHECK_ARG(lambda >= 0.0 && lambda <= 64.0, "sparse_pattern_capture: lambda must be in [0, 64] (got %g)",
+                  lambda);
+    SSA_CHECK_ARG(scaling == SSA_SCALE_ROW || scaling == SSA_SCALE_MAP,
+                  "sparse_pattern_capture: scaling must be SSA_SCALE_ROW or SSA_SCALE_MAP (got %d)", scaling);
+    SSA_CHECK_ARG((reinterpret_cast<uintptr_t>(true_mask) & 3u) == 0,
+                  "sparse_pattern_capture: true_mask must be 4-byte aligned");
     SSA_CHECK_ARG(eps >= 0.0 && eps < 1e300, "sparse_pattern_capture: eps must be finite and >= 0");
     SSA_CHECK_ARG(tau == tau && mu == mu, "sparse_pattern_capture: tau and mu must not be NaN");
     SSA_CHECK_ARG((reinterpret_cast<uintptr_t>(ws) & 3u) == 0,
@@ -357,6 +443,10 @@ extern "C" int sparse_pattern_capture(const float *maps, int n_maps, int L, doub
     p.vert_ptr = vert_ptr;
     p.vert_cols = vert_cols;
     p.status = dev_status;
+    p.scaling = scaling;
+    p.map_mm = reinterpret_cast<uint32_t *>(p.staging);  // free until the select kernel
+    p.bits = true_mask;
+    p.bits_words = (L + 31) / 32;
 
     SSA_CUDA_TRY(cudaMemsetAsync(p.hits, 0, static_cast<size_t>(n_maps) * 2 * L * sizeof(int32_t), s));
     const size_t smem = 2 * static_cast<size_t>(L) * sizeof(int32_t);
@@ -368,17 +458,37 @@ extern "C" int sparse_pattern_capture(const float *maps, int n_maps, int L, doub
         chunks *= 2;
     p.row_chunks = chunks;
     const unsigned grid = static_cast<unsigned>(n_maps) * chunks;
-    if (L <= 512) {
-        capture_hits_kernel<16><<<grid, kCaptureThreads, smem, s>>>(p);
-    } else {
-        capture_hits_kernel<32><<<grid, kCaptureThreads, smem, s>>>(p);
+    if (scaling == SSA_SCALE_MAP) {
+        capture_minmax_init_kernel<<<(n_maps + 255) / 256, 256, 0, s>>>(p.map_mm, n_maps);
+        SSA_LAUNCH_CHECK();
+        capture_minmax_kernel<<<grid, kCaptureThreads, 0, s>>>(p);
+        SSA_LAUNCH_CHECK();
     }
+    const int tr = lambda == 0.5 ? TR_SQRT : (lambda == 1.0 ? TR_LINEAR : TR_POW);
+    auto launch_hits = [&](auto MK) {
+        constexpr int MAXK = decltype(MK)::value;
+        if (tr == TR_SQRT) capture_hits_kernel<MAXK, TR_SQRT><<<grid, kCaptureThreads, smem, s>>>(p);
+        else if (tr == TR_LINEAR) capture_hits_kernel<MAXK, TR_LINEAR><<<grid, kCaptureThreads, smem, s>>>(p);
+        else capture_hits_kernel<MAXK, TR_POW><<<grid, kCaptureThreads, smem, s>>>(p);
+    };
+    if (L <= 512) launch_hits(std::integral_constant<int, 16>{});
+    else launch_hits(std::integral_constant<int, 32>{});
     SSA_LAUNCH_CHECK();
     capture_select_kernel<<<n_maps, kCaptureThreads, 0, s>>>(p);
     SSA_LAUNCH_CHECK();
     capture_pack_kernel<<<n_maps, kCaptureThreads, 0, s>>>(p);
     SSA_LAUNCH_CHECK();
     return SSA_OK;
+}
+
+extern "C" int sparse_pattern_capture(const float *maps, int n_maps, int L, double lambda,
+                                      double tau, double mu, double eps, int32_t *diag_ptr,
+                                      int32_t *diag_offsets, int32_t *vert_ptr,
+                                      int32_t *vert_cols, void *ws, size_t ws_bytes,
+                                      int32_t *dev_status, void *stream) {
+    return sparse_pattern_capture_ex(maps, n_maps, L, lambda, tau, mu, eps, SSA_SCALE_ROW, diag_ptr,
+                                     diag_offsets, vert_ptr, vert_cols, nullptr, ws, ws_bytes,
+                                     dev_status, stream);
 }
 
 // ---------------------------------------------------------------------------------

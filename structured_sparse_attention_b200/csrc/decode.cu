@@ -292,6 +292,10 @@ extern "C" int sparse_attn_decode(const void *Q, const void *K, const void *V, i
     SSA_CHECK_ARG(kv_map || H_q % H_kv == 0,
                   "sparse_attn_decode: H_q (%d) must be a multiple of H_kv (%d) without kv_map", H_q,
                   H_kv);
+    if (plan->bitmap_slots != 0) {
+        set_error("sparse_attn_decode: Case-2 plans (element-bitmap tiles) are not supported by decoding");
+        return SSA_ERR_UNSUPPORTED;
+    }
     SSA_CHECK_ARG(plan->S == S_cache && plan->n_heads == H_q,
                   "sparse_attn_decode: plan (S=%d heads=%d) does not match S_cache=%d H_q=%d", plan->S,
                   plan->n_heads, S_cache, H_q);

@@ -53,6 +53,11 @@ struct PlanParams {
     uint32_t *tile_flags;
     int32_t *stripe_cnt;
     int32_t *ext_dptr, *ext_doff, *ext_vptr, *ext_vcol;
+    // Case 2 (tmask non-null): the true masks [H][L][bw] and the bitmap tiles
+    const uint32_t *tmask;
+    int L, bw;      // capture length, words per true-mask row (ceil(L / 32))
+    int nL, slots;  // query blocks holding a row < min(L, S); bitmap slots per head
+    uint64_t *tile_bits;
 };
 
 __global__ void validate_lists_kernel(PlanParams p) {
@@ -223,6 +228,103 @@ __device__ int eval_window(const int32_t *D, int nD, const int32_t *C, int nC, i
     return full ? 2 : 1;
 }
 
+// Diagonal and column masks of the window key0 .. key0 + 127 for query block qb (the
+// dmask / cmask of eval_window, without its listing decision).
+__device__ void window_masks(const int32_t *D, int nD, const int32_t *C, int nC, int qb, int key0,
+                             uint64_t (&dm)[4], uint64_t (&cm)[2]) {
+    const int base = kTile * qb - key0 - (kTile - 1);  // r of dmask bit 0
+    const int lb = lower_bound_i32(D, nD, max(base, 0));
+    const int ub = lower_bound_i32(D, nD, base + 2 * kTile - 1);
+    dm[0] = dm[1] = dm[2] = dm[3] = 0;
+    for (int k = lb; k < ub; ++k) {
+        const int t = __ldg(D + k) - base;
+        dm[t >> 6] |= 1ull << (t & 63);
+    }
+    cm[0] = cm[1] = 0;
+    for (int k = lower_bound_i32(C, nC, key0); k < nC; ++k) {
+        const int jl = __ldg(C + k) - key0;
+        if (jl >= kTile) break;
+        cm[jl >> 6] |= 1ull << (jl & 63);
+    }
+}
+
+// Case 2, one warp per query block qb < nL of head h: element-bitmap tiles for the key
+// blocks kb = 0..qb (key0 = 128 kb), listed when any cell is set.  Cell (i, j) of a tile:
+// i < S and j <= i and, for i < L, bit j of row i of the head's true mask; for i >= L,
+// i - j an extended diagonal or j an extended column.  Returns the tiles listed.
+template <bool FILL>
+__device__ int bitmap_tiles(const PlanParams &p, int h, int qb, const int32_t *D, int nD, const int32_t *C,
+                            int nC, int64_t pos) {
+    const int lane = threadIdx.x & 31;
+    const int lo = kTile * qb;
+    const uint32_t *tm = p.tmask + static_cast<size_t>(h) * p.L * p.bw;
+    int count = 0;
+    for (int kb = 0; kb <= qb; ++kb) {
+        uint64_t dm[4], cm[2];
+        const bool past_L = lo + kTile > p.L;  // the block holds rows >= L
+        if (past_L) window_masks(D, nD, C, nC, qb, kTile * kb, dm, cm);
+        uint64_t rb[4][2];
+        uint64_t any = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int il = lane + 32 * q, i = lo + il;
+            uint64_t b0 = 0, b1 = 0;
+            if (i < p.S) {
+                if (i < p.L) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const int wi = 4 * kb + x;  // word of columns 32 wi .. 32 wi + 31
+                        w[x] = wi < p.bw ? __ldg(tm + static_cast<size_t>(i) * p.bw + wi) : 0u;
+                    }
+                    b0 = static_cast<uint64_t>(w[0]) | (static_cast<uint64_t>(w[1]) << 32);
+                    b1 = static_cast<uint64_t>(w[2]) | (static_cast<uint64_t>(w[3]) << 32);
+                } else {
+                    row_diag_mask(dm, il, b0, b1);  // diagonals (r >= 0, so j <= i)
+                    b0 |= cm[0];
+                    b1 |= cm[1];
+                }
+                if (kb == qb) {  // the diagonal tile: columns jl <= il only
+                    const int n = il + 1;
+                    b0 &= n >= 64 ? ~0ull : ((1ull << n) - 1ull);
+                    b1 &= n >= 128 ? ~0ull : (n <= 64 ? 0ull : ((1ull << (n - 64)) - 1ull));
+                }
+            }
+            rb[q][0] = b0;
+            rb[q][1] = b1;
+            any |= b0 | b1;
+        }
+        const int slot = h * p.slots + qb * (qb + 1) / 2 + kb;
+        if (FILL) {  // every slot is written, listed or not
+            uint64_t *bits = p.tile_bits + static_cast<size_t>(slot) * kTile * 2;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int il = lane + 32 * q;
+                bits[2 * il] = rb[q][0];
+                bits[2 * il + 1] = rb[q][1];
+            }
+        }
+        if (!__any_sync(0xffffffffu, any != 0)) continue;
+        if (FILL) {
+            const int64_t t = pos + count;
+            if (t < p.capacity) {
+                if (lane == 0) {
+                    p.tile_key0[t] = kTile * kb;
+                    uint64_t *dst = p.tile_dmask + 4 * t;
+                    dst[0] = static_cast<uint64_t>(slot);  // the bitmap's slot
+                    dst[1] = dst[2] = dst[3] = 0;
+                    p.tile_cmask[2 * t] = p.tile_cmask[2 * t + 1] = 0;
+                    p.tile_flags[t] = 2u;  // BITMAP
+                }
+            } else if (lane == 0) {
+                report(p.dev_status, SSA_ERR_CAPACITY);
+            }
+        }
+        ++count;
+    }
+    return count;
+}
+
 // One warp per (head, query block).  FILL = false: count; FILL = true: write tiles.
 template <bool FILL>
 __global__ void __launch_bounds__(128) plan_tiles_kernel(PlanParams p) {
@@ -233,6 +335,14 @@ __global__ void __launch_bounds__(128) plan_tiles_kernel(PlanParams p) {
     const int32_t *D = p.doff + p.dptr[h];
     const int32_t *C = p.vcol + p.vptr[h];
     const int nD = p.ext_counts[2 * h], nC = p.ext_counts[2 * h + 1];
+    if (p.tmask && qb < p.nL) {  // Case 2: element-bitmap tiles, no stripe tiles
+        const int n = bitmap_tiles<FILL>(p, h, qb, D, nD, C, nC, FILL ? p.tile_ptr[item] : 0);
+        if (lane == 0) {
+            if (FILL) p.stripe_cnt[item] = 0;
+            else p.tile_counts[item] = n;
+        }
+        return;
+    }
     // windows are chosen over all 128 rows of the block (lo .. hi), even past S
     const int lo = kTile * qb, hi = lo + kTile - 1;
     if (FILL && lane == 0) p.stripe_cnt[item] = lower_bound_i32(C, nC, min(hi, p.S - 1) + 1);
@@ -336,11 +446,11 @@ extern "C" size_t sparse_pattern_extend_ws_bytes(int n_heads, int S) {
            align_up(sizeof(int32_t) * static_cast<size_t>(n_heads) * static_cast<size_t>(S)) + 256;
 }
 
-extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
-                                     const int32_t *diag_offsets, const int32_t *vert_ptr,
-                                     const int32_t *vert_cols, int S, ssa_plan_sizes *sizes,
-                                     const ssa_plan *plan, void *ws, size_t ws_bytes,
-                                     int32_t *dev_status, void *stream) {
+namespace {
+
+int extend_impl(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offsets, const int32_t *vert_ptr,
+                const int32_t *vert_cols, const uint32_t *true_mask, int L, int S, ssa_plan_sizes *sizes,
+                const ssa_plan *plan, void *ws, size_t ws_bytes, int32_t *dev_status, void *stream) {
     SSA_CHECK_ARG(diag_ptr && diag_offsets && vert_ptr && vert_cols && ws,
                   "sparse_pattern_extend: null pointer argument");
     SSA_CHECK_ARG(n_heads >= 1 && S >= 1, "sparse_pattern_extend: n_heads and S must be >= 1");
@@ -380,6 +490,15 @@ extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
 
     const int items = n_heads * nqb;
     const unsigned tile_grid = static_cast<unsigned>((items + 3) / 4);
+    int slots = 0;
+    if (true_mask) {
+        p.tmask = true_mask;
+        p.L = L;
+        p.bw = (L + 31) / 32;
+        p.nL = (min(L, S) + kTile - 1) / kTile;
+        slots = p.nL * (p.nL + 1) / 2;
+        p.slots = slots;
+    }
     SSA_CUDA_TRY(cudaMemsetAsync(p.totals, 0, sizeof(Totals), s));
 
     if (plan == nullptr) {
@@ -405,6 +524,7 @@ extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
         sizes->n_vert = host.n_vert;
         sizes->max_vert = host.max_vert;
         sizes->n_tiles = host.n_tiles;
+        sizes->bitmap_slots = slots;
         if (host.status != 0) {
             set_error("sparse_pattern_extend: a pattern list is not strictly ascending and >= 0");
             return SSA_ERR_INVALID;
@@ -422,6 +542,13 @@ extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
                       plan->stripe_cnt,
                   "sparse_pattern_extend: null plan array");
     SSA_CHECK_ARG(plan->n_tiles >= 0, "sparse_pattern_extend: negative tile capacity");
+    if (true_mask) {
+        SSA_CHECK_ARG(plan->tile_bits && plan->bitmap_slots == slots && aligned16(plan->tile_bits),
+                      "sparse_pattern_extend_case2: plan needs tile_bits (16-byte aligned) for %d bitmap "
+                      "slots per head",
+                      slots);
+        p.tile_bits = plan->tile_bits;
+    }
     p.tile_ptr = plan->tile_ptr;
     p.capacity = plan->n_tiles;
     p.tile_key0 = plan->tile_key0;
@@ -452,4 +579,28 @@ extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
     plan_tiles_kernel<true><<<tile_grid, 128, 0, s>>>(p);
     SSA_LAUNCH_CHECK();
     return SSA_OK;
+}
+
+}  // namespace
+
+extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
+                                     const int32_t *diag_offsets, const int32_t *vert_ptr,
+                                     const int32_t *vert_cols, int S, ssa_plan_sizes *sizes,
+                                     const ssa_plan *plan, void *ws, size_t ws_bytes,
+                                     int32_t *dev_status, void *stream) {
+    return extend_impl(n_heads, diag_ptr, diag_offsets, vert_ptr, vert_cols, nullptr, 0, S, sizes, plan, ws,
+                       ws_bytes, dev_status, stream);
+}
+
+extern "C" int sparse_pattern_extend_case2(int n_heads, const int32_t *diag_ptr,
+                                           const int32_t *diag_offsets, const int32_t *vert_ptr,
+                                           const int32_t *vert_cols, const uint32_t *true_mask, int L,
+                                           int S, ssa_plan_sizes *sizes, const ssa_plan *plan, void *ws,
+                                           size_t ws_bytes, int32_t *dev_status, void *stream) {
+    SSA_CHECK_ARG(true_mask, "sparse_pattern_extend_case2: null true_mask");
+    SSA_CHECK_ARG(L >= 1 && L <= 1024, "sparse_pattern_extend_case2: L must be in [1, 1024] (got %d)", L);
+    SSA_CHECK_ARG((reinterpret_cast<uintptr_t>(true_mask) & 3u) == 0,
+                  "sparse_pattern_extend_case2: true_mask must be 4-byte aligned");
+    return extend_impl(n_heads, diag_ptr, diag_offsets, vert_ptr, vert_cols, true_mask, L, S, sizes, plan, ws,
+                       ws_bytes, dev_status, stream);
 }

@@ -45,10 +45,14 @@ def test_host_argument_checks(lib):
     from structured_sparse_attention_b200 import binding
     P = C.c_void_p
     dummy = P(256)
-    # unsupported lambda and L are rejected before any device work
-    rc = lib.sparse_pattern_capture(dummy, 1, 16, 0.7, 0.3, 0.8, 1e-8, dummy, dummy, dummy, dummy,
+    # lambda outside [0, 64], an unknown scaling and an unsupported L are rejected
+    # before any device work
+    rc = lib.sparse_pattern_capture(dummy, 1, 16, -0.5, 0.3, 0.8, 1e-8, dummy, dummy, dummy, dummy,
                                     dummy, 1 << 20, None, None)
-    assert rc == -2 and b"lambda" in lib.ssa_last_error()
+    assert rc == -1 and b"lambda" in lib.ssa_last_error()
+    rc = lib.sparse_pattern_capture_ex(dummy, 1, 16, 0.5, 0.3, 0.8, 1e-8, 2, dummy, dummy, dummy, dummy,
+                                       None, dummy, 1 << 20, None, None)
+    assert rc == -1 and b"scaling" in lib.ssa_last_error()
     rc = lib.sparse_pattern_capture(dummy, 1, 2048, 0.5, 0.3, 0.8, 1e-8, dummy, dummy, dummy, dummy,
                                     dummy, 1 << 30, None, None)
     assert rc == -2

@@ -76,3 +76,66 @@ def test_capture_rejects_negative_entries():
     with pytest.raises(ssa.SSAError) as e:
         _run(maps)
     assert e.value.code == -1
+
+
+# --- the optional readings and outputs of sparse_pattern_capture_ex ---------------------
+
+def _bits_to_mask(bits, L):
+    """uint32 words [L][ceil(L/32)] (as int32) -> uint8 [L, L]."""
+    w = bits.astype(np.uint32)
+    j = np.arange(L)
+    return ((w[:, j // 32] >> (j % 32).astype(np.uint32)) & 1).astype(np.uint8)
+
+
+@pytest.mark.parametrize("L", [37, 128, 512])
+@pytest.mark.parametrize("lam", [0.5, 1.0])
+def test_capture_per_map_scaling_matches_oracle(ora, L, lam):
+    maps = inputs.averaged_maps(200 + L, 4, L=L, n_samples=3)
+    for tau, mu in ((0.02, 0.5), (0.1, 0.3), (0.3, 0.05)):
+        _same(_run(maps, lam=lam, tau=tau, mu=mu, scaling="map"),
+              ora.capture(maps, lam=lam, tau=tau, mu=mu, scaling="map"))
+
+
+@pytest.mark.parametrize("lam", [0.0, 0.25, 0.7, 1.5, 2.0, 3.0])
+def test_capture_general_lambda_matches_oracle(ora, lam):
+    # pow / log are not correctly rounded on either side; on these maps no entry lies
+    # within their error of tau, so the lists agree exactly
+    maps = inputs.averaged_maps(17, 4, L=256, n_samples=3)
+    for scaling in ("row", "map"):
+        tau = 0.3 if scaling == "row" else 0.05
+        _same(_run(maps, lam=lam, tau=tau, mu=0.5, scaling=scaling),
+              ora.capture(maps, lam=lam, tau=tau, mu=0.5, scaling=scaling))
+
+
+def test_capture_scaling_fixture_true_masks(ora):
+    # the hand-derived fixture (exact binary fractions, ties on tau), through the bitmap
+    import json
+    import os
+
+    import structured_sparse_attention_b200 as ssa
+    from conftest import GOLDEN
+    fx = json.load(open(os.path.join(GOLDEN, "scaling_cases.json")))
+    amap = np.array(fx["map"], np.float32)[None]
+    for c in fx["cases"]:
+        out = ssa.capture(torch.from_numpy(amap).to("cuda:0"), lam=c["lambda"], tau=c["tau"], eps=0.0,
+                          scaling=c["scaling"], true_mask=True)
+        M = _bits_to_mask(out["true_mask"][0].cpu().numpy(), 4)
+        assert [M[i, :i + 1].tolist() for i in range(4)] == c["M"], c
+        assert not np.triu(M, 1).any()
+
+
+@pytest.mark.parametrize("L", [5, 100, 512, 700])
+def test_capture_true_mask_bitmap_matches_oracle(ora, L):
+    import structured_sparse_attention_b200 as ssa
+    maps = inputs.averaged_maps(300 + L, 3, L=L, n_samples=2)
+    for scaling in ("row", "map"):
+        tau = 0.3 if scaling == "row" else 0.05
+        out = ssa.capture(torch.from_numpy(maps).to("cuda:0"), tau=tau, scaling=scaling, true_mask=True)
+        got = out["true_mask"].cpu().numpy()
+        for m in range(len(maps)):
+            np.testing.assert_array_equal(_bits_to_mask(got[m], L), ora.true_mask(maps[m], tau=tau, scaling=scaling))
+        # the lists of the same call are those of the oracle
+        dp = out["diag_ptr"].cpu().numpy()
+        vp = out["vert_ptr"].cpu().numpy()
+        _same((dp, out["diag_offsets"].cpu().numpy()[:dp[-1]], vp, out["vert_cols"].cpu().numpy()[:vp[-1]]),
+              ora.capture(maps, tau=tau, scaling=scaling))

@@ -121,3 +121,91 @@ def test_block_replaces_the_patterns_there(ora):
     assert (O[0, :L] == 0).all() and (LSE[0, :L] == -np.inf).all()
     f = lambda a: inputs.f32_from_bf16_bits(a).astype(np.float64)
     np.testing.assert_array_equal(O[0, L:], f(v[0, L:]))  # past the block: the diagonal r = 0
+
+
+# --- the Case-2 tile plan (element-bitmap tiles over the first block) -------------------
+
+def _plan_cells(pl, S, ext, h):
+    """The (i, j) cells a plan retains for head h, cell by cell from its tiles: bitmap
+    tiles by their bits, band windows by the diagonal and column masks, stripe tiles by
+    the stripe counts (columns c <= i among the first stripe_cnt kept columns)."""
+    T, nqb = 128, pl["nqb"]
+    dp, do, vp, vo = ext
+    C = vo[vp[h]:vp[h + 1]]
+    cells = set()
+    for qb in range(nqb):
+        it = h * nqb + qb
+        for t in range(pl["tile_ptr"][it], pl["tile_ptr"][it + 1]):
+            k0 = int(pl["tile_key0"][t])
+            for il in range(T):
+                i = T * qb + il
+                if i >= S:
+                    break
+                for jl in range(T):
+                    j = k0 + jl
+                    if pl["tile_flags"][t] & 2:
+                        w = pl["tile_bits"][int(pl["tile_dmask"][t][0]), il, jl // 64]
+                        on = (int(w) >> (jl % 64)) & 1
+                    else:
+                        tt = il - jl + 127
+                        dm = int(pl["tile_dmask"][t][tt // 64])
+                        cm = int(pl["tile_cmask"][t][jl // 64])
+                        on = ((dm >> (tt % 64)) & 1) and not ((cm >> (jl % 64)) & 1)
+                    if on:
+                        assert j <= i and (i, j) not in cells
+                        cells.add((i, j))
+        sc = int(pl["stripe_cnt"][it])
+        for il in range(T):
+            i = T * qb + il
+            if i >= S:
+                break
+            for c in C[:sc]:
+                if c <= i:
+                    assert (i, int(c)) not in cells
+                    cells.add((i, int(c)))
+    return cells
+
+
+def _case2_cells(diags_h, verts_h, tm_h, L, S):
+    D, Cs = set(np.asarray(diags_h).tolist()), set(np.asarray(verts_h).tolist())
+    out = set()
+    for i in range(S):
+        for j in range(i + 1):
+            if i < L:
+                if tm_h[i, j]:
+                    out.add((i, j))
+            elif (i - j) in D or j in Cs:
+                out.add((i, j))
+    return out
+
+
+@pytest.mark.parametrize("L,S", [(128, 300), (200, 300), (256, 256), (100, 90), (300, 700)])
+def test_case2_plan_retains_exactly_the_case2_cells(ora, L, S):
+    rng = np.random.default_rng(L + S)
+    diags = [np.array([0, 3, 40, 129]), np.array([1, 2, 255])]
+    verts = [np.array([5, 130, 260]), np.array([0, 200])]
+    diags = [d[d < S] for d in diags]
+    verts = [c[c < S] for c in verts]
+    ext = _ext(ora, diags, verts, S)
+    tm = (rng.random((2, L, L)) < 0.25).astype(np.uint8)
+    pl = ora.plan_case2(ext, S, tm)
+    for h in range(2):
+        assert _plan_cells(pl, S, ext, h) == _case2_cells(diags[h], verts[h], tm[h], L, S)
+
+
+def test_case2_plan_with_pattern_block_matches_case_one(ora):
+    # a true mask equal to the patterns' cells: the same cells as the plain plan
+    S, L = 400, 256
+    diags = [np.array([0, 3, 40, 129])]
+    verts = [np.array([5, 130])]
+    ext = _ext(ora, diags, verts, S)
+    pl2 = ora.plan_case2(ext, S, _pattern_block(diags, verts, L))
+    pl1 = ora.plan(ext, S)
+    pl1["tile_bits"] = np.zeros((1, 128, 2), np.uint64)
+    assert _plan_cells(pl2, S, ext, 0) == _plan_cells(pl1, S, ext, 0)
+    # past the first block the plan is the plain one, tile for tile
+    nqb, nL = pl1["nqb"], 2
+    a1, a2 = pl1["tile_ptr"][nL], pl2["tile_ptr"][nL]
+    np.testing.assert_array_equal(pl1["tile_key0"][a1:], pl2["tile_key0"][a2:])
+    np.testing.assert_array_equal(pl1["tile_flags"][a1:], pl2["tile_flags"][a2:])
+    assert (pl2["tile_flags"][:a2] == 2).all() and (pl2["stripe_cnt"][:nL] == 0).all()
