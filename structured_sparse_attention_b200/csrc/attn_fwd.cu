@@ -33,9 +33,11 @@
 //                    then QK^T of region h of the tile at u into the same 64 columns
 //                    (N = 64).  So while the softmax works on region b, the tensor core
 //                    runs region a's PV and the next tile's region-a QK^T: the softmax no
-//                    longer waits for the MMAs of its own tile.  The two issuers run
-//                    independently (an issue order between the slots made each wait for
-//                    the other slot's softmax).
+//                    longer waits for the MMAs of its own tile.  Slot 1's issuer follows
+//                    slot 0's (a bracket issues only once slot 0 has issued the same one;
+//                    slot 0 never waits for slot 1), which staggers the two softmaxes on
+//                    the MUFU without coupling them both ways (a strict alternation made
+//                    each wait for the other slot's softmax).
 //     warps 0-3      softmax of slot 0 (query block 2p), one thread per query row
 //     warps 4-7      softmax of slot 1 (query block 2p+1)
 //                    per region: tcgen05.ld S (64 columns), element mask from the plan
@@ -148,6 +150,7 @@ struct Shared {
     uint32_t kflags[kMaxStages];
     uint32_t tmem_base;
     int abort;
+    int lead;  // brackets issued by slot 0's issuer (slot 1 follows it)
 };
 static_assert(sizeof(Shared) <= 1024, "barrier block too large");
 
@@ -410,6 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sh->mma_drain, 2);
         mbar_init(&sh->softmax_done, 2 * kSlotThreads);
         sh->abort = 0;
+        sh->lead = 0;
         fence_barrier_init();
     }
     if (warp == kWarpMma0) {
@@ -620,6 +624,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         in = !end && (f & f_in(s));
                         if (in && (f & f_first(s)) && !wait(&sh->q_full[s], qcnt & 1)) break;
                     }
+                    // slot 1 follows slot 0: a bracket issues only after slot 0 issued it
+                    if (s == 1 && ok) {
+                        volatile int *lead = &sh->lead;
+                        const int want = 2 * u + h + 1;
+                        if (*lead < want) {
+                            const uint64_t t0 = global_timer_ns();
+                            while (*lead < want) {
+                                if (*abort || static_cast<int64_t>(global_timer_ns() - t0) >= lim) {
+                                    ok = false;
+                                    break;
+                                }
+                            }
+                        }
+                        if (!ok) break;
+                    }
                     // 2. PV of region h of the slot's tile at u-1, then QK^T of region h of the
                     // tile at u
                     tc_fence_after();
@@ -651,6 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // phase of step u-1 (never in the previous one, where it would stand in
                     // for the other slot's PV still reading the stage, and never a phase
                     // ahead of the producer, as for a no-op step that no slot reads).
+                    if (s == 0) *reinterpret_cast<volatile int *>(&sh->lead) = 2 * u + h + 1;
                     if (in) umma_commit(&sh->s_full[s][h]);
                     if (h == 1) {
                         if (pend) {

@@ -9,7 +9,8 @@ tensor pipe executes MMA groups in issue order; a commit completes when every gr
 issued before it has completed.  Each key tile is processed as two key regions (keys
 0-63 and 64-127): per region an S-ready and a P-ready barrier, and one MMA bracket per
 region (PV of that region of the previous tile, QK^T of that region of this tile), so
-region a's MMAs run while the softmax works on region b.
+region a's MMAs run while the softmax works on region b.  Slot 1's issuer issues a bracket
+only after slot 0's issuer has issued the same one (slot 0 never waits for slot 1).
 
 Checked in every run:
   * no deadlock: every role finishes;
@@ -56,7 +57,8 @@ class Sim(Engine):
         self.s_full = [[B(f"s_full{s}{h}", 1) for h in range(2)] for s in range(2)]
         self.p_full = [[B(f"p_full{s}{h}", 1) for h in range(2)] for s in range(2)]
         self.pv_a = [B(f"pv_a{s}", 1) for s in range(2)]
-        self.pv_done = [[], []]  # per slot: completion time of the PV of each region, in order
+        self.pv_done = [[], []]
+        self.lead = 0  # per slot: completion time of the PV of each region, in order
         self.o_full = [B(f"o_full{s}", 1) for s in range(2)]
         self.o_empty = [B(f"o_empty{s}", 1) for s in range(2)]
         self.ring = [None] * RING
@@ -212,6 +214,9 @@ def mma_issuer(sim, s):
                 inn = (not end) and s in fl
                 if inn and fl[s][0]:
                     yield ("wait", sim.q_full[s], qcnt)
+            if s == 1:
+                while sim.lead < 2 * u + h + 1:
+                    yield ("delay", 5)
             if pend:
                 if h == 0 and pfirst:
                     if sim.first_pv[s] > sim.epi_done[s]:
@@ -229,6 +234,8 @@ def mma_issuer(sim, s):
                 if h == 0:
                     sim.consumed.append((s, tile))
                 sim.mma(400, [f"K{u % NK}", f"Q{s}"])
+            if s == 0:
+                sim.lead = 2 * u + h + 1
             if inn:
                 sim.commit(sim.s_full[s][h])
             if h == 1:
