@@ -60,6 +60,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <climits>
 
 #include "common.cuh"
@@ -86,19 +87,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kBoxBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr int64_t kDrainLimitNs = 1000000000LL;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if the max grows by > 256x
-// Exponentials on the FMA pipe: one pair in every kEmuEvery pairs of a row's 128
-// logits is computed by exp2_fma2 instead of the MUFU ex2, which alone would take as
-// long as the tile's MMAs.  Coefficients: degree-4 minimax fit of 2^f on [-1/2, 1/2]
-// (Remez exchange; printed by exp2_poly.py), relative error <= 2.7e-6 in fp32.
-constexpr int kEmuEvery = 0;  // 0: every exponential on the MUFU
-__host__ __device__ constexpr bool emulated_pair(int k) {
-    return kEmuEvery > 0 && (k % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1;
-}
-constexpr float kExp2C0 = 0.9999992847442627f;
-constexpr float kExp2C1 = 0.6931217908859253f;
-constexpr float kExp2C2 = 0.240247443318367f;
-constexpr float kExp2C3 = 0.05591785907745361f;
-constexpr float kExp2C4 = 0.009570102207362652f;
 constexpr size_t kCounterBytes = 256;     // work counter at the start of the workspace
 constexpr int kMaxSmem = 232448;          // 227 KB opt-in per block
 
@@ -184,26 +172,6 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
     return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
            (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
            (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// 2^x for a pair of floats on the FMA pipe (Cody-Waite style reduction): n = rint(x)
-// by adding 1.5 * 2^23, f = x - n in [-1/2, 1/2], 2^f by the minimax polynomial, and 2^n
-// added to the exponent field.  x is clamped to >= -126, so -inf (a masked logit) gives
-// 2^-126 instead of 0; the softmax treats a row whose max stayed -inf as empty.
-__device__ __forceinline__ void exp2_fma2(float x0, float x1, float &p0, float &p1) {
-    const uint64_t x = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-    const uint64_t t = f2_add(x, f2_pack(12582912.0f, 12582912.0f));
-    const uint64_t n = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
-    const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x);
-    uint64_t q = f2_fma(f2_pack(kExp2C4, kExp2C4), f, f2_pack(kExp2C3, kExp2C3));
-    q = f2_fma(q, f, f2_pack(kExp2C2, kExp2C2));
-    q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
-    q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
-    float q0, q1, t0, t1;
-    f2_unpack(q, q0, q1);
-    f2_unpack(t, t0, t1);
-    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
 // Instruction descriptor, kind::f16: bf16 A/B, fp32 accumulate, A K-major.
@@ -925,13 +893,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             float x0, x1;
                             f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), sl2x2, nm2),
                                       x0, x1);
-                            float p0, p1;
-                            if (emulated_pair(k)) {
-                                exp2_fma2(x0, x1, p0, p1);
-                            } else {
-                                p0 = ex2_approx(x0);
-                                p1 = ex2_approx(x1);
-                            }
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                             acc[k & 3] = f2_add(acc[k & 3], f2_pack(p0, p1));
                             const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
                             pk[k] = *reinterpret_cast<const uint32_t *>(&pb);
@@ -1079,16 +1041,24 @@ int launch(const void *Q, const void *K, const void *V, uint16_t *KC, uint16_t *
         mVC = mV;
     }
     SSA_CUDA_TRY(cudaMemsetAsync(p.work_counter, 0, sizeof(int), s));
-    SSA_CUDA_TRY(cudaFuncSetAttribute(sparse_attn_fwd_kernel<D>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-    // setmaxnreg.inc can only draw on the registers the block was launched with: refuse
-    // to launch unless the compiled kernel was given exactly the planned allocation.
-    cudaFuncAttributes fa;
-    SSA_CUDA_TRY(cudaFuncGetAttributes(&fa, sparse_attn_fwd_kernel<D>));
-    if (fa.numRegs != kLaunchRegs) {
-        set_error("sparse_attn_fwd: kernel compiled with %d registers per thread, expected %d",
-                  fa.numRegs, kLaunchRegs);
-        return SSA_ERR_UNSUPPORTED;
+    // Once per device: the shared-memory opt-in, and a check that the compiled kernel was
+    // given exactly the planned register allocation (setmaxnreg.inc can only draw on the
+    // registers the block was launched with).
+    static std::atomic<uint64_t> ready{0};
+    int dev = 0;
+    SSA_CUDA_TRY(cudaGetDevice(&dev));
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0;
+    if (!bit || !(ready.load() & bit)) {
+        SSA_CUDA_TRY(cudaFuncSetAttribute(sparse_attn_fwd_kernel<D>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+        cudaFuncAttributes fa;
+        SSA_CUDA_TRY(cudaFuncGetAttributes(&fa, sparse_attn_fwd_kernel<D>));
+        if (fa.numRegs != kLaunchRegs) {
+            set_error("sparse_attn_fwd: kernel compiled with %d registers per thread, expected %d",
+                      fa.numRegs, kLaunchRegs);
+            return SSA_ERR_UNSUPPORTED;
+        }
+        ready.fetch_or(bit);
     }
     const long long items = static_cast<long long>(p.H) * ((p.nqb + 1) / 2);
     const unsigned grid = static_cast<unsigned>(items < sm_count() ? items : sm_count());

@@ -1,4 +1,4 @@
-"""Coefficients of the FMA-pipe exp2 used by the attention softmax.
+"""Coefficients of the FMA-pipe exp2 of the kernels (common.cuh, exp2_fma2).
 
 Method (Cody and Waite, "Software Manual for the Elementary Functions", 1980: argument
 reduction; Remez exchange for the minimax fit):
@@ -7,7 +7,7 @@ reduction; Remez exchange for the minimax fit):
   2^n is applied by adding n to the exponent field of the polynomial's value.
 
 Run this file to print the coefficients (rounded to fp32) and the error bounds; the
-kernel's constants (attn_fwd.cu, kExp2C*) are its output, and a CPU test checks that
+kernels' constants (common.cuh, kExp2C*) are its output, and a CPU test checks that
 they agree and that the fp32 evaluation meets the bound.
 """
 

@@ -1,6 +1,6 @@
-"""The FMA-pipe exp2 of the attention softmax: constants and error bound (CPU).
+"""The FMA-pipe exp2 of the kernels (the maps' row sums): constants and error bound (CPU).
 
-The kernel's coefficients (attn_fwd.cu, kExp2C0..4) must be exactly what
+The kernels' coefficients (common.cuh, kExp2C0..4) must be exactly what
 csrc/exp2_poly.py derives (Remez minimax of 2^f on [-1/2, 1/2]), and the kernel's fp32
 step sequence (clamp, 1.5 * 2^23 rounding shift, Horner, exponent-field add) must stay
 within 3e-6 relative error of exp2 over the whole input range the softmax produces."""
@@ -19,7 +19,7 @@ import exp2_poly  # noqa: E402
 
 
 def kernel_constants():
-    src = open(os.path.join(CSRC, "attn_fwd.cu")).read()
+    src = open(os.path.join(CSRC, "common.cuh")).read()
     vals = dict(re.findall(r"constexpr float kExp2C(\d) = ([0-9eE+\-.]+)f;", src))
     return np.array([np.float32(vals[str(k)]) for k in range(len(vals))], np.float32)
 
