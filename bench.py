@@ -16,6 +16,7 @@ runs an independent replica (weak scaling), time = max over ranks.
 from __future__ import annotations
 
 import argparse
+import itertools
 import json
 import os
 import subprocess
@@ -85,16 +86,11 @@ def profiled_traffic(workload):
     """DRAM bytes per attention launch from the ncu record of this workload
     (profiles/sparse_attn_fwd_<workload>_dram.json), if the attention sources are still
     the ones it was taken on (else None)."""
-    import hashlib
     path = os.path.join(ROOT, "profiles", f"sparse_attn_fwd_{workload}_dram.json")
     if not os.path.exists(path):
         return None
     rec = json.load(open(path))
-    csrc = os.path.join(ROOT, "structured_sparse_attention_b200", "csrc")
-    h = hashlib.sha256()
-    for f in ("attn_fwd.cu", "common.cuh"):
-        h.update(open(os.path.join(csrc, f), "rb").read())
-    if rec.get("source_sha256_16") != h.hexdigest()[:16]:
+    if rec.get("source_sha256_16") != attn_source_hash():
         return None
     try:
         return float(rec["traffic_bytes_per_launch"])
@@ -226,42 +222,43 @@ def run_capture(args):
 SWEEP_WORKLOADS = {
     "capture-sweep-128maps-l512": (128, 512, 65536),  # maps, L, S of the extended mask
 }
-SWEEP_GRID = {"lam": (0.5, 1.0), "tau": (0.1, 0.2, 0.3, 0.4, 0.5), "mu": (0.6, 0.7, 0.8, 0.9)}
+SWEEP_GRID = {"scaling": ("row", "map"), "lam": (0.0, 0.25, 0.5, 1.0, 2.0), "tau": (0.1, 0.2, 0.3, 0.4, 0.5),
+              "mu": (0.6, 0.7, 0.8, 0.9)}
 
 
 def capture_sweep(capture, planted, S, grid=SWEEP_GRID):
-    """For every (lambda, tau, mu) of `grid`: the kept diagonals and columns per map, the
-    recall and precision of the planted patterns, and the density of the extended mask at
-    S (retained pairs / causal pairs, mean over maps).  `capture(lam, tau, mu)` returns the
-    host CSR lists (diag_ptr, diag_offsets, vert_ptr, vert_cols) of the maps whose planted
-    (diagonals, columns) are `planted`."""
+    """For every (scaling, lambda, tau, mu) of `grid`: the kept diagonals and columns per map,
+    the recall and precision of the planted patterns, and the density of the extended mask
+    at S (retained pairs / causal pairs, mean over maps).  `capture(lam, tau, mu, scaling)`
+    returns the host CSR lists (diag_ptr, diag_offsets, vert_ptr, vert_cols) of the maps
+    whose planted (diagonals, columns) are `planted`; scaling is "row" (each row scaled to
+    [0, 1] by its own causal min and max) or "map" (by the map's), default ("row",)."""
     n = len(planted)
     causal = S * (S + 1) / 2
     rows = []
-    for lam in grid["lam"]:
-        for tau in grid["tau"]:
-            for mu in grid["mu"]:
-                dp, do, vp, vc = (np.asarray(a) for a in capture(lam, tau, mu))
-                diags = [do[dp[m]:dp[m + 1]] for m in range(n)]
-                verts = [vc[vp[m]:vp[m + 1]] for m in range(n)]
-                tp = fp = fn = 0
-                for m in range(n):
-                    pd, pc = set(np.asarray(planted[m][0]).tolist()), set(np.asarray(planted[m][1]).tolist())
-                    kd, kc = set(diags[m].tolist()), set(verts[m].tolist())
-                    tp += len(pd & kd) + len(pc & kc)
-                    fp += len(kd - pd) + len(kc - pc)
-                    fn += len(pd - kd) + len(pc - kc)
-                dens = nnz_per_head(diags, verts, S) / causal
-                rows.append({"lam": lam, "tau": tau, "mu": mu,
-                             "diags_per_map": float(np.mean([len(x) for x in diags])),
-                             "cols_per_map": float(np.mean([len(x) for x in verts])),
-                             "recall": tp / max(tp + fn, 1), "precision": tp / max(tp + fp, 1),
-                             "density_at_S": float(dens.mean())})
+    for scaling, lam, tau, mu in itertools.product(grid.get("scaling", ("row",)), grid["lam"], grid["tau"],
+                                                   grid["mu"]):
+        dp, do, vp, vc = (np.asarray(a) for a in capture(lam, tau, mu, scaling))
+        diags = [do[dp[m]:dp[m + 1]] for m in range(n)]
+        verts = [vc[vp[m]:vp[m + 1]] for m in range(n)]
+        tp = fp = fn = 0
+        for m in range(n):
+            pd, pc = set(np.asarray(planted[m][0]).tolist()), set(np.asarray(planted[m][1]).tolist())
+            kd, kc = set(diags[m].tolist()), set(verts[m].tolist())
+            tp += len(pd & kd) + len(pc & kc)
+            fp += len(kd - pd) + len(kc - pc)
+            fn += len(pd - kd) + len(pc - kc)
+        dens = nnz_per_head(diags, verts, S) / causal
+        rows.append({"scaling": scaling, "lam": lam, "tau": tau, "mu": mu,
+                     "diags_per_map": float(np.mean([len(x) for x in diags])),
+                     "cols_per_map": float(np.mean([len(x) for x in verts])),
+                     "recall": tp / max(tp + fn, 1), "precision": tp / max(tp + fp, 1),
+                     "density_at_S": float(dens.mean())})
     return rows
 
 
 def run_capture_sweep(args):
-    """Time the library's capture over the (lambda, tau, mu) grid on synthetic averaged maps
+    """Time the library's capture over the (scaling, lambda, tau, mu) grid on synthetic averaged maps
     and report what each setting keeps (one JSON line; the capture kernels are HBM-bound)."""
     import torch
 
@@ -278,14 +275,15 @@ def run_capture_sweep(args):
     out = ssa.capture(maps, ws=ws, status=status)
     times = []
 
-    def capture(lam, tau, mu):
+    def capture(lam, tau, mu, scaling):
         for _ in range(args.warmup):
-            ssa.capture(maps, lam=lam, tau=tau, mu=mu, out=out, ws=ws, status=status)
+            ssa.capture(maps, lam=lam, tau=tau, mu=mu, scaling=scaling, out=out, ws=ws, status=status)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(args.steps):
-            ssa.capture(maps, lam=lam, tau=tau, mu=mu, out=out, ws=ws, status=status, check=False)
+            ssa.capture(maps, lam=lam, tau=tau, mu=mu, scaling=scaling, out=out, ws=ws, status=status,
+                        check=False)
         e1.record()
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1) / args.steps)

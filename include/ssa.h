@@ -122,7 +122,10 @@ SSA_API size_t sparse_pattern_capture_ws_bytes(int n_maps, int L);
  *   vert_cols    device int32 [n_maps * L]   kept c, ascending within each map
  *   ws           device workspace of at least sparse_pattern_capture_ws_bytes()
  * A negative or non-finite map entry sets SSA_ERR_INVALID in dev_status; the lists
- * are then unspecified.
+ * are then unspecified.  When maps is 16-byte aligned and L a multiple of 4, rows are
+ * staged into shared memory by bulk copies whose waits are bounded
+ * (ssa_set_wait_limit_ns): an expired wait sets SSA_ERR_TIMEOUT in dev_status, the
+ * kernel waits (again bounded) for its copies in flight and the lists are unspecified.
  */
 SSA_API int sparse_pattern_capture(const float *maps, int n_maps, int L, double lambda, double tau,
                            double mu, double eps, int32_t *diag_ptr, int32_t *diag_offsets,
@@ -390,11 +393,12 @@ SSA_API const char *ssa_last_error(void);
 SSA_API int ssa_version(void);
 
 /*
- * Time limit, in nanoseconds, of every bounded wait inside the attention kernel
- * (default 2e9; 0 makes a wait give up at its first unsuccessful poll).  When a wait
- * expires the kernel writes SSA_ERR_TIMEOUT to dev_status, drains its own copies and
- * tensor-core work in flight, frees its tensor memory and returns.  Process-wide;
- * meant for fault-handling tests.  Returns the previous value.
+ * Time limit, in nanoseconds, of every bounded wait inside the kernels that wait on
+ * copies or tensor-core work (attention, averaged maps, capture; default 2e9; 0 makes a
+ * wait give up at its first unsuccessful poll).  When a wait expires the kernel writes
+ * SSA_ERR_TIMEOUT to dev_status, drains its own copies and tensor-core work in flight,
+ * frees its tensor memory and returns.  Process-wide; meant for fault-handling tests.
+ * Returns the previous value.
  */
 SSA_API int64_t ssa_set_wait_limit_ns(int64_t ns);
 

@@ -139,3 +139,21 @@ def test_capture_true_mask_bitmap_matches_oracle(ora, L):
         vp = out["vert_ptr"].cpu().numpy()
         _same((dp, out["diag_offsets"].cpu().numpy()[:dp[-1]], vp, out["vert_cols"].cpu().numpy()[:vp[-1]]),
               ora.capture(maps, tau=tau, scaling=scaling))
+
+
+@pytest.mark.parametrize("scaling", ["row", "map"])
+def test_capture_unaligned_maps_take_the_direct_loads(ora, scaling):
+    # maps whose base is 4 bytes past a 16-byte boundary: rows are not staged by bulk
+    # copies (they need 16-byte aligned rows) but loaded directly; same lists either way
+    import structured_sparse_attention_b200 as ssa
+    n, L = 5, 512
+    maps = inputs.averaged_maps(41, n, L=L, n_samples=2)
+    buf = torch.zeros(n * L * L + 4, dtype=torch.float32, device="cuda:0")
+    view = buf[1:1 + n * L * L].view(n, L, L)
+    view.copy_(torch.from_numpy(maps))
+    assert view.data_ptr() % 16 == 4
+    out = ssa.capture(view, scaling=scaling)
+    dp, vp = out["diag_ptr"].cpu().numpy(), out["vert_ptr"].cpu().numpy()
+    got = (dp, out["diag_offsets"].cpu().numpy()[:dp[-1]], vp, out["vert_cols"].cpu().numpy()[:vp[-1]])
+    _same(got, ora.capture(maps, scaling=scaling))
+    _same(got, _run(maps, scaling=scaling))
