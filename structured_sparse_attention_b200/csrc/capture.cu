@@ -484,14 +484,13 @@ __global__ void __launch_bounds__(kCaptureThreads, 3)
             }
         }
     }
-    if (BULK && s_abort) {
+    __syncthreads();
+    if (BULK && s_abort && threadIdx.x == 0) {
         // a row copy did not land within the wait limit: wait (again bounded) for every
         // copy of this CTA before it may exit
-        if (threadIdx.x == 0)
-            for (int r = 0; r < R; ++r)
-                if (!mbar_wait(&s_bar[r], 0, p.wait_ns, nullptr)) break;
+        for (int r = 0; r < R; ++r)
+            if (!mbar_wait(&s_bar[r], 0, p.wait_ns, nullptr)) break;
     }
-    __syncthreads();
     if (threadIdx.x == 0 && s_bad) report(p.status, SSA_ERR_INVALID);
     if (s_abort) return;
     int32_t *hits = p.hits + static_cast<size_t>(m) * 2 * L;
