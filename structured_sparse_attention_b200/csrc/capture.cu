@@ -216,6 +216,14 @@ __device__ __forceinline__ void bulk_load_1d(void *dst, const void *src, uint32_
         : "memory");
 }
 
+// Bounded wait for a staged row: a non-blocking test first (a limit of 0 gives up when it
+// fails), then sleeping in try_wait until the limit.
+__device__ __forceinline__ bool row_wait(uint64_t *bar, uint32_t parity, int64_t limit_ns, volatile int *abort) {
+    if (mbar_test(bar, parity)) return true;
+    if (limit_ns <= 0) return false;
+    return mbar_wait(bar, parity, limit_ns, abort);
+}
+
 // Bit t of the low byte of x moved to bit 4t.
 __device__ __forceinline__ uint32_t spread4(uint32_t x) {
     x &= 0xffu;
@@ -233,6 +241,10 @@ __device__ __forceinline__ int snake_row(int t, int warp) {
     return kCaptureWarps * t + ((t & 1) ? kCaptureWarps - 1 - warp : warp);
 }
 constexpr int kHitsMaxRows = 128;
+// Limit of each wait for a copy still in flight after a timeout (independent of the
+// wait-limit knob, which may be 0): the CTA must not exit while a copy can still land
+// in its shared memory.
+constexpr int64_t kHitsDrainLimitNs = 1000000000LL;
 __host__ __device__ __forceinline__ int round4(int x) { return (x + 3) & ~3; }
 
 // Shared-memory bytes of a hits CTA whose rows hold `row_floats` floats in total.
@@ -338,7 +350,7 @@ __global__ void __launch_bounds__(kCaptureThreads, 3)
         if (r >= R) break;
         const int i = chunk + p.row_chunks * r, n = i + 1;
         if (BULK) {
-            const bool ok = mbar_wait(&s_bar[r], 0, p.wait_ns, &s_abort);
+            const bool ok = row_wait(&s_bar[r], 0, p.wait_ns, &s_abort);
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) {
                     s_abort = 1;
@@ -489,7 +501,7 @@ __global__ void __launch_bounds__(kCaptureThreads, 3)
         // a row copy did not land within the wait limit: wait (again bounded) for every
         // copy of this CTA before it may exit
         for (int r = 0; r < R; ++r)
-            if (!mbar_wait(&s_bar[r], 0, p.wait_ns, nullptr)) break;
+            if (!mbar_wait(&s_bar[r], 0, kHitsDrainLimitNs, nullptr)) break;
     }
     if (threadIdx.x == 0 && s_bad) report(p.status, SSA_ERR_INVALID);
     if (s_abort) return;
