@@ -633,12 +633,15 @@ def run_gpu(args, rank, world, local, dist):
                 "frac": achieved / hbm_gbs}
     traffic = args.traffic if args.traffic is not None else profiled_traffic(args.workload)
     roof.update({"traffic": traffic, "traffic_source": ("command line" if args.traffic is not None else
-                 "profiles/ summary (dram__bytes_read.sum + dram__bytes_write.sum, one launch)" if traffic else None),
+                 f"profiles/sparse_attn_fwd_{args.workload}_dram.json (dram__bytes_read.sum + dram__bytes_write.sum "
+                 "per launch, ncu)" if traffic else None),
                  "kernel": "sparse_attn_fwd (stripe gather + attention kernel)",
                  "peak_source": f"{peak_kind} ({'burst' if bound == 'tensor' else 'copy'})",
                  "algorithmic": {"flops": flops, "bytes": algo_bytes},
                  "roofline_ms": max(t_tensor, t_hbm, t_mufu) * 1e3,
                  "frac_of_roofline_time": max(t_tensor, t_hbm, t_mufu) * 1e3 / attn_ms,
+                 # against the slower of the tensor and HBM bounds alone (no MUFU bound)
+                 "frac_of_tensor_hbm_bound": max(t_tensor, t_hbm) * 1e3 / attn_ms,
                  "bounds_ms": {"tensor": t_tensor * 1e3, "hbm": t_hbm * 1e3, "mufu": t_mufu * 1e3}})
 
     line = {
