@@ -64,6 +64,7 @@
 #include <climits>
 
 #include "common.cuh"
+#include "trace.h"
 
 namespace ssa {
 namespace {
@@ -1084,6 +1085,7 @@ extern "C" int sparse_attn_fwd(const void *Q, const void *K, const void *V, int 
                                int S, int d, const ssa_plan *plan, const int32_t *kv_map,
                                float scale, void *O, float *LSE, void *ws, size_t ws_bytes,
                                int32_t *dev_status, void *stream) {
+    ssa::TraceRange trace_range("sparse_attn_fwd");
     SSA_CHECK_ARG(Q && K && V && O && LSE && plan, "sparse_attn_fwd: null pointer argument");
     if (d != 64 && d != 128) {
         set_error("sparse_attn_fwd: head dimension must be 64 or 128 (got %d)", d);

@@ -28,6 +28,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "trace.h"
 
 namespace ssa {
 namespace {
@@ -711,6 +712,7 @@ extern "C" int sparse_pattern_capture_ex(const float *maps, int n_maps, int L, d
                                          int32_t *vert_ptr, int32_t *vert_cols,
                                          uint32_t *true_mask, void *ws, size_t ws_bytes,
                                          int32_t *dev_status, void *stream) {
+    ssa::TraceRange trace_range("sparse_pattern_capture_ex");
     SSA_CHECK_ARG(maps && diag_ptr && diag_offsets && vert_ptr && vert_cols && ws,
                   "sparse_pattern_capture: null pointer argument");
     SSA_CHECK_ARG(n_maps >= 1, "sparse_pattern_capture: n_maps must be >= 1 (got %d)", n_maps);
@@ -880,6 +882,7 @@ extern "C" int sparse_pattern_capture_noalloc(const float *maps, int n_maps, int
                                               int32_t *diag_offsets, int32_t *vert_ptr,
                                               int32_t *vert_cols, int32_t *dev_status,
                                               void *stream) {
+    ssa::TraceRange trace_range("sparse_pattern_capture_noalloc");
     SSA_CHECK_ARG(n_maps >= 1 && L >= 1, "sparse_pattern_capture_noalloc: n_maps and L must be >= 1");
     const size_t need = sparse_pattern_capture_ws_bytes(n_maps, L);
     if (need > kNoAllocScratchBytes) {

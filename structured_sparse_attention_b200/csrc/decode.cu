@@ -25,6 +25,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "trace.h"
 
 namespace ssa {
 namespace {
@@ -280,6 +281,7 @@ extern "C" int sparse_attn_decode(const void *Q, const void *K, const void *V, i
                                   const ssa_plan *plan, const int32_t *kv_map, float scale,
                                   void *O, float *LSE, void *ws, size_t ws_bytes,
                                   int32_t *dev_status, void *stream) {
+    ssa::TraceRange trace_range("sparse_attn_decode");
     SSA_CHECK_ARG(Q && K && V && pos && plan && O && LSE && ws,
                   "sparse_attn_decode: null pointer argument");
     if (d != 64 && d != 128) {

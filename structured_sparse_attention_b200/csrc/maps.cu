@@ -35,6 +35,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "trace.h"
 
 namespace ssa {
 namespace {
@@ -574,6 +575,7 @@ using namespace ssa;
 
 extern "C" int sparse_attn_maps(const void *Q, const void *K, int n_maps, int B, int L, int d, float scale,
                                 float *maps, int32_t *dev_status, void *stream) {
+    ssa::TraceRange trace_range("sparse_attn_maps");
     SSA_CHECK_ARG(Q && K && maps, "sparse_attn_maps: null pointer argument");
     if (d != 64 && d != 128) {
         set_error("sparse_attn_maps: head dimension must be 64 or 128 (got %d)", d);

@@ -19,6 +19,7 @@
 //   plan_tiles_kernel      count pass / fill pass of the band windows + stripe counts
 //   plan_totals_kernel     totals for the sizing pass
 #include "common.cuh"
+#include "trace.h"
 
 namespace ssa {
 namespace {
@@ -588,6 +589,7 @@ extern "C" int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr,
                                      const int32_t *vert_cols, int S, ssa_plan_sizes *sizes,
                                      const ssa_plan *plan, void *ws, size_t ws_bytes,
                                      int32_t *dev_status, void *stream) {
+    ssa::TraceRange trace_range("sparse_pattern_extend");
     return extend_impl(n_heads, diag_ptr, diag_offsets, vert_ptr, vert_cols, nullptr, 0, S, sizes, plan, ws,
                        ws_bytes, dev_status, stream);
 }
@@ -597,6 +599,7 @@ extern "C" int sparse_pattern_extend_case2(int n_heads, const int32_t *diag_ptr,
                                            const int32_t *vert_cols, const uint32_t *true_mask, int L,
                                            int S, ssa_plan_sizes *sizes, const ssa_plan *plan, void *ws,
                                            size_t ws_bytes, int32_t *dev_status, void *stream) {
+    ssa::TraceRange trace_range("sparse_pattern_extend_case2");
     SSA_CHECK_ARG(true_mask, "sparse_pattern_extend_case2: null true_mask");
     SSA_CHECK_ARG(L >= 1 && L <= 1024, "sparse_pattern_extend_case2: L must be in [1, 1024] (got %d)", L);
     SSA_CHECK_ARG((reinterpret_cast<uintptr_t>(true_mask) & 3u) == 0,
