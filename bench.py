@@ -539,6 +539,38 @@ def run_gpu(args, rank, world, local, dist):
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during timing")
 
+    # ---------------- the same path step, captured once into a CUDA graph and replayed ----------------
+    # (13 launches per step: the replay removes the host launch overhead between them)
+    g_ms_local, g_err = float("nan"), None
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            path_step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            path_step()
+        graph.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        g_ms_local = g0.elapsed_time(g1) / args.steps
+        del graph
+    except RuntimeError as exc:  # capture unsupported here: reported, the rest still runs
+        g_err = str(exc).splitlines()[0][:200]
+    g_ms = max_over_ranks(g_ms_local, dist, dev)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during the graph replays")
+    path_graph = ({"error": g_err} if g_err is not None else
+                  {"what": "the same path step captured once into a CUDA graph and replayed",
+                   "ms_per_step": g_ms, "tokens_per_s": world * S / (g_ms / 1e3)})
+
     # ---------------- end-to-end through the public API with host buffers ----------------
     e2e = None
     if not args.no_e2e:
@@ -658,7 +690,7 @@ def run_gpu(args, rank, world, local, dist):
                  "ms_per_step": path_ms, "tokens_per_s": world * S / (path_ms / 1e3),
                  "stages_ms": {"capture": stage_ms["cap"], "extend_fill": stage_ms["ext"],
                                "attn_fwd": stage_ms["attn"]},
-                 "gpu_launches_per_step": sum(LAUNCHES.values())},
+                 "gpu_launches_per_step": sum(LAUNCHES.values()), "graph": path_graph},
         "effective_tflops": flops / (attn_ms / 1e3) / 1e12,
         "roofline": roof,
         "clocks": clocks,
