@@ -246,6 +246,13 @@ typedef struct ssa_plan {
     /* Case-2 plans only (sparse_pattern_extend_case2; zero / NULL otherwise): */
     int32_t bitmap_slots; /* from ssa_plan_sizes */
     uint64_t *tile_bits;  /* [n_heads * bitmap_slots][128][2] (uint64), 16-byte aligned */
+    /* Capacities of ext_diag_offsets and ext_vert_cols (n_diag, n_vert from
+     * ssa_plan_sizes).  A fill pass whose extended lists need more (in total, or more
+     * than max_vert columns for one head) changes nothing in the plan and reports
+     * SSA_ERR_CAPACITY in dev_status; the tile arrays are checked against n_tiles the
+     * same way. */
+    int32_t n_diag;
+    int32_t n_vert;
 } ssa_plan;
 
 /* Workspace bytes of either pass of sparse_pattern_extend (about 4 * n_heads * S for

@@ -52,7 +52,8 @@ class PlanStruct(C.Structure):
                 ("ext_vert_ptr", C.c_void_p), ("ext_vert_cols", C.c_void_p),
                 ("tile_ptr", C.c_void_p), ("tile_key0", C.c_void_p), ("tile_dmask", C.c_void_p),
                 ("tile_cmask", C.c_void_p), ("tile_flags", C.c_void_p), ("stripe_cnt", C.c_void_p),
-                ("bitmap_slots", C.c_int32), ("tile_bits", C.c_void_p)]
+                ("bitmap_slots", C.c_int32), ("tile_bits", C.c_void_p),
+                ("n_diag", C.c_int32), ("n_vert", C.c_int32)]
 
 
 _lib = None
@@ -232,6 +233,7 @@ class Plan:
         st = PlanStruct()
         st.n_heads, st.S, st.nqb, st.max_vert = H, sizes.S, nqb, sizes.max_vert
         st.n_tiles = int(sizes.n_tiles)
+        st.n_diag, st.n_vert = int(sizes.n_diag), int(sizes.n_vert)
         for name in ("ext_diag_ptr", "ext_diag_offsets", "ext_vert_ptr", "ext_vert_cols", "tile_ptr",
                      "tile_key0", "tile_dmask", "tile_cmask", "tile_flags", "stripe_cnt"):
             setattr(st, name, getattr(self, name).data_ptr())

@@ -18,6 +18,9 @@
 //                          holding each kept diagonal
 //   plan_tiles_kernel      count pass / fill pass of the band windows + stripe counts
 //   plan_totals_kernel     totals for the sizing pass
+//   plan_check_kernel      fill pass: the lists fit the plan's capacities, else every
+//                          later kernel of the pass returns at once (the plan keeps its
+//                          previous content) and SSA_ERR_CAPACITY is reported
 #include "common.cuh"
 #include "trace.h"
 
@@ -33,6 +36,7 @@ struct Totals {  // device-side result of the sizing pass
     int32_t n_vert;
     int32_t max_vert;
     int64_t n_tiles;
+    int32_t abort;  // fill pass: the lists do not fit the plan; the rest of the pass is skipped
 };
 
 struct PlanParams {
@@ -48,6 +52,7 @@ struct PlanParams {
     int32_t *dev_status;
     // fill pass outputs
     int64_t capacity;
+    int32_t cap_diag, cap_vert, cap_max_vert;  // list capacities of the plan
     int32_t *tile_key0;
     uint64_t *tile_dmask;
     uint64_t *tile_cmask;
@@ -87,9 +92,11 @@ __global__ void validate_lists_kernel(PlanParams p) {
     }
 }
 
-// out[k] = sum_{k' < k} in[k' * stride + offset] for k in [0, n]; one block.
+// out[k] = sum_{k' < k} in[k' * stride + offset] for k in [0, n]; one block.  Nothing
+// is written when *abort is set (abort may be null).
 __global__ void __launch_bounds__(kScanThreads)
-    exclusive_scan_kernel(const int32_t *in, int n, int stride, int offset, int32_t *out) {
+    exclusive_scan_kernel(const int32_t *in, int n, int stride, int offset, int32_t *out, const int32_t *abort) {
+    if (abort && *abort) return;
     __shared__ int32_t s_warp[kScanThreads / 32];
     __shared__ int32_t s_carry;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -121,6 +128,7 @@ __global__ void __launch_bounds__(kScanThreads)
 }
 
 __global__ void extend_copy_kernel(PlanParams p) {
+    if (p.totals->abort) return;
     const int h = blockIdx.x;
     const int32_t *D = p.doff + p.dptr[h];
     const int32_t *C = p.vcol + p.vptr[h];
@@ -145,6 +153,7 @@ __global__ void extend_copy_kernel(PlanParams p) {
 __global__ void __launch_bounds__(kScanThreads) run_start_kernel(PlanParams p) {
     __shared__ int32_t s_warp[kScanThreads / 32];
     __shared__ int32_t s_carry;
+    if (p.totals->abort) return;
     const int h = blockIdx.x;
     const int32_t *D = p.doff + p.dptr[h];
     const int nd = p.ext_counts[2 * h];
@@ -331,7 +340,7 @@ template <bool FILL>
 __global__ void __launch_bounds__(128) plan_tiles_kernel(PlanParams p) {
     const int item = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (item >= p.H * p.nqb) return;
+    if (item >= p.H * p.nqb || p.totals->abort) return;
     const int h = item / p.nqb, qb = item % p.nqb;
     const int32_t *D = p.doff + p.dptr[h];
     const int32_t *C = p.vcol + p.vptr[h];
@@ -392,6 +401,26 @@ __global__ void __launch_bounds__(128) plan_tiles_kernel(PlanParams p) {
         k = ks - 1;
     }
     if (!FILL && lane == 0) p.tile_counts[item] = count;
+}
+
+// Fill pass: the extended lists must fit the plan's arrays (sized by an earlier sizing
+// pass): total diagonals, total columns, and each head's columns within max_vert (the
+// attention workspace's stripe buffers).  Otherwise the rest of the pass is skipped.
+__global__ void __launch_bounds__(256) plan_check_kernel(PlanParams p) {
+    __shared__ int s_bad;
+    if (threadIdx.x == 0) s_bad = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int h = threadIdx.x; h < p.H; h += blockDim.x) bad |= p.ext_counts[2 * h + 1] > p.cap_max_vert;
+    if (bad) s_bad = 1;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int nd = p.ext_scan[p.H], nc = p.ext_scan[(p.H + 1) + p.H];
+        if (s_bad || nd > p.cap_diag || nc > p.cap_vert) {
+            p.totals->abort = 1;
+            report(p.dev_status, SSA_ERR_CAPACITY);
+        }
+    }
 }
 
 __global__ void plan_totals_kernel(PlanParams p) {
@@ -511,7 +540,7 @@ int extend_impl(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offset
         SSA_LAUNCH_CHECK();
         plan_tiles_kernel<false><<<tile_grid, 128, 0, s>>>(p);
         SSA_LAUNCH_CHECK();
-        exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.tile_counts, items, 1, 0, p.tile_ptr);
+        exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.tile_counts, items, 1, 0, p.tile_ptr, nullptr);
         SSA_LAUNCH_CHECK();
         plan_totals_kernel<<<1, 1024, 0, s>>>(p);
         SSA_LAUNCH_CHECK();
@@ -550,8 +579,13 @@ int extend_impl(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offset
                       slots);
         p.tile_bits = plan->tile_bits;
     }
+    SSA_CHECK_ARG(plan->n_diag >= 0 && plan->n_vert >= 0 && plan->max_vert >= 0,
+                  "sparse_pattern_extend: negative list capacity in the plan");
     p.tile_ptr = plan->tile_ptr;
     p.capacity = plan->n_tiles;
+    p.cap_diag = plan->n_diag;
+    p.cap_vert = plan->n_vert;
+    p.cap_max_vert = plan->max_vert;
     p.tile_key0 = plan->tile_key0;
     p.tile_dmask = plan->tile_dmask;
     p.tile_cmask = plan->tile_cmask;
@@ -564,10 +598,12 @@ int extend_impl(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offset
 
     validate_lists_kernel<<<n_heads, 128, 0, s>>>(p);
     SSA_LAUNCH_CHECK();
-    exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.ext_counts, n_heads, 2, 0, p.ext_scan);
+    exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.ext_counts, n_heads, 2, 0, p.ext_scan, nullptr);
     SSA_LAUNCH_CHECK();
     exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.ext_counts, n_heads, 2, 1,
-                                                     p.ext_scan + (n_heads + 1));
+                                                     p.ext_scan + (n_heads + 1), nullptr);
+    SSA_LAUNCH_CHECK();
+    plan_check_kernel<<<1, 256, 0, s>>>(p);
     SSA_LAUNCH_CHECK();
     extend_copy_kernel<<<n_heads, 128, 0, s>>>(p);
     SSA_LAUNCH_CHECK();
@@ -575,7 +611,7 @@ int extend_impl(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offset
     SSA_LAUNCH_CHECK();
     plan_tiles_kernel<false><<<tile_grid, 128, 0, s>>>(p);
     SSA_LAUNCH_CHECK();
-    exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.tile_counts, items, 1, 0, p.tile_ptr);
+    exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.tile_counts, items, 1, 0, p.tile_ptr, &p.totals->abort);
     SSA_LAUNCH_CHECK();
     plan_tiles_kernel<true><<<tile_grid, 128, 0, s>>>(p);
     SSA_LAUNCH_CHECK();

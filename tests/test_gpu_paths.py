@@ -71,3 +71,82 @@ def test_case2_gqa_per_map_scaling(ora):
     O, LSE = ssa.attn_fwd(t_bf16(q), t_bf16(k), t_bf16(v), plan)
     Oref, Lref = ora.attn_dense_case2(q, k, v, ext, d ** -0.5, tm)
     compare_attn(O, LSE, Oref, Lref)
+
+
+def test_path_replayed_from_cuda_graph_matches_eager(ora):
+    # capture -> extension fill pass -> attention, captured once into a CUDA graph: every
+    # call is capture-safe (no host synchronisation), and a replay on new queries gives
+    # exactly the eager results, which match the oracle
+    L, S, H, d = 256, 2048, 4, 64
+    maps_h = inputs.averaged_maps(inputs.SEED_BASE + 80, H, L=L, n_samples=3)
+    q_a, k_h, v_h = inputs.qkv(inputs.SEED_BASE + 82, H, H, S, d)
+    q_b = inputs.qkv(inputs.SEED_BASE + 83, H, H, S, d)[0]
+    maps = torch.from_numpy(maps_h).to(dev())
+    q, k, v = t_bf16(q_a), t_bf16(k_h), t_bf16(v_h)
+    cap = ssa.capture(maps)
+    ws = torch.empty(max(ssa.load().sparse_pattern_capture_ws_bytes(H, L), 16), dtype=torch.uint8, device=dev())
+    plan = ssa.extend(cap["diag_ptr"], cap["diag_offsets"], cap["vert_ptr"], cap["vert_cols"], S)
+    O = torch.empty_like(q)
+    LSE = torch.empty((H, S), dtype=torch.float32, device=dev())
+    aws = torch.empty(max(ssa.attn_ws_bytes(plan, d), 16), dtype=torch.uint8, device=dev())
+    status = torch.zeros(1, dtype=torch.int32, device=dev())
+
+    def step():
+        ssa.capture(maps, out=cap, ws=ws, status=status, check=False)
+        ssa.refill(plan, cap["diag_ptr"], cap["diag_offsets"], cap["vert_ptr"], cap["vert_cols"], status=status)
+        ssa.attn_fwd(q, k, v, plan, out=O, lse=LSE, ws=aws, status=status, check=False)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    q.copy_(t_bf16(q_b))  # new queries, same maps: the replay recomputes the whole path
+    graph.replay()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    O_g, L_g = O.clone(), LSE.clone()
+    step()
+    torch.cuda.synchronize()
+    assert torch.equal(O_g, O) and torch.equal(L_g, LSE)
+    ext = ora.extend(*ora.capture(maps_h), S)
+    Oref, Lref = ora.attn_dense(q_b, k_h, v_h, ext, d ** -0.5)
+    compare_attn(O_g, L_g, Oref, Lref)
+    del graph
+
+
+def test_refill_beyond_the_plan_reports_capacity(ora):
+    # a fill pass whose lists need more than the plan was sized for changes nothing in the
+    # plan and reports SSA_ERR_CAPACITY (-3): more diagonals in total, then more columns
+    # for one head than the plan's max_vert
+    from gpu_util import lists_to_device
+    S, d = 1024, 64
+    diags = [np.arange(0, 40, dtype=np.int32), np.array([0, 7], np.int32)]
+    verts = [np.array([3, 99], np.int32), np.array([5], np.int32)]
+    dev_lists, host = lists_to_device(diags, verts)
+    plan = ssa.extend(*dev_lists, S)
+    before = plan.to_numpy()
+    bigger = [
+        ([np.arange(0, 90, dtype=np.int32), np.array([0, 7], np.int32)], verts),
+        (diags, [np.array([3, 99], np.int32), np.array([5, 6, 9], np.int32)]),
+    ]
+    for dg, vt in bigger:
+        status = torch.zeros(1, dtype=torch.int32, device=dev())
+        lists_b, _ = lists_to_device(dg, vt)
+        ssa.refill(plan, *lists_b, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == -3
+        after = plan.to_numpy()
+        for key in before:
+            pairs = zip(before[key], after[key]) if key == "ext" else [(before[key], after[key])]
+            for a, b in pairs:
+                np.testing.assert_array_equal(a, b, err_msg=key)
+    # the plan still serves the lists it was sized for
+    q, k, v = inputs.qkv(inputs.SEED_BASE + 90, 2, 2, S, d)
+    O, LSE = ssa.attn_fwd(t_bf16(q), t_bf16(k), t_bf16(v), plan)
+    Oref, Lref = ora.attn_dense(q, k, v, ora.extend(*host, S), d ** -0.5)
+    compare_attn(O, LSE, Oref, Lref)
