@@ -88,6 +88,18 @@ def test_host_argument_checks(lib):
     assert rc == -1
 
 
+def test_decode_rejects_case2_plans_before_any_device_work(lib):
+    # element-bitmap tiles are a prefill-only plan form: decoding says so on the host
+    from structured_sparse_attention_b200 import binding
+    dummy = C.c_void_p(256)
+    plan = binding.PlanStruct()
+    plan.S, plan.n_heads, plan.nqb, plan.bitmap_slots = 256, 1, 2, 3
+    pos = C.c_void_p(256)
+    rc = lib.sparse_attn_decode(dummy, dummy, dummy, 1, 1, 1, 256, 64, pos, C.byref(plan), None, 0.1, dummy,
+                                dummy, dummy, 1 << 20, None, None)
+    assert rc == -2 and b"Case-2" in lib.ssa_last_error()
+
+
 def test_wait_limit_knob(lib):
     old = lib.ssa_set_wait_limit_ns(12345)
     assert lib.ssa_set_wait_limit_ns(old) == 12345
