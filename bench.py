@@ -35,7 +35,7 @@ METRIC = "sparse-attn prefill tokens/s & effective TFLOP/s vs roofline, per mask
 UNIT = "tokens/s"
 
 # Kernels launched per call (the library's own kernels).
-LAUNCHES = {"capture": 3, "extend_fill": 8, "attn": 2}
+LAUNCHES = {"capture": 3, "extend_fill": 9, "attn": 2}  # library kernels per call of each stage
 
 WORKLOADS = {
     # name: (H_q, H_kv, S, d, pattern builder)
@@ -540,7 +540,7 @@ def run_gpu(args, rank, world, local, dist):
         raise RuntimeError(f"device status {int(status.item())} during timing")
 
     # ---------------- the same path step, captured once into a CUDA graph and replayed ----------------
-    # (13 launches per step: the replay removes the host launch overhead between them)
+    # (14 launches per step: the replay removes the host launch overhead between them)
     g_ms_local, g_err = float("nan"), None
     try:
         side = torch.cuda.Stream()
