@@ -93,7 +93,10 @@ __global__ void validate_lists_kernel(PlanParams p) {
 }
 
 // out[k] = sum_{k' < k} in[k' * stride + offset] for k in [0, n]; one block.  Nothing
-// is written when *abort is set (abort may be null).
+// is written when *abort is set (abort may be null).  Chunks of kScanThreads x kScanPer
+// elements: each thread loads kScanPer consecutive elements at once (all loads in flight
+// together), then one block scan of the threads' sums.
+constexpr int kScanPer = 8;
 __global__ void __launch_bounds__(kScanThreads)
     exclusive_scan_kernel(const int32_t *in, int n, int stride, int offset, int32_t *out, const int32_t *abort) {
     if (abort && *abort) return;
@@ -102,10 +105,18 @@ __global__ void __launch_bounds__(kScanThreads)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) s_carry = 0;
     __syncthreads();
-    for (int start = 0; start < n; start += kScanThreads) {
-        const int k = start + threadIdx.x;
-        const int v = k < n ? in[static_cast<size_t>(k) * stride + offset] : 0;
-        int x = v;
+    for (int start = 0; start < n; start += kScanThreads * kScanPer) {
+        const int k0 = start + threadIdx.x * kScanPer;
+        int v[kScanPer];
+#pragma unroll
+        for (int t = 0; t < kScanPer; ++t) {
+            const int k = k0 + t;
+            v[t] = k < n ? in[static_cast<size_t>(k) * stride + offset] : 0;
+        }
+        int sum = 0;
+#pragma unroll
+        for (int t = 0; t < kScanPer; ++t) sum += v[t];
+        int x = sum;  // inclusive scan of the threads' sums within the warp
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -113,15 +124,26 @@ __global__ void __launch_bounds__(kScanThreads)
         }
         if (lane == 31) s_warp[warp] = x;
         __syncthreads();
-        int before = 0, total = 0;
-        for (int w = 0; w < kScanThreads / 32; ++w) {
-            if (w < warp) before += s_warp[w];
-            total += s_warp[w];
+        if (warp == 0) {  // exclusive scan of the warp totals
+            const int w = lane < kScanThreads / 32 ? s_warp[lane] : 0;
+            int y = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int z = __shfl_up_sync(0xffffffffu, y, o);
+                if (lane >= o) y += z;
+            }
+            if (lane < kScanThreads / 32) s_warp[lane] = y - w;
         }
-        const int carry = s_carry;
-        if (k < n) out[k] = carry + before + x - v;
         __syncthreads();
-        if (threadIdx.x == 0) s_carry = carry + total;
+        int run = s_carry + s_warp[warp] + x - sum;  // before this thread's first element
+#pragma unroll
+        for (int t = 0; t < kScanPer; ++t) {
+            const int k = k0 + t;
+            if (k < n) out[k] = run;
+            run += v[t];
+        }
+        __syncthreads();
+        if (threadIdx.x == kScanThreads - 1) s_carry = run;  // the last thread's end: the chunk total
         __syncthreads();
     }
     if (threadIdx.x == 0) out[n] = s_carry;
