@@ -17,14 +17,15 @@
  *     to QK^T / sqrt(d_k) before softmax.
  *   - Referee Report, minor comment 1: the stabiliser eps (1e-8 in the main text).
  * Readings where the page is silent (all listed in the design notes): row-wise
- * min-max scaling of the Box-Cox output before tau; t >= tau and gamma >= mu; a
- * constant row counts as t = 1; masked logits are excluded from the softmax (-inf),
+ * min-max scaling of the Box-Cox output before tau (map-wise as an option); t >= tau
+ * and gamma >= mu; a constant row (or map) counts as t = 1; masked logits are excluded from the softmax (-inf),
  * not multiplied by 0; an empty row gives O = 0 and LSE = -inf; LSE is the natural
  * log-sum-exp of the scaled logits.
  *
- * Parity status: capture follows the reading above (the page gives no worked example,
- * so the min-max reading itself is "parity unpinned" against the paper; the arithmetic
- * is pinned by closed forms and invariants in the tests).
+ * Parity status: capture follows the readings above (the page gives no worked example,
+ * so which min-max reading the paper used is "parity unpinned" against the paper; the
+ * arithmetic of both is pinned by closed forms, hand-derived masks and invariants in
+ * the tests).
  *
  * All floating point is IEEE binary64, built with -ffp-contract=off (no FMA fusion).
  */
