@@ -273,10 +273,14 @@ SSA_API size_t sparse_pattern_extend_ws_bytes(int n_heads, int S);
  *   sizes        host, always filled when plan == NULL (sizing pass)
  *   plan         NULL: sizing pass -- enqueues the counting kernels, copies the
  *                totals to the host and SYNCHRONISES `stream`; returns
- *                SSA_ERR_INVALID if a list is malformed.
+ *                SSA_ERR_INVALID if a list is malformed, SSA_ERR_CAPACITY if the plan
+ *                would hold more than INT32_MAX tiles (tile_ptr is int32).
  *                non-NULL: fill pass -- writes every plan array (no synchronisation);
- *                plan->n_tiles must be >= the sized n_tiles (else SSA_ERR_CAPACITY in
- *                dev_status); plan->n_heads/S/nqb/max_vert must match the sizes.
+ *                the new lists and tiles are counted in the workspace first, and only
+ *                when they fit the plan's capacities (n_diag, n_vert, max_vert,
+ *                n_tiles) is the plan written; otherwise it keeps its previous content
+ *                and SSA_ERR_CAPACITY goes to dev_status.  plan->n_heads/S/nqb must
+ *                match the call.
  *   ws           device workspace of at least sparse_pattern_extend_ws_bytes()
  */
 SSA_API int sparse_pattern_extend(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offsets,

@@ -12,15 +12,20 @@
 //
 // Kernels (one warp per (head, query block) for the tile work)
 //   validate_lists_kernel  lists sorted, unique, non-negative; kept counts r < S, c < S
-//   exclusive_scan_kernel  single-block scan (list offsets, tile offsets)
+//   exclusive_scan_kernel  single-block scan (list offsets, tile offsets; exact 64-bit
+//                          total)
 //   extend_copy_kernel     the extended CSR lists
 //   run_start_kernel       per head: first index of the run (offsets <= 128 apart)
 //                          holding each kept diagonal
 //   plan_tiles_kernel      count pass / fill pass of the band windows + stripe counts
 //   plan_totals_kernel     totals for the sizing pass
-//   plan_check_kernel      fill pass: the lists fit the plan's capacities, else every
-//                          later kernel of the pass returns at once (the plan keeps its
-//                          previous content) and SSA_ERR_CAPACITY is reported
+//   plan_check_kernel      fill pass: the lists and the tiles fit the plan's capacities,
+//                          else the kernels that write the plan return at once (the plan
+//                          keeps its previous content) and SSA_ERR_CAPACITY is reported
+//
+// Fill pass order: everything that sizes the new plan (validation, list scans, run
+// starts, tile counts, tile scan) writes only the workspace; the capacity check follows;
+// only then are the plan's lists and tiles written (tile_ptr by the fill kernel).
 #include "common.cuh"
 #include "trace.h"
 
@@ -35,8 +40,8 @@ struct Totals {  // device-side result of the sizing pass
     int32_t n_diag;
     int32_t n_vert;
     int32_t max_vert;
-    int64_t n_tiles;
-    int32_t abort;  // fill pass: the lists do not fit the plan; the rest of the pass is skipped
+    int64_t n_tiles;  // exact total of the tile scan
+    int32_t abort;    // fill pass: the new plan does not fit; nothing of the plan is written
 };
 
 struct PlanParams {
@@ -46,7 +51,8 @@ struct PlanParams {
     int32_t *ext_scan;     // [2 (H+1)]: exclusive scans of the two count arrays
     int32_t *tile_counts;  // [H*nqb]
     int32_t *run0;         // [H][S]: run start index of each kept diagonal
-    int32_t *tile_ptr;     // [H*nqb + 1] (workspace in the sizing pass, plan in the fill pass)
+    int32_t *tile_pos;     // [H*nqb + 1] workspace: exclusive scan of tile_counts
+    int32_t *tile_ptr;     // [H*nqb + 1] fill pass: the plan's copy of tile_pos
     Totals *totals;
     int32_t *ws_status;
     int32_t *dev_status;
@@ -92,16 +98,20 @@ __global__ void validate_lists_kernel(PlanParams p) {
     }
 }
 
-// out[k] = sum_{k' < k} in[k' * stride + offset] for k in [0, n]; one block.  Nothing
-// is written when *abort is set (abort may be null).  Chunks of kScanThreads x kScanPer
-// elements: each thread loads kScanPer consecutive elements at once (all loads in flight
-// together), then one block scan of the threads' sums.
+// out[k] = sum_{k' < k} in[k' * stride + offset] for k in [0, n] (inputs >= 0); one
+// block.  Sums are taken in 64 bits: out[] holds them clamped to INT32_MAX, and *total
+// (may be null) the exact sum of all n, so that a caller can tell an int32 overflow
+// from a fit.  Chunks of kScanThreads x kScanPer elements: each thread loads kScanPer
+// consecutive elements at once (all loads in flight together), then one block scan of
+// the threads' sums.
 constexpr int kScanPer = 8;
+__device__ __forceinline__ int32_t clamp_i32(int64_t x) {
+    return static_cast<int32_t>(x < INT32_MAX ? x : INT32_MAX);
+}
 __global__ void __launch_bounds__(kScanThreads)
-    exclusive_scan_kernel(const int32_t *in, int n, int stride, int offset, int32_t *out, const int32_t *abort) {
-    if (abort && *abort) return;
-    __shared__ int32_t s_warp[kScanThreads / 32];
-    __shared__ int32_t s_carry;
+    exclusive_scan_kernel(const int32_t *in, int n, int stride, int offset, int32_t *out, int64_t *total) {
+    __shared__ int64_t s_warp[kScanThreads / 32];
+    __shared__ int64_t s_carry;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) s_carry = 0;
     __syncthreads();
@@ -113,40 +123,43 @@ __global__ void __launch_bounds__(kScanThreads)
             const int k = k0 + t;
             v[t] = k < n ? in[static_cast<size_t>(k) * stride + offset] : 0;
         }
-        int sum = 0;
+        int64_t sum = 0;
 #pragma unroll
         for (int t = 0; t < kScanPer; ++t) sum += v[t];
-        int x = sum;  // inclusive scan of the threads' sums within the warp
+        int64_t x = sum;  // inclusive scan of the threads' sums within the warp
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
             if (lane >= o) x += y;
         }
         if (lane == 31) s_warp[warp] = x;
         __syncthreads();
         if (warp == 0) {  // exclusive scan of the warp totals
-            const int w = lane < kScanThreads / 32 ? s_warp[lane] : 0;
-            int y = w;
+            const int64_t w = lane < kScanThreads / 32 ? s_warp[lane] : 0;
+            int64_t y = w;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int z = __shfl_up_sync(0xffffffffu, y, o);
+                const int64_t z = __shfl_up_sync(0xffffffffu, y, o);
                 if (lane >= o) y += z;
             }
             if (lane < kScanThreads / 32) s_warp[lane] = y - w;
         }
         __syncthreads();
-        int run = s_carry + s_warp[warp] + x - sum;  // before this thread's first element
+        int64_t run = s_carry + s_warp[warp] + x - sum;  // before this thread's first element
 #pragma unroll
         for (int t = 0; t < kScanPer; ++t) {
             const int k = k0 + t;
-            if (k < n) out[k] = run;
+            if (k < n) out[k] = clamp_i32(run);
             run += v[t];
         }
         __syncthreads();
         if (threadIdx.x == kScanThreads - 1) s_carry = run;  // the last thread's end: the chunk total
         __syncthreads();
     }
-    if (threadIdx.x == 0) out[n] = s_carry;
+    if (threadIdx.x == 0) {
+        out[n] = clamp_i32(s_carry);
+        if (total) *total = s_carry;
+    }
 }
 
 __global__ void extend_copy_kernel(PlanParams p) {
@@ -175,7 +188,6 @@ __global__ void extend_copy_kernel(PlanParams p) {
 __global__ void __launch_bounds__(kScanThreads) run_start_kernel(PlanParams p) {
     __shared__ int32_t s_warp[kScanThreads / 32];
     __shared__ int32_t s_carry;
-    if (p.totals->abort) return;
     const int h = blockIdx.x;
     const int32_t *D = p.doff + p.dptr[h];
     const int nd = p.ext_counts[2 * h];
@@ -357,18 +369,24 @@ __device__ int bitmap_tiles(const PlanParams &p, int h, int qb, const int32_t *D
     return count;
 }
 
-// One warp per (head, query block).  FILL = false: count; FILL = true: write tiles.
+// One warp per (head, query block).  FILL = false: count; FILL = true: write the tiles
+// at the offsets of the tile scan and copy those offsets into the plan's tile_ptr.
 template <bool FILL>
 __global__ void __launch_bounds__(128) plan_tiles_kernel(PlanParams p) {
     const int item = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (item >= p.H * p.nqb || p.totals->abort) return;
+    const int items = p.H * p.nqb;
+    if (item >= items || (FILL && p.totals->abort)) return;
+    if (FILL && lane == 0) {
+        p.tile_ptr[item] = p.tile_pos[item];
+        if (item == items - 1) p.tile_ptr[items] = p.tile_pos[items];
+    }
     const int h = item / p.nqb, qb = item % p.nqb;
     const int32_t *D = p.doff + p.dptr[h];
     const int32_t *C = p.vcol + p.vptr[h];
     const int nD = p.ext_counts[2 * h], nC = p.ext_counts[2 * h + 1];
     if (p.tmask && qb < p.nL) {  // Case 2: element-bitmap tiles, no stripe tiles
-        const int n = bitmap_tiles<FILL>(p, h, qb, D, nD, C, nC, FILL ? p.tile_ptr[item] : 0);
+        const int n = bitmap_tiles<FILL>(p, h, qb, D, nD, C, nC, FILL ? p.tile_pos[item] : 0);
         if (lane == 0) {
             if (FILL) p.stripe_cnt[item] = 0;
             else p.tile_counts[item] = n;
@@ -385,7 +403,7 @@ __global__ void __launch_bounds__(128) plan_tiles_kernel(PlanParams p) {
     int k = lower_bound_i32(D, nD, hi + 1) - 1;
     int next = 0;
     int count = 0;
-    int64_t pos = FILL ? p.tile_ptr[item] : 0;
+    int64_t pos = FILL ? p.tile_pos[item] : 0;
     while (k >= 0) {
         const int ks = run0[k];
         const int a = max(0, lo - __ldg(D + k)), b = hi - __ldg(D + ks);
@@ -425,9 +443,10 @@ __global__ void __launch_bounds__(128) plan_tiles_kernel(PlanParams p) {
     if (!FILL && lane == 0) p.tile_counts[item] = count;
 }
 
-// Fill pass: the extended lists must fit the plan's arrays (sized by an earlier sizing
-// pass): total diagonals, total columns, and each head's columns within max_vert (the
-// attention workspace's stripe buffers).  Otherwise the rest of the pass is skipped.
+// Fill pass: the new plan must fit the plan's arrays (sized by an earlier sizing pass):
+// total diagonals, total columns, each head's columns within max_vert (the attention
+// workspace's stripe buffers) and the tiles within n_tiles (and int32 offsets).
+// Otherwise the kernels that write the plan return at once.
 __global__ void __launch_bounds__(256) plan_check_kernel(PlanParams p) {
     __shared__ int s_bad;
     if (threadIdx.x == 0) s_bad = 0;
@@ -438,13 +457,15 @@ __global__ void __launch_bounds__(256) plan_check_kernel(PlanParams p) {
     __syncthreads();
     if (threadIdx.x == 0) {
         const int nd = p.ext_scan[p.H], nc = p.ext_scan[(p.H + 1) + p.H];
-        if (s_bad || nd > p.cap_diag || nc > p.cap_vert) {
+        const int64_t nt = p.totals->n_tiles;
+        if (s_bad || nd > p.cap_diag || nc > p.cap_vert || nt > p.capacity || nt > INT32_MAX) {
             p.totals->abort = 1;
             report(p.dev_status, SSA_ERR_CAPACITY);
         }
     }
 }
 
+// Sizing pass: list totals and the largest column count (n_tiles comes from the tile scan).
 __global__ void plan_totals_kernel(PlanParams p) {
     __shared__ int32_t s[3][32];
     int nd = 0, nv = 0, mv = 0;
@@ -477,7 +498,6 @@ __global__ void plan_totals_kernel(PlanParams p) {
         p.totals->n_diag = nd;
         p.totals->n_vert = nv;
         p.totals->max_vert = mv;
-        p.totals->n_tiles = p.tile_ptr[p.H * p.nqb];
     }
 }
 
@@ -535,7 +555,7 @@ int extend_impl(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offset
     w += align_up(sizeof(int32_t) * 2 * (n_heads + 1));
     p.tile_counts = reinterpret_cast<int32_t *>(w);
     w += align_up(sizeof(int32_t) * n_heads * nqb);
-    int32_t *ws_tile_ptr = reinterpret_cast<int32_t *>(w);
+    p.tile_pos = reinterpret_cast<int32_t *>(w);
     w += align_up(sizeof(int32_t) * (n_heads * nqb + 1));
     p.run0 = reinterpret_cast<int32_t *>(w);
     p.dev_status = dev_status;
@@ -555,14 +575,14 @@ int extend_impl(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offset
 
     if (plan == nullptr) {
         SSA_CHECK_ARG(sizes, "sparse_pattern_extend: sizes must not be NULL in the sizing pass");
-        p.tile_ptr = ws_tile_ptr;
         validate_lists_kernel<<<n_heads, 128, 0, s>>>(p);
         SSA_LAUNCH_CHECK();
         run_start_kernel<<<n_heads, kScanThreads, 0, s>>>(p);
         SSA_LAUNCH_CHECK();
         plan_tiles_kernel<false><<<tile_grid, 128, 0, s>>>(p);
         SSA_LAUNCH_CHECK();
-        exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.tile_counts, items, 1, 0, p.tile_ptr, nullptr);
+        exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.tile_counts, items, 1, 0, p.tile_pos,
+                                                         &p.totals->n_tiles);
         SSA_LAUNCH_CHECK();
         plan_totals_kernel<<<1, 1024, 0, s>>>(p);
         SSA_LAUNCH_CHECK();
@@ -580,6 +600,11 @@ int extend_impl(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offset
         if (host.status != 0) {
             set_error("sparse_pattern_extend: a pattern list is not strictly ascending and >= 0");
             return SSA_ERR_INVALID;
+        }
+        if (host.n_tiles > INT32_MAX) {
+            set_error("sparse_pattern_extend: %lld tiles exceed the int32 tile offsets of a plan",
+                      static_cast<long long>(host.n_tiles));
+            return SSA_ERR_CAPACITY;
         }
         return SSA_OK;
     }
@@ -618,6 +643,7 @@ int extend_impl(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offset
     p.ext_vptr = plan->ext_vert_ptr;
     p.ext_vcol = plan->ext_vert_cols;
 
+    // sizing of the new plan (workspace only), the capacity check, then the plan's writes
     validate_lists_kernel<<<n_heads, 128, 0, s>>>(p);
     SSA_LAUNCH_CHECK();
     exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.ext_counts, n_heads, 2, 0, p.ext_scan, nullptr);
@@ -625,15 +651,15 @@ int extend_impl(int n_heads, const int32_t *diag_ptr, const int32_t *diag_offset
     exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.ext_counts, n_heads, 2, 1,
                                                      p.ext_scan + (n_heads + 1), nullptr);
     SSA_LAUNCH_CHECK();
-    plan_check_kernel<<<1, 256, 0, s>>>(p);
-    SSA_LAUNCH_CHECK();
-    extend_copy_kernel<<<n_heads, 128, 0, s>>>(p);
-    SSA_LAUNCH_CHECK();
     run_start_kernel<<<n_heads, kScanThreads, 0, s>>>(p);
     SSA_LAUNCH_CHECK();
     plan_tiles_kernel<false><<<tile_grid, 128, 0, s>>>(p);
     SSA_LAUNCH_CHECK();
-    exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.tile_counts, items, 1, 0, p.tile_ptr, &p.totals->abort);
+    exclusive_scan_kernel<<<1, kScanThreads, 0, s>>>(p.tile_counts, items, 1, 0, p.tile_pos, &p.totals->n_tiles);
+    SSA_LAUNCH_CHECK();
+    plan_check_kernel<<<1, 256, 0, s>>>(p);
+    SSA_LAUNCH_CHECK();
+    extend_copy_kernel<<<n_heads, 128, 0, s>>>(p);
     SSA_LAUNCH_CHECK();
     plan_tiles_kernel<true><<<tile_grid, 128, 0, s>>>(p);
     SSA_LAUNCH_CHECK();

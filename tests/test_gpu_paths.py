@@ -120,9 +120,10 @@ def test_path_replayed_from_cuda_graph_matches_eager(ora):
 
 
 def test_refill_beyond_the_plan_reports_capacity(ora):
-    # a fill pass whose lists need more than the plan was sized for changes nothing in the
-    # plan and reports SSA_ERR_CAPACITY (-3): more diagonals in total, then more columns
-    # for one head than the plan's max_vert
+    # a fill pass whose new plan needs more than the plan was sized for changes nothing in
+    # the plan and reports SSA_ERR_CAPACITY (-3): more diagonals in total; more columns
+    # for one head than the plan's max_vert; lists of the same lengths whose diagonals lie
+    # further apart, so that only the tile count grows (30 -> 51 tiles)
     from gpu_util import lists_to_device
     S, d = 1024, 64
     diags = [np.arange(0, 40, dtype=np.int32), np.array([0, 7], np.int32)]
@@ -130,9 +131,14 @@ def test_refill_beyond_the_plan_reports_capacity(ora):
     dev_lists, host = lists_to_device(diags, verts)
     plan = ssa.extend(*dev_lists, S)
     before = plan.to_numpy()
+    spread = [np.arange(0, 1000, 25, dtype=np.int32), np.array([0, 7], np.int32)]
+    n_ref = ora.plan(ora.extend(*host, S), S)["n_tiles"]
+    n_spread = ora.plan(ora.extend(*lists_to_device(spread, verts)[1], S), S)["n_tiles"]
+    assert len(spread[0]) == len(diags[0]) and n_spread > n_ref == len(before["tile_key0"])
     bigger = [
         ([np.arange(0, 90, dtype=np.int32), np.array([0, 7], np.int32)], verts),
         (diags, [np.array([3, 99], np.int32), np.array([5, 6, 9], np.int32)]),
+        (spread, verts),
     ]
     for dg, vt in bigger:
         status = torch.zeros(1, dtype=torch.int32, device=dev())
