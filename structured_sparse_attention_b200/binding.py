@@ -300,10 +300,7 @@ def extend(diag_ptr, diag_offsets, vert_ptr, vert_cols, S: int, *, stream=None, 
     cs, s = _stream(stream)
     sizes = PlanSizes()
     if true_mask is not None:
-        _need_cuda(true_mask, "true_mask", torch.int32)
-        if true_mask.dim() != 3 or true_mask.shape[0] != H or true_mask.shape[2] != (true_mask.shape[1] + 31) // 32:
-            raise SSAError(-1, "true_mask must be [H, L, ceil(L/32)] int32")
-        L = true_mask.shape[1]
+        L = _check_true_mask(true_mask, H)
         run = lambda pl: lib.sparse_pattern_extend_case2(H, _ptr(diag_ptr), _ptr(diag_offsets), _ptr(vert_ptr),
                                                          _ptr(vert_cols), _ptr(true_mask), L, S, C.byref(sizes),
                                                          pl, _ptr(ws), ws.numel(), _ptr(status), cs)
@@ -323,18 +320,49 @@ def extend(diag_ptr, diag_offsets, vert_ptr, vert_cols, S: int, *, stream=None, 
     return plan
 
 
-def refill(plan: Plan, diag_ptr, diag_offsets, vert_ptr, vert_cols, *, stream=None, status=None):
-    """Re-run only the fill pass of sparse_pattern_extend into an existing plan (same sizes)."""
+def _check_true_mask(true_mask, H):
+    _need_cuda(true_mask, "true_mask", torch.int32)
+    if true_mask.dim() != 3 or true_mask.shape[0] != H or true_mask.shape[2] != (true_mask.shape[1] + 31) // 32:
+        raise SSAError(-1, "true_mask must be [H, L, ceil(L/32)] int32")
+    return true_mask.shape[1]
+
+
+def refill(plan: Plan, diag_ptr, diag_offsets, vert_ptr, vert_cols, *, true_mask=None, stream=None,
+           status=None):
+    """Re-run only the fill pass of sparse_pattern_extend into an existing plan (same sizes).
+    A Case-2 plan (made with a true mask) is refilled through sparse_pattern_extend_case2
+    with `true_mask` (by default the mask it was made with).  Nothing synchronises: a new
+    plan that does not fit leaves the plan as it was and sets SSA_ERR_CAPACITY in status."""
     lib = load()
+    for t, nm in ((diag_ptr, "diag_ptr"), (diag_offsets, "diag_offsets"), (vert_ptr, "vert_ptr"),
+                  (vert_cols, "vert_cols")):
+        _need_cuda(t, nm, torch.int32)
     H, S = plan.n_heads, plan.S
+    if diag_ptr.numel() != H + 1 or vert_ptr.numel() != H + 1:
+        raise SSAError(-1, f"diag_ptr and vert_ptr must hold {H + 1} offsets (the plan's heads + 1)")
     if diag_offsets.numel() == 0:
         diag_offsets = torch.zeros(1, dtype=torch.int32, device=diag_ptr.device)
     if vert_cols.numel() == 0:
         vert_cols = torch.zeros(1, dtype=torch.int32, device=diag_ptr.device)
+    if status is not None:
+        _need_cuda(status, "status", torch.int32)
     cs, _ = _stream(stream)
-    _check(lib.sparse_pattern_extend(H, _ptr(diag_ptr), _ptr(diag_offsets), _ptr(vert_ptr),
-                                     _ptr(vert_cols), S, C.byref(plan.sizes), C.byref(plan.struct),
-                                     _ptr(plan._ws), plan._ws.numel(), _ptr(status), cs))
+    lists = (_ptr(diag_ptr), _ptr(diag_offsets), _ptr(vert_ptr), _ptr(vert_cols))
+    if plan.tile_bits is not None:
+        tm = getattr(plan, "_true_mask", None) if true_mask is None else true_mask
+        if tm is None:
+            raise SSAError(-1, "refilling a Case-2 plan needs its true_mask")
+        L = _check_true_mask(tm, H)
+        _check(lib.sparse_pattern_extend_case2(H, *lists, _ptr(tm), L, S, C.byref(plan.sizes),
+                                               C.byref(plan.struct), _ptr(plan._ws), plan._ws.numel(),
+                                               _ptr(status), cs))
+        plan._true_mask = tm
+    else:
+        if true_mask is not None:
+            raise SSAError(-1, "a plan made without a true mask has no bitmap tiles: "
+                               "make it with extend(..., true_mask=...)")
+        _check(lib.sparse_pattern_extend(H, *lists, S, C.byref(plan.sizes), C.byref(plan.struct),
+                                         _ptr(plan._ws), plan._ws.numel(), _ptr(status), cs))
 
 
 # ------------------------------------------------------------------------------------

@@ -156,3 +156,41 @@ def test_refill_beyond_the_plan_reports_capacity(ora):
     O, LSE = ssa.attn_fwd(t_bf16(q), t_bf16(k), t_bf16(v), plan)
     Oref, Lref = ora.attn_dense(q, k, v, ora.extend(*host, S), d ** -0.5)
     compare_attn(O, LSE, Oref, Lref)
+
+
+def test_case2_refill_goes_through_the_bitmap_fill(ora):
+    # refilling a Case-2 plan with a true mask that keeps a random half of the captured
+    # cells (so the new plan fits) gives the plan a fresh sparse_pattern_extend_case2
+    # makes from it, the oracle's Case-2 plan, and attention that matches the oracle;
+    # a refill without a mask reuses the one the plan holds
+    L, S, H, d = 256, 600, 2, 64
+    maps = inputs.averaged_maps(inputs.SEED_BASE + 74, H, L=L, n_samples=3)
+    cap = ssa.capture(torch.from_numpy(maps).to(dev()), true_mask=True)
+    lists = (cap["diag_ptr"], cap["diag_offsets"], cap["vert_ptr"], cap["vert_cols"])
+    plan = ssa.extend(*lists, S, true_mask=cap["true_mask"])
+    g = np.random.default_rng(inputs.SEED_BASE + 75)
+    keep = g.integers(0, 2 ** 32, size=tuple(cap["true_mask"].shape), dtype=np.uint64).astype(np.uint32)
+    tm_sub = cap["true_mask"] & torch.from_numpy(keep.view(np.int32)).to(dev())
+    for mask in (tm_sub, None):
+        status = torch.zeros(1, dtype=torch.int32, device=dev())
+        ssa.refill(plan, *lists, true_mask=mask, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        got, fresh = plan.to_numpy(), ssa.extend(*lists, S, true_mask=tm_sub).to_numpy()
+        n = int(fresh["tile_ptr"][-1])
+        assert n <= plan.n_tiles
+        for key in ("tile_ptr", "stripe_cnt", "tile_bits"):
+            np.testing.assert_array_equal(got[key], fresh[key], err_msg=key)
+        for key in ("tile_key0", "tile_dmask", "tile_cmask", "tile_flags"):
+            np.testing.assert_array_equal(got[key][:n], fresh[key][:n], err_msg=key)
+    w = tm_sub.cpu().numpy().astype(np.uint32)
+    j = np.arange(L)
+    tmb = ((w[..., j // 32] >> (j % 32).astype(np.uint32)) & 1).astype(np.uint8)
+    ext = ora.extend(*ora.capture(maps), S)
+    pref = ora.plan_case2(ext, S, tmb)
+    for key in ("tile_ptr", "stripe_cnt", "tile_bits"):
+        np.testing.assert_array_equal(got[key], pref[key], err_msg=key)
+    q, k, v = inputs.qkv(inputs.SEED_BASE + 76, H, H, S, d)
+    O, LSE = ssa.attn_fwd(t_bf16(q), t_bf16(k), t_bf16(v), plan)
+    Oref, Lref = ora.attn_dense_case2(q, k, v, ext, d ** -0.5, tmb)
+    compare_attn(O, LSE, Oref, Lref)
