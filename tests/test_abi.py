@@ -127,3 +127,6 @@ def test_binding_rejects_host_tensors_before_any_call(lib):
         binding.capture(torch.zeros((1, 16, 16), dtype=torch.float32))
     with pytest.raises(binding.SSAError):
         binding.extend(*(torch.zeros(2, dtype=torch.int32) for _ in range(4)), 64)
+    with pytest.raises(binding.SSAError) as e:
+        binding.refill(object(), *(torch.zeros(2, dtype=torch.int32) for _ in range(4)))
+    assert e.value.code == -1 and "CUDA" in str(e.value)
