@@ -1,0 +1,126 @@
+"""Mutation check of the oracle's pins (CPU only).
+
+Each case plants one plausible mistake in a copy of oracle/ssa_oracle.c (a dropped term,
+a wrong comparison, a swapped index or operand, an off-by-one bound), builds it with the
+oracle's own flags, and runs the pin file of that routine against it: at least one pin
+must fail.  An unmutated copy run the same way must pass, which checks the harness.  The
+mistakes are planted in the oracle on the CPU only; nothing here touches the library.
+"""
+
+import concurrent.futures as cf
+import os
+import subprocess
+import sys
+
+import pytest
+
+from conftest import ROOT
+
+SRC = os.path.join(ROOT, "oracle", "ssa_oracle.c")
+
+CAP, PLAN, ATTN, MAPS, CASE2 = ("tests/test_oracle_capture.py", "tests/test_oracle_plan.py",
+                                "tests/test_oracle_attn.py", "tests/test_oracle_maps.py",
+                                "tests/test_oracle_case2.py")
+
+# (name, text in ssa_oracle.c (exactly one occurrence), replacement, pin files)
+MUTANTS = [
+    ("box-cox: eps dropped", "double z = v + eps;", "double z = v;", CAP),
+    ("true mask: t > tau instead of t >= tau", "bit = (t >= tau) ? 1 : 0;", "bit = (t > tau) ? 1 : 0;", CAP),
+    ("true mask: constant row scores 0", "t = 1.0;\n", "t = 0.0;\n", CAP),
+    ("true mask: row min / max over the whole row, not its causal part",
+     "        for (int j = 0; j <= i; ++j) {\n            double x = (double)row[j];",
+     "        for (int j = 0; j < L; ++j) {\n            double x = (double)row[j];", CAP),
+    ("true mask: per-map scaling ignored", "if (scaling == 1) {\n            mn = map_mn;",
+     "if (scaling == 2) {\n            mn = map_mn;", CAP),
+    ("gamma: mask transposed", "num += M[(size_t)i * L + (i - r)];", "num += M[(size_t)(i - r) * L + i];", CAP),
+    ("gamma: denominator off by one", "gamma_diag[r] = (double)num / (double)den;",
+     "gamma_diag[r] = (double)num / (double)(den + 1);", CAP),
+    ("select: diagonal ties dropped", "if (gamma_diag[r] >= mu)", "if (gamma_diag[r] > mu)", CAP),
+    ("select: column ties dropped", "if (gamma_vert[c] >= mu)", "if (gamma_vert[c] > mu)", CAP),
+    ("extend: diagonal r = S kept", "if (D[k] < S) ext_diag_offsets[od++] = D[k];",
+     "if (D[k] <= S) ext_diag_offsets[od++] = D[k];", PLAN),
+    ("extend: column c = S kept", "if (C[k] < S) ext_vert_cols[oc++] = C[k];",
+     "if (C[k] <= S) ext_vert_cols[oc++] = C[k];", PLAN),
+    ("plan (interval): FULL ignores the columns",
+     "            int full = ((long)T * (qb + 1) <= S) && popcount256(dm) == 2 * T - 1 && cm[0] == 0 &&\n"
+     "                       cm[1] == 0;",
+     "            int full = ((long)T * (qb + 1) <= S) && popcount256(dm) == 2 * T - 1;", PLAN),
+    ("plan (brute): FULL without the whole-block condition",
+     "                int full = ((long)T * (qb + 1) <= S) && popcount256(dm)",
+     "                int full = 1 && popcount256(dm)", PLAN),
+    ("plan (interval): stripe count one short", "stripe_cnt[h * nqb + qb] = count_le(C, nc, (int32_t)hi_i);",
+     "stripe_cnt[h * nqb + qb] = count_le(C, nc, (int32_t)hi_i - 1);", PLAN),
+    # (a run boundary at a gap of exactly 128 changes nothing: the two runs' key ranges
+    # touch, so the windows are the same; a gap of 129 leaves an unneeded key between them)
+    ("plan (interval): offsets 129 apart taken as one run", "D[k] - D[k - 1] <= ORA_TILE",
+     "D[k] - D[k - 1] <= ORA_TILE + 1", PLAN),
+    ("nnz: a cell on a diagonal and a column counted twice", "total += own - shared;", "total += own;", PLAN),
+    ("attention: LSE in log2", "*lse = m + log(l);", "*lse = m + log2(l);", ATTN),
+    ("attention: GQA heads interleaved instead of grouped", "return kv_map ? kv_map[h] : h / (Hq / Hkv);",
+     "return kv_map ? kv_map[h] : h % Hkv;", ATTN),
+    ("attention: exponentials not shifted by the row max", "double p = exp(s[a] - m);",
+     "double p = exp(s[a]);", ATTN),
+    ("attention (rows): diagonal r = i skipped", "if (D[k] > i) continue;", "if (D[k] >= i) continue;", ATTN),
+    ("attention (dense): a column's first cell missing",
+     "for (long i = C[k]; i < S; ++i) Mt[(size_t)i * S + C[k]] = 1;",
+     "for (long i = C[k] + 1; i < S; ++i) Mt[(size_t)i * S + C[k]] = 1;", ATTN),
+    ("case 2: the true-mask block added to the patterns instead of replacing them",
+     "Mt[(size_t)i * S + j] = Bh[(size_t)i * Lb + j] ? 1 : 0;",
+     "Mt[(size_t)i * S + j] |= Bh[(size_t)i * Lb + j] ? 1 : 0;", CASE2),
+    ("maps: scale dropped", "s[j] = scale * dot;", "s[j] = dot;", MAPS),
+    ("maps: query and key rows swapped",
+     "bf16_bits_to_double(q[(size_t)i * d + c]) * bf16_bits_to_double(k[(size_t)j * d + c])",
+     "bf16_bits_to_double(q[(size_t)j * d + c]) * bf16_bits_to_double(k[(size_t)i * d + c])", MAPS),
+    ("maps: exponentials not shifted by the row max", "s[j] = exp(s[j] - mx);", "s[j] = exp(s[j]);", MAPS),
+    ("maps: mean over samples without 1/B", "row[j] += s[j] / sum / B;", "row[j] += s[j] / sum;", MAPS),
+    ("maps: softmax sum starts at 1", "double sum = 0.0;", "double sum = 1.0;", MAPS),
+]
+
+_DRIVER = (
+    "import sys\n"
+    "sys.path.insert(0, sys.argv[1])\n"
+    "from oracle import oracle as o\n"
+    "o.LIB = sys.argv[2]\n"
+    "o.build = lambda force=False: o.LIB\n"
+    "import pytest\n"
+    "sys.exit(pytest.main(['-x', '-q', '-p', 'no:cacheprovider', '-m', 'not gpu'] + sys.argv[3].split(',')))\n"
+)
+
+
+def _build_and_run(src_text, workdir, tests):
+    os.makedirs(workdir, exist_ok=True)
+    c_path = os.path.join(workdir, "ssa_oracle.c")
+    so_path = os.path.join(workdir, "libssa_oracle.so")
+    with open(c_path, "w") as f:
+        f.write(src_text)
+    subprocess.run(["gcc", "-std=c11", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+                    "-o", so_path, c_path, "-lm"], check=True)
+    env = dict(os.environ, OMP_NUM_THREADS="2")
+    p = subprocess.run([sys.executable, "-c", _DRIVER, ROOT, so_path, tests], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    return p.returncode, p.stdout[-1500:] + p.stderr[-1500:]
+
+
+@pytest.fixture(scope="module")
+def outcomes(tmp_path_factory):
+    base = tmp_path_factory.mktemp("mutants")
+    src = open(SRC).read()
+    jobs = {"unmutated": (src, ",".join((CAP, PLAN, ATTN, MAPS, CASE2)))}
+    for name, old, new, tests in MUTANTS:
+        assert src.count(old) == 1, f"{name}: the text to mutate must occur exactly once"
+        jobs[name] = (src.replace(old, new), tests)
+    with cf.ThreadPoolExecutor(max_workers=8) as ex:
+        futs = {name: ex.submit(_build_and_run, text, str(base / f"m{k}"), tests)
+                for k, (name, (text, tests)) in enumerate(jobs.items())}
+        return {name: f.result() for name, f in futs.items()}
+
+
+def test_unmutated_copy_passes_every_pin(outcomes):
+    rc, log = outcomes["unmutated"]
+    assert rc == 0, log
+
+
+@pytest.mark.parametrize("name", [m[0] for m in MUTANTS])
+def test_planted_mistake_fails_a_pin(outcomes, name):
+    rc, log = outcomes[name]
+    assert rc == 1, f"{name}: pins {'passed' if rc == 0 else f'ended with code {rc}'}\n{log}"

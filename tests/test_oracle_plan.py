@@ -93,10 +93,11 @@ def test_plan_main_diagonal_only(ora):
         assert not p["stripe_cnt"].any()
 
 
-def test_plan_full_causal(ora):
+@pytest.mark.parametrize("routine", ["brute", "interval"])
+def test_plan_full_causal(ora, routine):
     S = 512
     ext = _ext(ora, [np.arange(S, dtype=np.int32)], [np.array([], np.int32)], S)
-    p = ora.plan(ext, S)
+    p = ora.plan(ext, S, routine)
     assert p["n_tiles"] == 4 * 5 // 2
     for qb in range(4):
         a, b = p["tile_ptr"][qb], p["tile_ptr"][qb + 1]
@@ -110,29 +111,46 @@ def test_plan_full_causal(ora):
                                                        0xFFFFFFFFFFFFFFFF, 0x7FFFFFFFFFFFFFFF]
 
 
-def test_plan_column_owned_by_stripes(ora):
+@pytest.mark.parametrize("routine", ["brute", "interval"])
+def test_plan_column_owned_by_stripes(ora, routine):
     # D = {128}, C = {0..127}: the only window of block 1 (keys 0..127) holds band
     # elements in columns of C only, so it is not listed; the stripe phase owns them.
     S = 256
     ext = _ext(ora, [np.array([128], np.int32)], [np.arange(128, dtype=np.int32)], S)
-    p = ora.plan(ext, S)
+    p = ora.plan(ext, S, routine)
     assert p["n_tiles"] == 0
     assert p["stripe_cnt"].tolist() == [128, 128]
-    # one excluded column stops a tile from being FULL but keeps it listed
+    # one excluded column stops a tile from being FULL but keeps it listed: the window
+    # of block 1 at keys 0..127 sees every diagonal (r = 1..255), column 5 excludes one
     ext = _ext(ora, [np.arange(S, dtype=np.int32)], [np.array([5], np.int32)], S)
-    p = ora.plan(ext, S)
+    p = ora.plan(ext, S, routine)
     t = p["tile_ptr"][1]
     assert p["tile_key0"][t] == 0 and p["tile_flags"][t] == 0
     assert p["tile_cmask"][t].tolist() == [1 << 5, 0]
+    assert p["tile_dmask"][t].tolist() == [2**64 - 1, 2**64 - 1, 2**64 - 1, 2**63 - 1]
 
 
-def test_plan_ragged_tail_is_not_full(ora):
+@pytest.mark.parametrize("routine", ["brute", "interval"])
+def test_plan_ragged_tail_is_not_full(ora, routine):
     S = 200  # second block has 72 rows
     ext = _ext(ora, [np.arange(S, dtype=np.int32)], [np.array([], np.int32)], S)
-    p = ora.plan(ext, S)
+    p = ora.plan(ext, S, routine)
     a, b = p["tile_ptr"][1], p["tile_ptr"][2]
     assert p["tile_key0"][a:b].tolist() == [0, T]
     assert p["tile_flags"][a:b].tolist() == [0, 0]
+    # S = 400: the ragged block 3 (rows 384..399) has windows that see all 255 diagonals
+    # and no column (keys 0..127 and 128..255: r = 257..511 and 129..383, all kept up
+    # to S - 1 = 399 for the second); FULL needs the whole block inside S, so none is
+    S = 400
+    ext = _ext(ora, [np.arange(S, dtype=np.int32)], [np.array([], np.int32)], S)
+    p = ora.plan(ext, S, routine)
+    a, b = p["tile_ptr"][3], p["tile_ptr"][4]
+    assert p["tile_key0"][a:b].tolist() == [0, T, 2 * T, 3 * T]
+    assert p["tile_dmask"][a + 1].tolist() == [2**64 - 1, 2**64 - 1, 2**64 - 1, 2**63 - 1]
+    assert p["tile_flags"][a:b].tolist() == [0, 0, 0, 0]
+    # the same window in the whole block 2 (rows 256..383, keys 0..127: r = 129..383) is FULL
+    a2 = p["tile_ptr"][2]
+    assert p["tile_key0"][a2] == 0 and p["tile_flags"][a2] == 1
 
 
 @pytest.mark.parametrize("seed", range(12))
@@ -204,3 +222,17 @@ def test_plan_windows_skip_gaps_between_diagonal_runs(ora):
         p = ora.plan(ext, S, routine)
         a, b = p["tile_ptr"][7], p["tile_ptr"][8]
         assert p["tile_key0"][a:b].tolist() == [196, 895, 1023]
+
+
+@pytest.mark.parametrize("routine", ["brute", "interval"])
+def test_plan_runs_128_and_129_apart(ora, routine):
+    # Block 2 (rows 256..383).  D = {0, 128}: the keys reached by r = 128 (128..255) and by
+    # r = 0 (256..383) touch, so the windows are 128 and 256.  D = {0, 129}: r = 129
+    # reaches 127..254 and r = 0 reaches 256..383; key 255 is needed by no row (it would
+    # need r in 1..128), so the second window starts at 256, not at 255: 127 and 256.
+    S = 512
+    for D, want in (([0, 128], [128, 256]), ([0, 129], [127, 256])):
+        ext = _ext(ora, [np.array(D, np.int32)], [np.array([], np.int32)], S)
+        p = ora.plan(ext, S, routine)
+        a, b = p["tile_ptr"][2], p["tile_ptr"][3]
+        assert p["tile_key0"][a:b].tolist() == want, (D, routine)
