@@ -215,3 +215,23 @@ def test_per_map_scaling_invariants(ora):
         on, off = m[cells & (M == 1)], m[cells & (M == 0)]
         if on.size and off.size:
             assert on.min() > off.max()
+
+
+@pytest.mark.parametrize("scaling", ["row", "map"])
+def test_entries_above_the_diagonal_play_no_part(ora, scaling):
+    # The pattern pool and the maps are causal: the true mask, its row (or map) min and
+    # max, and so the capture depend on the entries j <= i only.  Values written above
+    # the diagonal, larger and smaller than every causal entry, change nothing.
+    L = 96
+    maps = inputs.averaged_maps(31, 3, L=L, n_samples=3)
+    junk = maps.copy()
+    iu = np.triu_indices(L, 1)
+    junk[:, iu[0], iu[1]] = np.where((iu[0] + iu[1]) % 2 == 0, 7.0, 1e-30).astype(np.float32)
+    for m in range(3):
+        for lam in (0.5, 1.0):
+            a = ora.true_mask(maps[m], lam=lam, scaling=scaling)
+            b = ora.true_mask(junk[m], lam=lam, scaling=scaling)
+            np.testing.assert_array_equal(a, b)
+            assert not a[iu].any()
+    for x, y in zip(ora.capture(maps, scaling=scaling), ora.capture(junk, scaling=scaling)):
+        np.testing.assert_array_equal(x, y)

@@ -74,6 +74,31 @@ MUTANTS = [
     ("maps: exponentials not shifted by the row max", "s[j] = exp(s[j] - mx);", "s[j] = exp(s[j]);", MAPS),
     ("maps: mean over samples without 1/B", "row[j] += s[j] / sum / B;", "row[j] += s[j] / sum;", MAPS),
     ("maps: softmax sum starts at 1", "double sum = 0.0;", "double sum = 1.0;", MAPS),
+    ("box-cox: general lambda takes the reciprocal power", "return (pow(z, lambda) - 1.0) / lambda;",
+     "return (pow(z, 1.0 / lambda) - 1.0) / lambda;", CAP),
+    ("true mask: map min / max over the whole map, not its causal part",
+     "    for (int i = 0; i < L; ++i)\n        for (int j = 0; j <= i; ++j) {\n            double x = (double)map[",
+     "    for (int i = 0; i < L; ++i)\n        for (int j = 0; j < L; ++j) {\n            double x = (double)map[", CAP),
+    ("gamma: column mask transposed", "num += M[(size_t)i * L + c];", "num += M[(size_t)c * L + i];", CAP),
+    ("capture: diagonal offsets advanced by the column count", "diag_ptr[m + 1] = diag_ptr[m] + cnt_d[m];",
+     "diag_ptr[m + 1] = diag_ptr[m] + cnt_v[m];", CAP),
+    ("plan (brute): a window of column cells only is listed", "if (j <= i && isD[i - j] && !isC[j])",
+     "if (j <= i && isD[i - j])", PLAN),
+    ("plan (interval): rows past S make a window listed", "if (nrows - 1 < il_hi) il_hi = nrows - 1;", "", PLAN),
+    ("plan (brute): stripe count one long", "count_le(C, nc, last_row)", "count_le(C, nc, last_row + 1)", PLAN),
+    ("plan (interval): diagonal mask shifted by one", "long base = lo - key0 - (T - 1);",
+     "long base = lo - key0 - T;", PLAN),
+    ("nnz: shared cells counted up to S", "if ((long long)C[k] + D[q] < S) ++shared;",
+     "if ((long long)C[k] + D[q] <= S) ++shared;", PLAN),
+    ("attention (rows): column c = i skipped", "if (C[k] > i) continue;", "if (C[k] >= i) continue;", ATTN),
+    ("attention (dense): a diagonal's first cell missing", "for (long i = D[k]; i < S; ++i)",
+     "for (long i = D[k] + 1; i < S; ++i)", ATTN),
+    ("attention: scale dropped", "s[a] = scale * dot;", "s[a] = dot;", ATTN),
+    ("attention: output not normalised", "for (int k = 0; k < d; ++k) o[k] /= l;", "", ATTN),
+    ("attention: empty row gives LSE 0", "*lse = -INFINITY;", "*lse = 0.0;", ATTN),
+    ("case 2: the block's diagonal cells kept from the patterns",
+     "for (int j = 0; j <= i; ++j) Mt[(size_t)i * S + j] = Bh", "for (int j = 0; j < i; ++j) Mt[(size_t)i * S + j] = Bh",
+     CASE2),
 ]
 
 _DRIVER = (
