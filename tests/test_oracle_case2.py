@@ -209,3 +209,41 @@ def test_case2_plan_with_pattern_block_matches_case_one(ora):
     np.testing.assert_array_equal(pl1["tile_key0"][a1:], pl2["tile_key0"][a2:])
     np.testing.assert_array_equal(pl1["tile_flags"][a1:], pl2["tile_flags"][a2:])
     assert (pl2["tile_flags"][:a2] == 2).all() and (pl2["stripe_cnt"][:nL] == 0).all()
+
+
+@pytest.mark.parametrize("L,S,nL", [(512, 300, 3), (512, 1000, 4), (384, 1500, 3), (200, 100, 1), (128, 128, 1)])
+def test_case2_bitmap_layout(ora, L, S, nL):
+    # bitmap blocks are the query blocks holding a row below min(L, S): nL of them, with a
+    # slot per (qb, kb <= qb), slot = h * slots + qb (qb + 1) / 2 + kb; listed tiles are
+    # those with a set cell, and every slot of a listed tile is its own
+    H = 2
+    slots = nL * (nL + 1) // 2
+    assert ora.case2_bitmap_slots(L, S) == (nL, slots)
+    diags = [np.array([0, 3]), np.array([1])]
+    verts = [np.array([5]), np.array([0])]
+    ext = _ext(ora, [d[d < S] for d in diags], [c[c < S] for c in verts], S)
+    tm = (np.random.default_rng(L * S).random((H, L, L)) < 0.3).astype(np.uint8)
+    pl = ora.plan_case2(ext, S, tm)
+    assert pl["bitmap_slots"] == slots and pl["tile_bits"].shape == (H * slots, 128, 2)
+    nqb = pl["nqb"]
+    seen = set()
+    for h in range(H):
+        for qb in range(min(nL, nqb)):
+            it = h * nqb + qb
+            for t in range(pl["tile_ptr"][it], pl["tile_ptr"][it + 1]):
+                kb = int(pl["tile_key0"][t]) // 128
+                slot = int(pl["tile_dmask"][t][0])
+                assert pl["tile_flags"][t] == 2 and slot == h * slots + qb * (qb + 1) // 2 + kb
+                assert pl["tile_bits"][slot].any() and slot not in seen
+                seen.add(slot)
+
+
+def test_case2_empty_bitmap_tile_is_not_listed(ora):
+    # L = S = 256 and a true mask of the main diagonal only: block 1's key block 0 (rows
+    # 128..255, keys 0..127) holds no cell, so block 1 lists key block 1 alone
+    L = S = 256
+    ext = _ext(ora, [np.array([], np.int64)], [np.array([], np.int64)], S)
+    tm = np.eye(L, dtype=np.uint8)[None]
+    pl = ora.plan_case2(ext, S, tm)
+    assert pl["tile_key0"][pl["tile_ptr"][0]:pl["tile_ptr"][1]].tolist() == [0]
+    assert pl["tile_key0"][pl["tile_ptr"][1]:pl["tile_ptr"][2]].tolist() == [128]

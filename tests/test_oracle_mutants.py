@@ -1,9 +1,9 @@
 """Mutation check of the oracle's pins (CPU only).
 
-Each case plants one plausible mistake in a copy of oracle/ssa_oracle.c (a dropped term,
-a wrong comparison, a swapped index or operand, an off-by-one bound), builds it with the
-oracle's own flags, and runs the pin file of that routine against it: at least one pin
-must fail.  An unmutated copy run the same way must pass, which checks the harness.  The
+Each case plants one plausible mistake in a copy of the oracle (oracle/ssa_oracle.c, or
+the Case-2 plan routine of oracle/oracle.py): a dropped term, a wrong comparison, a
+swapped index or operand, an off-by-one bound.  The copy is built with the oracle's own
+flags and the pin file of that routine runs against it: at least one pin must fail.  An unmutated copy run the same way must pass, which checks the harness.  The
 mistakes are planted in the oracle on the CPU only; nothing here touches the library.
 """
 
@@ -17,6 +17,7 @@ import pytest
 from conftest import ROOT
 
 SRC = os.path.join(ROOT, "oracle", "ssa_oracle.c")
+PY_SRC = os.path.join(ROOT, "oracle", "oracle.py")
 
 CAP, PLAN, ATTN, MAPS, CASE2 = ("tests/test_oracle_capture.py", "tests/test_oracle_plan.py",
                                 "tests/test_oracle_attn.py", "tests/test_oracle_maps.py",
@@ -101,27 +102,45 @@ MUTANTS = [
      CASE2),
 ]
 
+# Mistakes in the Case-2 plan routine (Python, over the C routines' lists).
+PY_MUTANTS = [
+    ("case 2 plan: past row L the columns are dropped", "cell[il, c] = (i - j) in D or j in Cs",
+     "cell[il, c] = (i - j) in D", CASE2),
+    ("case 2 plan: bitmap blocks keep their stripe counts", "                stripe[it] = 0\n", "", CASE2),
+    ("case 2 plan: slots of a head overlap", "slot = h * slots + qb * (qb + 1) // 2 + kb",
+     "slot = h * slots + qb * qb // 2 + kb", CASE2),
+    ("case 2 plan: bitmap blocks counted from L even when S < L",
+     "nL = (min(L, S) + TILE - 1) // TILE", "nL = (L + TILE - 1) // TILE", CASE2),
+    ("case 2 plan: empty bitmap tiles listed", "                    if not cell.any():\n                        continue\n",
+     "", CASE2),
+]
+
+# The copy is a package of its own (oracle/__init__.py, oracle.py, the built C library)
+# placed first on the path, so the pins import it instead of the repository's oracle.
 _DRIVER = (
     "import sys\n"
     "sys.path.insert(0, sys.argv[1])\n"
+    "sys.path.insert(0, sys.argv[2])\n"
     "from oracle import oracle as o\n"
-    "o.LIB = sys.argv[2]\n"
+    "assert o.__file__.startswith(sys.argv[2])\n"
+    "o.LIB = sys.argv[3]\n"
     "o.build = lambda force=False: o.LIB\n"
     "import pytest\n"
-    "sys.exit(pytest.main(['-x', '-q', '-p', 'no:cacheprovider', '-m', 'not gpu'] + sys.argv[3].split(',')))\n"
+    "sys.exit(pytest.main(['-x', '-q', '-p', 'no:cacheprovider', '-m', 'not gpu'] + sys.argv[4].split(',')))\n"
 )
 
 
-def _build_and_run(src_text, workdir, tests):
-    os.makedirs(workdir, exist_ok=True)
-    c_path = os.path.join(workdir, "ssa_oracle.c")
-    so_path = os.path.join(workdir, "libssa_oracle.so")
-    with open(c_path, "w") as f:
-        f.write(src_text)
+def _build_and_run(c_text, py_text, workdir, tests):
+    pkg = os.path.join(workdir, "oracle")
+    os.makedirs(pkg, exist_ok=True)
+    for name, text in (("ssa_oracle.c", c_text), ("oracle.py", py_text), ("__init__.py", "")):
+        with open(os.path.join(pkg, name), "w") as f:
+            f.write(text)
+    so_path = os.path.join(pkg, "libssa_oracle.so")
     subprocess.run(["gcc", "-std=c11", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
-                    "-o", so_path, c_path, "-lm"], check=True)
+                    "-o", so_path, os.path.join(pkg, "ssa_oracle.c"), "-lm"], check=True)
     env = dict(os.environ, OMP_NUM_THREADS="2")
-    p = subprocess.run([sys.executable, "-c", _DRIVER, ROOT, so_path, tests], cwd=ROOT, env=env,
+    p = subprocess.run([sys.executable, "-c", _DRIVER, ROOT, workdir, so_path, tests], cwd=ROOT, env=env,
                        capture_output=True, text=True, timeout=600)
     return p.returncode, p.stdout[-1500:] + p.stderr[-1500:]
 
@@ -129,14 +148,17 @@ def _build_and_run(src_text, workdir, tests):
 @pytest.fixture(scope="module")
 def outcomes(tmp_path_factory):
     base = tmp_path_factory.mktemp("mutants")
-    src = open(SRC).read()
-    jobs = {"unmutated": (src, ",".join((CAP, PLAN, ATTN, MAPS, CASE2)))}
+    src, py = open(SRC).read(), open(PY_SRC).read()
+    jobs = {"unmutated": (src, py, ",".join((CAP, PLAN, ATTN, MAPS, CASE2)))}
     for name, old, new, tests in MUTANTS:
         assert src.count(old) == 1, f"{name}: the text to mutate must occur exactly once"
-        jobs[name] = (src.replace(old, new), tests)
+        jobs[name] = (src.replace(old, new), py, tests)
+    for name, old, new, tests in PY_MUTANTS:
+        assert py.count(old) == 1, f"{name}: the text to mutate must occur exactly once"
+        jobs[name] = (src, py.replace(old, new), tests)
     with cf.ThreadPoolExecutor(max_workers=8) as ex:
-        futs = {name: ex.submit(_build_and_run, text, str(base / f"m{k}"), tests)
-                for k, (name, (text, tests)) in enumerate(jobs.items())}
+        futs = {name: ex.submit(_build_and_run, c, p, str(base / f"m{k}"), tests)
+                for k, (name, (c, p, tests)) in enumerate(jobs.items())}
         return {name: f.result() for name, f in futs.items()}
 
 
@@ -145,7 +167,7 @@ def test_unmutated_copy_passes_every_pin(outcomes):
     assert rc == 0, log
 
 
-@pytest.mark.parametrize("name", [m[0] for m in MUTANTS])
+@pytest.mark.parametrize("name", [m[0] for m in MUTANTS + PY_MUTANTS])
 def test_planted_mistake_fails_a_pin(outcomes, name):
     rc, log = outcomes[name]
     assert rc == 1, f"{name}: pins {'passed' if rc == 0 else f'ended with code {rc}'}\n{log}"
