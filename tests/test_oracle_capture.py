@@ -93,6 +93,18 @@ def test_true_mask_constant_row_is_all_set(ora):
         assert M[i, :i + 1].all() and not M[i, i + 1:].any()
 
 
+def test_true_mask_constant_map_is_all_set_under_per_map_scaling(ora):
+    # per-map scaling (R19): a map whose causal entries are all equal has t = 1 at every
+    # causal cell, so every candidate pattern has gamma = 1 and is kept (even at tau = 1)
+    L = 8
+    amap = np.tril(np.full((L, L), 0.25, np.float32))
+    for tau in (0.3, 1.0):
+        M = ora.true_mask(amap, tau=tau, scaling="map")
+        assert (M == np.tril(np.ones((L, L), np.uint8))).all()
+    dp, do, vp, vc = ora.capture(amap[None], tau=1.0, mu=1.0, scaling="map")
+    assert do.tolist() == list(range(L)) and vc.tolist() == list(range(L))
+
+
 def test_invariants_on_synthetic_maps(ora):
     maps = inputs.averaged_maps(11, 3, L=128, n_samples=4)
     L = 128

@@ -100,6 +100,20 @@ MUTANTS = [
     ("case 2: the block's diagonal cells kept from the patterns",
      "for (int j = 0; j <= i; ++j) Mt[(size_t)i * S + j] = Bh", "for (int j = 0; j < i; ++j) Mt[(size_t)i * S + j] = Bh",
      CASE2),
+    ("plan items: stripe count one short", "if (stripe_cnt) stripe_cnt[a] = count_le(C, nc, (int32_t)hi_i);",
+     "if (stripe_cnt) stripe_cnt[a] = count_le(C, nc, (int32_t)hi_i - 1);", PLAN),
+    ("true mask: a constant map under per-map scaling not scored 1", "if (mx == mn) {",
+     "if (mx == mn && scaling == 0) {", CAP),
+    ("attention (rows): a cell on a diagonal and a column taken twice", "if (!mark[C[k]]) {", "if (1) {", ATTN),
+    ("extend: duplicate offsets accepted", "if (k > 0 && a[k] <= a[k - 1]) return 0;",
+     "if (k > 0 && a[k] < a[k - 1]) return 0;", PLAN),
+    ("extend: negative offsets accepted", "if (a[k] < 0) return 0;", "", PLAN),
+    ("maps: row max never taken", "if (s[j] > mx) mx = s[j];", "if (s[j] > mx) mx = 0.0;", MAPS),
+    ("attention: an explicit GQA map ignored", "return kv_map ? kv_map[h] : h / (Hq / Hkv);",
+     "return h / (Hq / Hkv);", ATTN),
+    ("attention: LSE without the row max", "*lse = m + log(l);", "*lse = log(l);", ATTN),
+    ("gamma: column denominator off by one", "gamma_vert[c] = (double)num / (double)den;",
+     "gamma_vert[c] = (double)num / (double)(den + 1);", CAP),
 ]
 
 # Mistakes in the Case-2 plan routine (Python, over the C routines' lists).

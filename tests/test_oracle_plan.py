@@ -236,3 +236,17 @@ def test_plan_runs_128_and_129_apart(ora, routine):
         p = ora.plan(ext, S, routine)
         a, b = p["tile_ptr"][2], p["tile_ptr"][3]
         assert p["tile_key0"][a:b].tolist() == want, (D, routine)
+
+
+def test_stripe_counts_at_block_ends(ora):
+    # columns exactly at a block's last row (127, 383) and at S - 1 = 999: block qb
+    # counts the columns c <= min(S - 1, 128 qb + 127), the same in every routine
+    S = 1000
+    ext = _ext(ora, [np.array([0], np.int32)], [np.array([127, 383, 999], np.int32)], S)
+    want = {0: 1, 1: 1, 2: 2, 3: 2, 6: 2, 7: 3}
+    for routine in ("brute", "interval"):
+        p = ora.plan(ext, S, routine)
+        assert {qb: int(p["stripe_cnt"][qb]) for qb in want} == want
+    items = np.array([[0, qb] for qb in want], np.int32)
+    sel = ora.plan_items(ext, S, items)
+    assert sel["stripe_cnt"].tolist() == list(want.values())
