@@ -132,14 +132,20 @@ def test_invariants_on_synthetic_maps(ora):
         assert ((gd >= 0) & (gd <= 1)).all() and ((gv >= 0) & (gv <= 1)).all()
 
 
-def test_capture_equals_stepwise_and_lists_sorted(ora):
+@pytest.mark.parametrize("scaling,lam,tau", [("row", 0.5, 0.3), ("map", 0.5, 0.05), ("map", 0.25, 0.4)])
+def test_capture_equals_stepwise_and_lists_sorted(ora, scaling, lam, tau):
     maps = inputs.averaged_maps(3, 4, L=96, n_samples=4)
-    dp, do, vp, vo = ora.capture(maps)
+    dp, do, vp, vo = ora.capture(maps, lam=lam, tau=tau, scaling=scaling)
+    differs = False
     for m in range(len(maps)):
-        kd, kv = ora.select(*ora.gamma(ora.true_mask(maps[m])), mu=0.8)
+        kd, kv = ora.select(*ora.gamma(ora.true_mask(maps[m], lam=lam, tau=tau, scaling=scaling)), mu=0.8)
         assert do[dp[m]:dp[m + 1]].tolist() == kd.tolist()
         assert vo[vp[m]:vp[m + 1]].tolist() == kv.tolist()
         assert np.all(np.diff(kd) > 0) and np.all(np.diff(kv) > 0)
+        other = "map" if scaling == "row" else "row"
+        od, ov = ora.select(*ora.gamma(ora.true_mask(maps[m], lam=lam, tau=tau, scaling=other)), mu=0.8)
+        differs |= od.tolist() != kd.tolist() or ov.tolist() != kv.tolist()
+    assert differs  # the two readings keep different lists on these maps
 
 
 def test_planted_patterns_are_recovered(ora):

@@ -125,6 +125,14 @@ PY_MUTANTS = [
      "slot = h * slots + qb * qb // 2 + kb", CASE2),
     ("case 2 plan: bitmap blocks counted from L even when S < L",
      "nL = (min(L, S) + TILE - 1) // TILE", "nL = (L + TILE - 1) // TILE", CASE2),
+    ("wrapper: capture passes mu for tau and tau for mu",
+     "lib().ora_capture(_p(maps), n, Ln, lam, tau, mu, eps,", "lib().ora_capture(_p(maps), n, Ln, lam, mu, tau, eps,",
+     CAP),
+    ("wrapper: true mask passes tau for eps and eps for tau",
+     "lib().ora_true_mask(_p(amap), Ln, lam, eps, tau, _p(M))", "lib().ora_true_mask(_p(amap), Ln, lam, tau, eps, _p(M))",
+     CAP),
+    ("wrapper: capture under per-map scaling scales per row", "mu, eps, SCALINGS[scaling], _p(dp)", "mu, eps, 0, _p(dp)",
+     CAP),
     ("case 2 plan: empty bitmap tiles listed", "                    if not cell.any():\n                        continue\n",
      "", CASE2),
 ]
