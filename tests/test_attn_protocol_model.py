@@ -28,7 +28,11 @@ Checked in every run:
     tile's region-b QK^T (which follows the previous tile's region-b PV), region b for
     the PV of this tile's region a (pv_a).
 The model also shows that releasing a V stage without first observing its fill (the
-rule the issuers follow) breaks the phase invariant for runs of tile-less items.
+rule the issuers follow) breaks the phase invariant for runs of tile-less items, and
+that each of these planted mistakes is caught: the first PV of an item without the
+o_empty wait; a region-b rescale without the pv_a wait; a region-a rescale without
+waiting for the tile's region-b QK^T; a K stage released by a plain arrival instead of
+a commit after its QK^T; a Q tile loaded without the q_empty wait.
 """
 
 import random
@@ -41,10 +45,11 @@ NK, NV, RING = 2, 3, 4
 
 
 class Sim(Engine):
-    def __init__(self, seed, items, release_without_fill=False):
+    def __init__(self, seed, items, release_without_fill=False, broken=""):
         super().__init__(seed)
         self.items = items
         self.release_without_fill = release_without_fill
+        self.broken = broken  # a planted protocol mistake (tests only), or ""
         B = self.barrier
         self.item_full = [B(f"item_full{r}", 1) for r in range(RING)]
         self.item_empty = [B(f"item_empty{r}", 1 + 2) for r in range(RING)]  # Q/V producer + 2 softmax
@@ -178,7 +183,7 @@ def qv_producer(sim):
             for s in sorted(fl):
                 if not fl[s][0]:
                     continue
-                if qn[s] >= 1:
+                if qn[s] >= 1 and sim.broken != "no_q_empty_wait":
                     yield ("wait", sim.q_empty[s], qn[s] - 1)
                 sim.tma(sim.q_full[s], f"Q{s}")
                 qn[s] += 1
@@ -206,7 +211,7 @@ def mma_issuer(sim, s):
                 yield ("wait", sim.v_full[v % NV], v // NV)
             if pend:
                 yield ("wait", sim.p_full[s][h], pcnt)
-                if h == 0 and pfirst and ocnt >= 1:
+                if h == 0 and pfirst and ocnt >= 1 and sim.broken != "no_o_empty_wait":
                     yield ("wait", sim.o_empty[s], ocnt - 1)
             if h == 0:
                 yield ("wait", sim.k_full[u % NK], u // NK)
@@ -249,7 +254,10 @@ def mma_issuer(sim, s):
                 if inn:
                     if fl[s][1]:
                         sim.commit(sim.q_empty[s])
-                    sim.commit(sim.k_empty[u % NK])
+                    if sim.broken == "k_release_by_arrival":
+                        sim.k_empty[u % NK].arrive()
+                    else:
+                        sim.commit(sim.k_empty[u % NK])
                     if fl[s][0]:
                         qcnt += 1
                 elif not end:
@@ -294,8 +302,9 @@ def softmax(sim, s):
                 if j > 0 and sim.rng.random() < 0.2:
                     # O rescale: O must hold exactly the PVs of the regions before this one
                     if h == 0:
-                        yield ("wait", sim.s_full[s][1], tcnt)
-                    else:
+                        if sim.broken != "no_region_b_wait":
+                            yield ("wait", sim.s_full[s][1], tcnt)
+                    elif sim.broken != "no_pv_a_wait":
                         yield ("wait", sim.pv_a[s], tcnt)
                     region = 2 * tcnt + h
                     done = sim.pv_done[s]
@@ -343,3 +352,15 @@ def test_release_without_observed_fill_breaks_phases():
         except ProtocolError:
             broken += 1
     assert broken > 0
+
+
+@pytest.mark.parametrize("broken", ["no_o_empty_wait", "no_pv_a_wait", "no_region_b_wait",
+                                    "k_release_by_arrival", "no_q_empty_wait"])
+def test_planted_protocol_mistakes_are_caught(broken):
+    caught = 0
+    for seed in range(40):
+        try:
+            Sim(seed, _items(seed, 30), broken=broken).run()
+        except ProtocolError:
+            caught += 1
+    assert caught > 0

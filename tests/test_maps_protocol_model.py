@@ -18,8 +18,12 @@ Checked in every run:
   * pass 2 reads the (m_b, 1 / l_b) part 0 wrote for the same item and sample;
   * a part's staging buffer is written only when no store is reading it, and each
     store sends one chunk written by all four warps of the part.
-The model also shows that a single exchange buffer (not double-buffered by sample
-parity) lets a part overwrite its slot before part 0 has read it.
+The model also shows that each of these protocol mistakes is caught: a single exchange
+buffer (not double-buffered by sample parity) lets a part overwrite its slot before
+part 0 has read it; without the stat_ready wait pass 2 reads statistics part 0 has not
+written; without the stg_free wait a part rewrites its staging buffer while the store
+reads it; an s_empty barrier that completes one warp early lets the issuer overwrite an
+S buffer that a warp has not loaded.
 """
 
 import random
@@ -42,15 +46,16 @@ def tile(t, nc, B):
 
 
 class MapsSim(Engine):
-    def __init__(self, seed, items, B, nrb, NS, single_xch=False):
+    def __init__(self, seed, items, B, nrb, NS, single_xch=False, broken=""):
         super().__init__(seed)
         self.items, self.B, self.nrb, self.NS = items, B, nrb, NS
         self.single_xch = single_xch
+        self.broken = broken  # a planted protocol mistake (tests only), or ""
         b_ = self.barrier
         self.full = [b_(f"full{i}", 1) for i in range(NS)]
         self.empty = [b_(f"empty{i}", 1) for i in range(NS)]
         self.s_full = [b_(f"s_full{i}", 1) for i in range(NSB)]
-        self.s_empty = [b_(f"s_empty{i}", NWARP) for i in range(NSB)]
+        self.s_empty = [b_(f"s_empty{i}", NWARP - (broken == "short_s_empty")) for i in range(NSB)]
         self.xch = [b_(f"xch{i}", NWARP) for i in range(2)]
         self.stat_ready = b_("stat_ready", WPP)
         self.stg_full = [b_(f"stg_full{h}", WPP) for h in range(PARTS)]
@@ -112,7 +117,7 @@ def softmax_warp(sim, w):
 
     def put_chunk(chunk):
         nonlocal ne
-        if ne >= 1:
+        if ne >= 1 and sim.broken != "no_stg_free_wait":
             yield ("wait", sim.stg_free[h], ne - 1)
         if sim.stg_reading[h]:
             raise ProtocolError(f"part {h}: staging written while a store reads it")
@@ -120,7 +125,7 @@ def softmax_warp(sim, w):
         sim.stg_full[h].arrive()
         if leader:
             yield ("wait", sim.stg_full[h], ne)
-            got = {sim.staging[(h, k)] for k in range(WPP)}
+            got = {sim.staging.get((h, k)) for k in range(WPP)}
             if got != {chunk}:
                 raise ProtocolError(f"part {h}: store of {chunk} sends {got}")
             sim.stg_reading[h] = True
@@ -136,7 +141,7 @@ def softmax_warp(sim, w):
         for t in range(T):
             pass2, b, c = tile(t, nc, B)
             sb = g % NSB
-            if pass2 and t == nc * B:
+            if pass2 and t == nc * B and sim.broken != "no_stat_ready_wait":
                 yield ("wait", sim.stat_ready, gi)
             yield ("wait", sim.s_full[sb], g // NSB)
             if sim.sbuf[sb] != g:
@@ -199,3 +204,15 @@ def test_single_exchange_buffer_breaks():
         except ProtocolError:
             broken += 1
     assert broken > 0
+
+
+@pytest.mark.parametrize("broken", ["no_stat_ready_wait", "no_stg_free_wait", "short_s_empty"])
+def test_planted_protocol_mistakes_are_caught(broken):
+    caught = 0
+    for seed in range(40):
+        items, B, nrb, NS = _case(seed)
+        try:
+            MapsSim(seed, items, B, nrb, NS, broken=broken).run()
+        except ProtocolError:
+            caught += 1
+    assert caught > 0
