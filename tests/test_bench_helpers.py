@@ -63,3 +63,13 @@ def test_profiled_traffic_follows_the_source_hash(tmp_path, monkeypatch):
 def test_committed_traffic_record_is_current():
     # the record in profiles/ was taken on the attention sources as committed
     assert bench.profiled_traffic("llama3-8b-layer-64k") is not None
+
+
+def test_peaks_measured_else_the_stated_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.load_peaks() == (6650.0, 1590.0, 1400.0, "fallback")
+    assert bench.sm_max_mhz() == 1965.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(
+        {"hbm_gbs": 6545.9, "bf16_tflops": 1667.7, "bf16_tflops_sustained": 1368.0, "sm_max_mhz": 1950.0}))
+    assert bench.load_peaks() == (6545.9, 1667.7, 1368.0, "measured")
+    assert bench.sm_max_mhz() == 1950.0
