@@ -45,7 +45,8 @@ extern "C" {
 
 #define SSA_OK 0
 #define SSA_ERR_INVALID (-1)     /* null pointer, bad size, unsorted/duplicate/negative list, bad map entry */
-#define SSA_ERR_UNSUPPORTED (-2) /* head dim not 64/128, lambda not 0.5/1, L > 1024 */
+#define SSA_ERR_UNSUPPORTED (-2) /* head dim not 64/128, capture L > 1024, Case-2 plan given to decoding,
+                                    a kernel build or device ordinal the library cannot use */
 #define SSA_ERR_CAPACITY (-3)    /* caller buffer or workspace too small */
 #define SSA_ERR_CUDA (-4)        /* a CUDA runtime/driver call failed */
 #define SSA_ERR_TIMEOUT (-5)     /* a bounded on-device wait expired */
