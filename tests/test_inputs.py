@@ -96,3 +96,17 @@ def test_csr_round_trip():
     assert ptr.tolist() == [0, 3, 3, 4] and vals.tolist() == [0, 3, 9, 5]
     back = inputs.from_csr(ptr, vals)
     assert all(np.array_equal(a, b) for a, b in zip(lists, back))
+
+
+def test_qk_samples_plant_what_capture_recovers(ora):
+    # the maps workload's rows (L = 512, 16 samples, d = 64): the oracle's averaged maps,
+    # captured at the pages' setting, keep every planted column and the main diagonal
+    n, B, L, d = 4, 16, 512, 64
+    q, k = inputs.qk_samples(inputs.SEED_BASE + 1, n, B, L=L, d=d)
+    assert q.shape == k.shape == (n, B, L, d)
+    maps = ora.attn_maps(q, k, d ** -0.5).astype(np.float32)
+    dp, do, vp, vc = ora.capture(maps)
+    planted = inputs.planted_map_patterns(inputs.SEED_BASE + 1, n, L)
+    for m in range(n):
+        assert 0 in do[dp[m]:dp[m + 1]].tolist()
+        assert set(planted[m][1].tolist()) <= set(vc[vp[m]:vp[m + 1]].tolist())
