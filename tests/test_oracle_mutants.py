@@ -112,6 +112,17 @@ MUTANTS = [
     ("attention: an explicit GQA map ignored", "return kv_map ? kv_map[h] : h / (Hq / Hkv);",
      "return h / (Hq / Hkv);", ATTN),
     ("attention: LSE without the row max", "*lse = m + log(l);", "*lse = log(l);", ATTN),
+    ("select: the one-cell diagonal r = L - 1 never considered",
+     "    for (int r = 0; r < L; ++r)\n        if (gamma_diag[r] >= mu)",
+     "    for (int r = 0; r < L - 1; ++r)\n        if (gamma_diag[r] >= mu)", CAP),
+    ("select: the one-cell column c = L - 1 never considered",
+     "    for (int c = 0; c < L; ++c)\n        if (gamma_vert[c] >= mu)",
+     "    for (int c = 0; c < L - 1; ++c)\n        if (gamma_vert[c] >= mu)", CAP),
+    ("gamma: a diagonal's first cell skipped", "for (int i = r; i < L; ++i) {", "for (int i = r + 1; i < L; ++i) {", CAP),
+    ("maps: the diagonal entry left out of the mean", "for (int j = 0; j <= i; ++j) row[j] += s[j] / sum / B;",
+     "for (int j = 0; j < i; ++j) row[j] += s[j] / sum / B;", MAPS),
+    ("attention: keys taken for values", "const uint16_t *vj = V + (size_t)J[a] * d;",
+     "const uint16_t *vj = K + (size_t)J[a] * d;", ATTN),
     ("gamma: column denominator off by one", "gamma_vert[c] = (double)num / (double)den;",
      "gamma_vert[c] = (double)num / (double)(den + 1);", CAP),
 ]
