@@ -130,3 +130,12 @@ def test_binding_rejects_host_tensors_before_any_call(lib):
     with pytest.raises(binding.SSAError) as e:
         binding.refill(object(), *(torch.zeros(2, dtype=torch.int32) for _ in range(4)))
     assert e.value.code == -1 and "CUDA" in str(e.value)
+
+
+def test_oracle_shares_no_code_with_the_library():
+    # the oracle includes only the C standard library and imports nothing of the package
+    src = open(os.path.join(ROOT, "oracle", "ssa_oracle.c")).read()
+    assert set(re.findall(r"#include\s*<([^>]+)>", src)) <= {"math.h", "stdint.h", "stdlib.h", "string.h"}
+    assert not re.search(r'#include\s*"', src)
+    py = open(os.path.join(ROOT, "oracle", "oracle.py")).read()
+    assert not re.search(r"structured_sparse_attention_b200|libssa\.so|import\s+ssa\b", py)
