@@ -1,5 +1,5 @@
-"""Every source, test, profile or fixture file that README.md name in
-backticks exists in the repository (a renamed or removed file shows up here)."""
+"""Every source, test, profile or fixture file that the repository's design notes and
+readme name in backticks exists (a renamed or removed file shows up here)."""
 
 import os
 import re
@@ -22,4 +22,4 @@ def test_named_files_exist(doc):
         names = [ref, os.path.join("structured_sparse_attention_b200", ref)]
         if not any(os.path.exists(os.path.join(ROOT, d, n)) for d in SEARCH for n in names):
             missing.append(ref)
-    assert not missing, f"{doc} names files that do not exist: {missing}"
+    assert not missing, f"{doc}: named files that do not exist: {missing}"
