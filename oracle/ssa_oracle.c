@@ -16,7 +16,7 @@
  *   - "Circularity Check", step 2 and the Referee Report summary: the mask is applied
  *     to QK^T / sqrt(d_k) before softmax.
  *   - Referee Report, minor comment 1: the stabiliser eps (1e-8 in the main text).
- * Readings where the page is silent (all listed in the design notes): row-wise
+ * Readings where the page is silent: row-wise
  * min-max scaling of the Box-Cox output before tau (map-wise as an option); t >= tau
  * and gamma >= mu; a constant row (or map) counts as t = 1; masked logits are excluded from the softmax (-inf),
  * not multiplied by 0; an empty row gives O = 0 and LSE = -inf; LSE is the natural

@@ -1,5 +1,5 @@
-"""Every source, test, profile or fixture file that the repository's design notes and
-readme name in backticks exists (a renamed or removed file shows up here)."""
+"""Every source, test, profile or fixture file named in backticks by the repository's
+top-level documents exists (a renamed or removed file shows up here)."""
 
 import os
 import re
